@@ -1,0 +1,20 @@
+"""Exact, IO-aware attention for B200 (sm_100a).
+
+The compute lives in ``libfa_sm100.so`` (hand-written CUDA, C ABI declared in
+``include/fa.h``); ``binding`` marshals torch tensors into that ABI.  Importing
+the package does not load the library; the first use of an entry point does,
+and fails loudly if the library is missing -- there is no fallback path.
+"""
+
+_BINDING_NAMES = ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_dropout_mask", "fa_last_device_error",
+                  "FAError", "load_library")
+
+
+def __getattr__(name):
+    if name in _BINDING_NAMES:
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)
+
+
+__all__ = list(_BINDING_NAMES)

@@ -1,0 +1,201 @@
+// fa_api.cu -- the C ABI (include/fa.h): argument validation, TMA descriptor
+// encoding, and launches on the caller's stream.  Validation happens before any
+// CUDA call, so a rejected call enqueues nothing and touches no output.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+// Device word that bounded device waits set when they give up (one per device,
+// in this module's static device memory).
+__device__ unsigned g_fa_error_word;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, d] bf16 row-major, boxes of 64 columns x 128 rows, 128-byte swizzle.
+bool encode_rows_map(CUtensorMap* tm, const void* base, long long rows, int d) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+unsigned* error_word_ptr() {
+  static unsigned* cache[128] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  if (dev < 128 && cache[dev]) return cache[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return nullptr;
+  if (dev < 128) cache[dev] = static_cast<unsigned*>(p);
+  return static_cast<unsigned*>(p);
+}
+
+bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shared validation of sizes / scalars.  Returns FA_OK or the error.
+fa_status check_common(int B, int H, int N, int d, float scale, float p_drop) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+uint32_t drop_threshold(float p_drop) {
+  // round-half-even(p * 65536) in double precision (default rounding mode)
+  return static_cast<uint32_t>(nearbyint(static_cast<double>(p_drop) * 65536.0));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: valid but unsupported configuration";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                 int causal, float scale, float p_drop, uint64_t seed, void* stream) {
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(LSE, 16))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, p_drop);
+  if (st != FA_OK) return st;
+
+  fa::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (!encode_rows_map(&a.tmQ, Q, rows, d) || !encode_rows_map(&a.tmK, K, rows, d) ||
+      !encode_rows_map(&a.tmV, V, rows, d))
+    return FA_ERR_CUDA;
+  a.O = O;
+  a.LSE = LSE;
+  a.err = error_word_ptr();
+  if (!a.err) return FA_ERR_CUDA;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.drop_t = drop_threshold(p_drop);
+  a.drop_scale = a.drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
+  a.seed_lo = static_cast<uint32_t>(seed);
+  a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  return fa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                 void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                 uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
+      misaligned(LSE, 16) || misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16) ||
+      misaligned(workspace, 256))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, p_drop);
+  if (st != FA_OK) return st;
+  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+
+  fa::BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (!encode_rows_map(&a.tmQ, Q, rows, d) || !encode_rows_map(&a.tmK, K, rows, d) ||
+      !encode_rows_map(&a.tmV, V, rows, d) || !encode_rows_map(&a.tmDO, dO, rows, d))
+    return FA_ERR_CUDA;
+  a.O = O;
+  a.dO = dO;
+  a.LSE = LSE;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  a.dQacc = static_cast<float*>(workspace);
+  a.Dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    round_up(static_cast<size_t>(rows) * d * sizeof(float), 256));
+  a.err = error_word_ptr();
+  if (!a.err) return FA_ERR_CUDA;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.drop_t = drop_threshold(p_drop);
+  a.drop_scale = a.drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
+  a.seed_lo = static_cast<uint32_t>(seed);
+  a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  return fa::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed, void* stream) {
+  if (!mask) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H * N >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return fa::launch_dropout_mask(mask, B, H, N, drop_threshold(p_drop), static_cast<uint32_t>(seed),
+                                 static_cast<uint32_t>(seed >> 32), static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+fa_status fa_last_device_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_error_word, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

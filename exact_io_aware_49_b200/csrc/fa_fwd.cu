@@ -1,0 +1,440 @@
+// fa_fwd.cu -- fused attention forward for sm_100a.
+//
+// What it computes: O = dropout(softmax(scale * Q K^T + causal mask)) V and
+// LSE_i = ln sum_j exp(scale * Q_i . K_j), tile by tile, never writing the
+// N x N scores or probabilities to device memory ("FlashAttention" glossary,
+// Tiling; "Flash Attention" glossary, How Flash Attention Works, steps 1-5).
+// The row statistics follow the online-softmax recurrence of "DL0056
+// FlashAttention", Mathematical Formulation: a running maximum m_i and
+// denominator l_i, with exp(m_old - m_new) rescaling the earlier partial sums
+// of l and of the output accumulator.
+//
+// Design (B200):
+//  * one CTA owns two 128-row query tiles (Q0, Q1) of one (b, h) and streams
+//    128-key K/V tiles through a multi-stage TMA + mbarrier ring;
+//  * S_q = Q_q K_t^T and O_q += P_q V_t run on the 5th-generation tensor cores
+//    (tcgen05.mma, bf16 in, fp32 accumulators in tensor memory).  TMEM holds
+//    S0 | S1 | O0 | O1 (512 columns); P_q (bf16) is written back over S_q and
+//    read by the PV MMA directly from TMEM;
+//  * warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q0 and Q1
+//    (one thread per query row: causal mask on the diagonal tile, running
+//    max / sum, exp2, Philox dropout, P to TMEM, and the epilogue); warp 8
+//    issues the MMAs; warp 9 issues the TMA loads.  While one warpgroup turns
+//    S into P, the tensor core works on the other query tile;
+//  * the O rescale is lazy: the stale maximum is kept until a row's maximum
+//    grows by more than 8 (log2 units).  l and O share the stale maximum, so
+//    the result is unchanged; P stays <= 2^8;
+//  * dropout never stores a mask: keep bits come from Philox keyed on
+//    (seed, b, h, i, j); kept P are left unscaled and 1/(1-p) is folded into
+//    the final normalisation.
+//  * a causal CTA processes only key tiles up to its diagonal; the grid puts
+//    the heaviest query blocks first.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "fa_internal.h"
+#include "philox.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kBM = 128;             // query rows per tile
+constexpr int kBN = 128;             // keys per tile
+constexpr int kFwdThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+// Register split (setmaxnreg): the kernel launches with kFwdLaunchRegs per
+// thread; softmax warpgroups grow to kSoftmaxRegs, the control warpgroup
+// (MMA, TMA, two idle warps) shrinks to kControlRegs.  The split must fit the
+// launch pool: 2*128*216 + 128*56 = 62464 <= 384*168 = 64512.
+constexpr int kFwdLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 56;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kFwdThreads * kFwdLaunchRegs, "register split");
+constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold, log2 units
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kTileBytes = kBN * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kBoxBytes = 128 * 128;     // one 128-row x 64-col box (128B rows)
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  // barriers: q, kfull[S], vfull[S], kvempty[S], s_ready[2], p_ready[2], o_ready[2], drain
+  static constexpr int kNumBars = 1 + 3 * kStages + 7;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot (4 B) + abort flag (4 B)
+  static constexpr int kBytes = kMisc + 16 + 1024;   // + slack for 1024-byte alignment
+};
+
+struct FwdBars {
+  uint64_t* q;
+  uint64_t* kfull;
+  uint64_t* vfull;
+  uint64_t* kvempty;
+  uint64_t* s_ready;
+  uint64_t* p_ready;
+  uint64_t* o_ready;
+  uint64_t* drain;
+};
+
+template <int D>
+__device__ __forceinline__ FwdBars fwd_bars(uint8_t* smem) {
+  using L = FwdSmem<D>;
+  uint64_t* b = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  FwdBars r;
+  r.q = b;
+  r.kfull = b + 1;
+  r.vfull = b + 1 + L::kStages;
+  r.kvempty = b + 1 + 2 * L::kStages;
+  r.s_ready = b + 1 + 3 * L::kStages;
+  r.p_ready = r.s_ready + 2;
+  r.o_ready = r.s_ready + 4;
+  r.drain = r.s_ready + 6;
+  return r;
+}
+
+struct FwdParams {
+  __nv_bfloat16* O;
+  float* LSE;
+  unsigned* err;
+  int H, N;
+  float scale_log2;
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
+};
+
+// S_q = Q_q * K^T : M = 128 query rows, N = 128 keys, K = D (both K-major).
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * FwdSmem<D>::kBoxBytes + (kk % 4) * 32;
+    mma_ss(tmem_s, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+  }
+}
+
+// O_q (+)= P_q * V : M = 128, N = D, K = 128 keys.  P (bf16, packed in pairs)
+// lives in TMEM over S_q; V is MN-major in shared memory (D contiguous).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    const uint64_t bdesc = sdesc_sw128(v_smem + kk * 2048, FwdSmem<D>::kBoxBytes, 1024);
+    mma_ts(tmem_o, tmem_p + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// All 384 threads meet here once their role is done; the MMA warp then frees TMEM.
+__device__ __forceinline__ void cta_teardown(uint32_t tmem, bool dealloc) {
+  tc_fence_before();
+  asm volatile("bar.sync 1, %0;" ::"n"(kFwdThreads) : "memory");
+  tc_fence_after();
+  if (dealloc) tmem_dealloc(tmem, 512);
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdSmem<D>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const FwdBars bar = fwd_bars<D>(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;  // b * H + h
+  const int N = p.N;
+  const int n_qt = N / kBM;
+  const int qb = CAUSAL ? (gridDim.y - 1 - blockIdx.y) : blockIdx.y;
+  const int qt0 = 2 * qb;
+  const int nq = min(2, n_qt - qt0);
+  // key tiles each query tile visits (causal: up to and including its diagonal)
+  int ntile[2];
+  ntile[0] = CAUSAL ? qt0 + 1 : n_qt;
+  ntile[1] = (nq == 2) ? (CAUSAL ? qt0 + 2 : n_qt) : 0;
+  const int nt_all = ntile[nq - 1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar.q, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bar.kfull[s], 1);
+      mbar_init(&bar.vfull[s], 1);
+      mbar_init(&bar.kvempty[s], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&bar.s_ready[q], 1);
+      mbar_init(&bar.p_ready[q], 4);
+      mbar_init(&bar.o_ready[q], 1);
+    }
+    mbar_init(bar.drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sm_q = smem_u32(smem + L::kQ);
+  const uint32_t sm_k = smem_u32(smem + L::kK);
+  const uint32_t sm_v = smem_u32(smem + L::kV);
+
+  if (warp >= 8) {
+    // control warpgroup: MMA issuer, TMA producer, two idle warps
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+    if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int row0 = bh * N;
+      mbar_expect_tx(bar.q, nq * L::kTileBytes);
+      for (int q = 0; q < nq; ++q)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(smem + L::kQ + q * L::kTileBytes + c * L::kBoxBytes, &tmQ, c * 64, row0 + (qt0 + q) * kBM,
+                      bar.q);
+      int issued = 0;
+      for (int t = 0; t < nt_all; ++t) {
+        const int s = t % S;
+        if (t >= S && !mbar_wait(&bar.kvempty[s], ((t / S) - 1) & 1, abort_flag, p.err)) break;
+        mbar_expect_tx(&bar.kfull[s], L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(smem + L::kK + s * L::kTileBytes + c * L::kBoxBytes, &tmK, c * 64, row0 + t * kBN,
+                      &bar.kfull[s]);
+        mbar_expect_tx(&bar.vfull[s], L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(smem + L::kV + s * L::kTileBytes + c * L::kBoxBytes, &tmV, c * 64, row0 + t * kBN,
+                      &bar.vfull[s]);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA's shared memory goes away
+        mbar_wait_drain(bar.q, 0);
+        for (int t = max(0, issued - S); t < issued; ++t) {
+          mbar_wait_drain(&bar.kfull[t % S], (t / S) & 1);
+          mbar_wait_drain(&bar.vfull[t % S], (t / S) & 1);
+        }
+      }
+    }
+    } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar.q, 0, abort_flag, p.err) && mbar_wait(&bar.kfull[0], 0, abort_flag, p.err);
+      if (ok) {
+        tc_fence_after();
+        for (int q = 0; q < nq; ++q) {
+          issue_qk<D>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k);
+          mma_commit(&bar.s_ready[q]);
+        }
+      }
+      for (int t = 0; ok && t < nt_all; ++t) {
+        const int s = t % S;
+        if (!mbar_wait(&bar.vfull[s], (t / S) & 1, abort_flag, p.err)) { ok = false; break; }
+        bool next_k_ready = false;
+        const int s1 = (t + 1) % S;
+        for (int q = 0; q < nq; ++q) {
+          if (t >= ntile[q]) continue;
+          if (!mbar_wait(&bar.p_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D>(tmem + 256 + q * D, tmem + q * 128, sm_v + s * L::kTileBytes, t > 0);
+          if (t == ntile[q] - 1) {
+            mma_commit(&bar.o_ready[q]);
+          } else {
+            if (!next_k_ready) {
+              if (!mbar_wait(&bar.kfull[s1], ((t + 1) / S) & 1, abort_flag, p.err)) { ok = false; break; }
+              tc_fence_after();
+              next_k_ready = true;
+            }
+            issue_qk<D>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k + s1 * L::kTileBytes);
+            mma_commit(&bar.s_ready[q]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bar.kvempty[s]);
+      }
+      if (!ok) {
+        mma_commit(bar.drain);  // wait for MMAs already issued before TMEM is freed
+        mbar_wait_drain(bar.drain, 0);
+      }
+    }
+    __syncwarp();
+    }
+    cta_teardown(tmem, warp == kMmaWarp);
+    return;
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    const int q = warp >> 2;
+    if (q < nq) {
+      const int wq = warp & 3;
+      const int r = wq * 32 + lane;  // row within the query tile == TMEM lane
+      const int i = (qt0 + q) * kBM + r;
+      const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+      const uint32_t t_s = t_lane + q * 128;
+      const uint32_t t_o = t_lane + 256 + q * D;
+      const float sl2 = p.scale_log2;
+      const DropConst dk = make_drop_const(p.drop_t);
+      const int h = bh % p.H;
+      const int b = bh / p.H;
+      float m = -CUDART_INF_F;  // running max of scale*log2(e)*S, possibly stale
+      float l = 0.f;            // running sum of exp2(x - m)
+      bool ok = true;
+      for (int t = 0; t < ntile[q]; ++t) {
+        if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, sr + c * 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence32(sr + c * 32);
+        float s[kBN];
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+        if (CAUSAL && t == ntile[q] - 1) {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c)
+            if (c > r) s[c] = -CUDART_INF_F;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < kBN; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const float m_new = fmaxf(m, m_tile);
+        if (__any_sync(0xffffffffu, m_new > m + kRescaleTau)) {
+          const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
+          l *= alpha;
+          if (t > 0) {
+            // O accumulator of this row: all earlier PV MMAs completed before S_t was committed
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orow[32];
+              tmem_ld32(t_o + c * 32, orow);
+              tmem_ld_wait();
+              reg_fence32(orow);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+              tmem_st32(t_o + c * 32, orow);
+            }
+          }
+          m = m_new;
+        }
+        const float neg_m = -m;
+        uint32_t pk[64];
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += rs0 + rs1;
+        if (DROPOUT) {
+#pragma unroll
+          for (int g = 0; g < kBN / 8; ++g) {
+            uint32_t w[4];
+            philox4x32_10(static_cast<uint32_t>(t * (kBN / 8) + g), static_cast<uint32_t>(i),
+                          static_cast<uint32_t>(h), static_cast<uint32_t>(b), p.seed_lo, p.seed_hi, w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pk[g * 4 + e] &= keep_mask_2x16(w[e], dk);
+          }
+        }
+        tmem_st32(t_s, pk);
+        tmem_st32(t_s + 32, pk + 32);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.p_ready[q]);
+      }
+      if (ok && mbar_wait(&bar.o_ready[q], 0, abort_flag, p.err)) {
+        // ---------------------------------------------------------- epilogue
+        tc_fence_after();
+        const float inv = p.drop_scale / l;
+        __nv_bfloat16* orow_g = p.O + (static_cast<size_t>(bh) * N + i) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_ld_wait();
+          reg_fence32(o);
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            packed[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+        p.LSE[static_cast<size_t>(bh) * N + i] = (m + lg2_approx(l)) * 0.69314718055994531f;
+      }
+    }
+    cta_teardown(tmem, false);
+  }
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
+  auto kern = fa_fwd_kernel<D, CAUSAL, DROPOUT>;
+  const int smem = FwdSmem<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg.inc only succeeds if the launch reserved the pool the split assumes
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
+  FwdParams p;
+  p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.LSE = a.LSE;
+  p.err = a.err;
+  p.H = a.H;
+  p.N = a.N;
+  p.scale_log2 = a.scale_log2;
+  p.drop_t = a.drop_t;
+  p.drop_scale = a.drop_scale;
+  p.seed_lo = a.seed_lo;
+  p.seed_hi = a.seed_hi;
+  const int n_qt = a.N / kBM;
+  dim3 grid(a.B * a.H, (n_qt + 1) / 2);
+  kern<<<grid, kFwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream) {
+  const bool drop = a.drop_t != 0;
+  if (a.d == 64) {
+    if (a.causal) return drop ? launch_fwd_t<64, true, true>(a, stream) : launch_fwd_t<64, true, false>(a, stream);
+    return drop ? launch_fwd_t<64, false, true>(a, stream) : launch_fwd_t<64, false, false>(a, stream);
+  }
+  if (a.causal) return drop ? launch_fwd_t<128, true, true>(a, stream) : launch_fwd_t<128, true, false>(a, stream);
+  return drop ? launch_fwd_t<128, false, true>(a, stream) : launch_fwd_t<128, false, false>(a, stream);
+}
+
+}  // namespace fa

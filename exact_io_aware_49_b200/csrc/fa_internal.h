@@ -1,0 +1,49 @@
+// fa_internal.h -- launch interfaces between the C-ABI shim and the kernel
+// translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+struct FwdArgs {
+  CUtensorMap tmQ, tmK, tmV;  // 2-D maps over [B*H*N, d] bf16, 64 x 128 boxes, 128B swizzle
+  void* O;                    // bf16 [B, H, N, d]
+  float* LSE;                 // fp32 [B, H, N]
+  unsigned* err;              // device error word
+  int B, H, N, d;
+  int causal;
+  float scale_log2;   // scale * log2(e)
+  uint32_t drop_t;    // keep <=> u16 >= drop_t (0: no dropout)
+  float drop_scale;   // 1 / (1 - p)
+  uint32_t seed_lo, seed_hi;
+};
+
+struct BwdArgs {
+  CUtensorMap tmQ, tmK, tmV, tmDO;  // same layout as the forward maps
+  const void* O;
+  const void* dO;
+  const float* LSE;
+  void* dQ;
+  void* dK;
+  void* dV;
+  float* dQacc;  // fp32 [B, H, N, d] workspace
+  float* Dvec;   // fp32 [B, H, N] workspace
+  unsigned* err;
+  int B, H, N, d;
+  int causal;
+  float scale;
+  float scale_log2;
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
+};
+
+cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_dropout_mask(uint8_t* mask, int B, int H, int N, uint32_t drop_t, uint32_t seed_lo,
+                                uint32_t seed_hi, cudaStream_t stream);
+
+}  // namespace fa

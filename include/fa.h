@@ -1,0 +1,138 @@
+/*
+ * fa.h -- C ABI of the exact, IO-aware attention library for B200 (sm_100a).
+ *
+ * The library computes exact scaled dot-product attention
+ *     O = softmax(scale * Q K^T + causal mask) V
+ * with optional attention dropout, tile by tile with the online-softmax
+ * recurrence (running row maximum m_i and denominator l_i, earlier partial
+ * sums rescaled when the maximum changes), without ever writing the N x N
+ * score or probability matrix to device memory.
+ *   - definition of the result: "Flash Attention" glossary (emergent.sh),
+ *     section "Why Regular Attention Becomes a Bottleneck"; exactness:
+ *     "DL0056 FlashAttention", Answer;
+ *   - the recurrence: "DL0056 FlashAttention", Mathematical Formulation;
+ *   - tiling / fusion: "FlashAttention" glossary (inferensys.com), Tiling and
+ *     Kernel Optimization; "Flash Attention" glossary, How Flash Attention
+ *     Works, steps 1-5;
+ *   - backward by recomputation from stored per-row outputs: "FlashAttention"
+ *     glossary, Recomputation; "Flash Attention" glossary, step 6;
+ *   - causal mask and dropout inside the fused kernel: "FlashAttention"
+ *     glossary, Causal Masking and Dropout bullets; the dropout pattern is
+ *     regenerated, not stored: "Flash Attention" glossary, Key Components.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are dense, row-major [B, H, N, d] (strides H*N*d, N*d, d, 1) with
+ *    elements of type bf16 (IEEE bfloat16, passed as void*).  Per-row
+ *    statistics (LSE) are fp32 [B, H, N].
+ *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
+ *    aligned.  The library allocates nothing and keeps no per-call state.
+ *  - Supported: d in {64, 128}; N a positive multiple of 128; B*H*N < 2^31.
+ *  - ``stream`` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call only enqueues work on it and returns; results are
+ *    ready when the stream reaches that point.
+ *  - Argument errors are detected on the host before anything is enqueued:
+ *    nothing is launched and no output is touched.  A failed launch returns
+ *    FA_ERR_CUDA.  No entry point exits or aborts the process.
+ *  - Device-side pipeline waits are bounded in time.  A wait that gives up
+ *    records a flag in a device word and makes the kernel return early; the
+ *    outputs of that call are then undefined and fa_last_device_error()
+ *    reports FA_ERR_TIMEOUT.
+ *  - LSE_i = m_i + ln(l_i) in natural-log units of the scaled scores:
+ *    LSE_i = ln(sum_j exp(scale * Q_i . K_j)) over the unmasked j.  Dropout
+ *    does not change it.
+ *  - Dropout: keep(i, j) <=> u16(seed, b, h, i, j) >= t with
+ *    t = round-half-even(p_drop * 65536); u16 comes from Philox4x32-10
+ *    (Salmon et al., SC'11) with key (seed mod 2^32, seed >> 32), counter
+ *    (j >> 3, i, h, b); key j takes 16 bits of output word (j >> 1) & 3, the
+ *    low half for even j and the high half for odd j.  Kept probabilities are
+ *    scaled by 1/(1 - p_drop).  p_drop = 0 disables dropout.
+ */
+#ifndef FA_SM100_H_
+#define FA_SM100_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, p_drop outside [0,1), ... */
+  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d not in {64,128}, N % 128 != 0, too large */
+  FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor-map encoding, ...) */
+  FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by fa_last_device_error) */
+} fa_status;
+
+/*
+ * Forward pass.
+ *   Q, K, V : in,  bf16 [B, H, N, d]
+ *   O       : out, bf16 [B, H, N, d]   O = dropout(softmax(scale*QK^T + mask)) V
+ *   LSE     : out, fp32 [B, H, N]      per-row log-sum-exp of the scaled scores
+ *   causal  : nonzero -> key j > query i is masked (square, top-left aligned)
+ *   scale   : finite score scale, usually 1/sqrt(d)
+ *   p_drop  : dropout probability in [0, 1); seed keys the dropout mask
+ * Source: the tiled forward ("FlashAttention" glossary, Tiling; "DL0056
+ * FlashAttention", Mathematical Formulation; "Flash Attention" glossary, steps
+ * 1-5).  O and LSE may not alias the inputs.
+ */
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                 int B, int H, int N, int d, int causal, float scale,
+                 float p_drop, uint64_t seed, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
+ * accumulator [B, H, N, d] plus the fp32 row statistic D [B, H, N], each
+ * rounded up to 256 bytes.  Linear in N ("FlashAttention" glossary: memory
+ * drops from O(N^2) to O(N)).  Returns 0 for non-positive sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass by recomputation ("FlashAttention" glossary, Recomputation;
+ * "Flash Attention" glossary, step 6 and Key Components on regenerating the
+ * dropout pattern).
+ *   Q, K, V, O, dO : in, bf16 [B, H, N, d]  (O from fa_fwd on the same inputs)
+ *   LSE            : in, fp32 [B, H, N]     (from fa_fwd)
+ *   dQ, dK, dV     : out, bf16 [B, H, N, d] gradients of sum(dO * O)
+ *   workspace      : device scratch of at least fa_bwd_workspace_size() bytes,
+ *                    256-byte aligned, owned by the caller, contents on entry
+ *                    ignored; it may be reused once the stream has passed
+ *                    this call.
+ * causal, scale, p_drop and seed must equal the values given to fa_fwd; the
+ * library cannot check this.  Steps: D_i = sum_c dO_ic O_ic and zeroing of
+ * the dQ accumulator; one pass over key tiles recomputing P from LSE and
+ * producing dK, dV and fp32 atomic contributions to dQ; conversion of dQ to
+ * bf16.
+ */
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV,
+                 int B, int H, int N, int d, int causal, float scale,
+                 float p_drop, uint64_t seed, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/*
+ * Test/inspection export: writes the dropout keep mask Z (1 = kept, 0 =
+ * dropped) as uint8 [B, H, N, N] into device memory ``mask`` with the same
+ * device Philox code the kernels use.  N here only needs to be positive.
+ */
+fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed,
+                          void* stream);
+
+/*
+ * Synchronises the device, then reads and clears the device error word that
+ * bounded waits set.  FA_OK when no wait gave up since the last call,
+ * FA_ERR_TIMEOUT otherwise, FA_ERR_CUDA if the device could not be read.
+ */
+fa_status fa_last_device_error(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H_ */

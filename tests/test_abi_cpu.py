@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI (no GPU): the library builds and loads, exports
+every entry point include/*.h declares, and rejects bad arguments before it
+makes any CUDA call.  Every call here carries at least one invalid argument,
+so nothing is ever launched."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_49_b200 import build, binding
+    build.build()
+    return binding.load_library()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        for m in re.finditer(r"\b(fa_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = _declared_functions()
+    for want in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_dropout_mask", "fa_last_device_error",
+                 "fa_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, prefix in [(0, b"FA_OK"), (1, b"FA_ERR_INVALID_ARG"), (2, b"FA_ERR_UNSUPPORTED"),
+                         (3, b"FA_ERR_CUDA"), (4, b"FA_ERR_TIMEOUT")]:
+        assert lib.fa_status_string(code).startswith(prefix)
+    assert lib.fa_status_string(99) == b"unknown fa_status"
+
+
+A = 0x10000  # a 16-byte-aligned fake address; calls below never get past validation
+
+
+def _fwd(lib, Q=A, K=A, V=A, O=A, L=A, B=1, H=1, N=128, d=64, causal=0, scale=0.125, p=0.0):
+    return lib.fa_fwd(Q, K, V, O, L, B, H, N, d, causal, scale, p, 0, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(Q=0), 1), (dict(K=0), 1), (dict(V=0), 1), (dict(O=0), 1), (dict(L=0), 1),
+    (dict(Q=A + 8), 1), (dict(O=A + 4), 1), (dict(L=A + 4), 1),
+    (dict(B=0), 1), (dict(H=-1), 1), (dict(N=0), 1), (dict(d=0), 1),
+    (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
+    (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("inf")), 1),
+    (dict(d=32), 2), (dict(d=96), 2), (dict(N=100), 2), (dict(N=129), 2),
+    (dict(B=1 << 16, H=1 << 8, N=1 << 7), 2),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, want):
+    assert _fwd(lib, **kw) == want
+
+
+def _bwd(lib, ws=A, ws_bytes=None, B=1, H=1, N=128, d=64, p=0.0, **ptrs):
+    names = ["Q", "K", "V", "O", "dO", "L", "dQ", "dK", "dV"]
+    vals = [ptrs.get(n, A) for n in names]
+    if ws_bytes is None:
+        ws_bytes = lib.fa_bwd_workspace_size(B, H, N, d)
+    return lib.fa_bwd(*vals, B, H, N, d, 1, 0.125, p, 0, ws, ws_bytes, None)
+
+
+def test_workspace_size_is_linear_in_n(lib):
+    s1 = lib.fa_bwd_workspace_size(2, 3, 1024, 128)
+    s2 = lib.fa_bwd_workspace_size(2, 3, 2048, 128)
+    assert s1 == 2 * 3 * 1024 * 128 * 4 + 2 * 3 * 1024 * 4
+    assert s2 == 2 * s1
+    assert lib.fa_bwd_workspace_size(0, 1, 128, 64) == 0
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(ws=0), 1), (dict(ws=A + 16), 1), (dict(dQ=0), 1), (dict(dO=A + 2), 1), (dict(L=0), 1),
+    (dict(ws_bytes=1000), 1), (dict(p=1.5), 1), (dict(d=256), 2), (dict(N=64), 2),
+])
+def test_bwd_rejects_bad_arguments(lib, kw, want):
+    assert _bwd(lib, **kw) == want
+
+
+def test_mask_rejects_bad_arguments(lib):
+    assert lib.fa_dropout_mask(None, 1, 1, 8, 0.1, 0, None) == 1
+    assert lib.fa_dropout_mask(A, 0, 1, 8, 0.1, 0, None) == 1
+    assert lib.fa_dropout_mask(A, 1, 1, 8, 1.0, 0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from exact_io_aware_49_b200 import binding
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(ImportError):
+        binding.load_library(str(tmp_path / "missing.so"))

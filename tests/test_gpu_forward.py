@@ -1,0 +1,114 @@
+"""GPU parity of fa_fwd against the fp64 oracle (called through the C ABI).
+
+Small workloads are compared element by element on every head; the large ones
+run at full size in the benchmark's launch configuration and are compared on
+whole heads (N = 4096) or on seeded query-row samples (N >= 16384), where each
+sampled row needs only its own row of scores in the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_49_b200 import workloads as wl
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, causal, scale, p, seed):
+    from exact_io_aware_49_b200 import fa_fwd
+    o, lse = fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal, scale, p, seed)
+    torch.cuda.synchronize()
+    return o.cpu(), lse.cpu()
+
+
+def _compare_heads(q, k, v, o, lse, heads, causal, scale, p, seed, rows_by_head=None):
+    for b, h in heads:
+        rows = None if rows_by_head is None else rows_by_head[(b, h)]
+        want_o, want_l = pu.oracle_fwd_head(q, k, v, b, h, causal, scale, p, seed, rows)
+        got_o = pu.f64(o[b, h]) if rows is None else pu.f64(o[b, h])[rows]
+        got_l = pu.f64(lse[b, h]) if rows is None else pu.f64(lse[b, h])[rows]
+        pu.check_o(got_o, want_o, f"head {(b, h)}")
+        pu.check_lse(got_l, want_l, f"head {(b, h)}")
+
+
+def _all_heads(B, H):
+    return [(b, h) for b in range(B) for h in range(H)]
+
+
+def test_single_tile_workload():
+    w = wl.WORKLOADS[0]
+    q, k, v, _ = wl.draw_inputs(w)
+    o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    _compare_heads(q, k, v, o, lse, _all_heads(w.B, w.H), w.causal, w.scale, w.p_drop, w.seed)
+
+
+def test_causal_n1024_all_heads():
+    w = wl.WORKLOADS[1]
+    q, k, v, _ = wl.draw_inputs(w)
+    o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    _compare_heads(q, k, v, o, lse, _all_heads(w.B, w.H), w.causal, w.scale, w.p_drop, w.seed)
+
+
+def test_causal_dropout_n4096_full_size():
+    w = wl.WORKLOADS[2]
+    q, k, v, _ = wl.draw_inputs(w)
+    o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    _compare_heads(q, k, v, o, lse, [(0, 0), (1, 7), (3, 15)], w.causal, w.scale, w.p_drop, w.seed)
+
+
+@pytest.mark.parametrize("idx", [3, 4])
+def test_long_context_full_size_sampled_rows(idx):
+    w = wl.WORKLOADS[idx]
+    q, k, v, _ = wl.draw_inputs(w)
+    o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    samples = wl.sample_rows(w, n_rows=256)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (0, w.H // 2)]
+    rows = {(b, h): samples[b][h].numpy() for b, h in heads}
+    _compare_heads(q, k, v, o, lse, heads, w.causal, w.scale, w.p_drop, w.seed, rows)
+
+
+# ---------------------------------------------------------------- edge cases
+
+@pytest.mark.parametrize("B,H,N,d,causal,p", [
+    (1, 1, 128, 128, True, 0.0),     # one tile, diagonal only
+    (1, 2, 384, 64, True, 0.0),      # odd number of query tiles: last CTA owns one tile
+    (1, 2, 384, 128, False, 0.1),    # odd tiles, non-causal, dropout
+    (2, 3, 640, 64, False, 0.0),     # non-causal, several key tiles per CTA (ragged tail of CTAs)
+    (1, 1, 1024, 128, True, 0.5),    # threshold exactly 0x8000
+    (1, 1, 512, 64, True, 0.7),      # threshold above 0x8000
+    (1, 2, 256, 128, False, 0.0),
+])
+def test_edge_shapes(B, H, N, d, causal, p):
+    w = wl.Workload("edge", B, H, N, d, causal, p, 77)
+    q, k, v, _ = wl.draw_inputs(w)
+    o, lse = _run(q, k, v, causal, w.scale, p, 1234)
+    _compare_heads(q, k, v, o, lse, _all_heads(B, H), causal, w.scale, p, 1234)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_q_closed_form_through_kernel(causal):
+    """Q = 0: O is the (prefix) mean of V and LSE = ln(count), independent of the oracle."""
+    B, H, N, d = 1, 2, 512, 64
+    g = torch.Generator().manual_seed(5)
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    k = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    o, lse = _run(q, k, v, causal, 0.125, 0.0, 0)
+    vv = v.to(torch.float64).numpy()
+    for h in range(H):
+        if causal:
+            want = np.cumsum(vv[0, h], axis=0) / np.arange(1, N + 1)[:, None]
+            want_l = np.log(np.arange(1, N + 1))
+        else:
+            want = np.broadcast_to(vv[0, h].mean(axis=0), (N, d))
+            want_l = np.full(N, np.log(N))
+        pu.check_o(pu.f64(o[0, h]), want, "Q=0")
+        pu.check_lse(pu.f64(lse[0, h]), want_l, "Q=0")
+
+
+def test_no_device_wait_timed_out():
+    from exact_io_aware_49_b200 import fa_last_device_error
+    assert fa_last_device_error() == 0
