@@ -42,6 +42,12 @@ def load_library(path=None):
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_prepare.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    lib.fa_bwd_prepare.restype = i
+    lib.fa_bwd_tiles.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp, sz, vp]
+    lib.fa_bwd_tiles.restype = i
+    lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
+    lib.fa_bwd_finish.restype = i
     lib.fa_dropout_mask.argtypes = [vp, i, i, i, f, u64, vp]
     lib.fa_dropout_mask.restype = i
     lib.fa_last_device_error.argtypes = []
@@ -113,6 +119,41 @@ def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspac
                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
                     float(p_drop), int(seed) & (2**64 - 1), workspace.data_ptr(), workspace.numel(), _stream(q))
     _raise(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_bwd_stages(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspace=None, dq=None, dk=None,
+                  dv=None, between=None):
+    """fa_bwd as its three ABI stages (prepare, tiles, finish).  ``between(i)``, if
+    given, is called before stage i and after the last (i = 0..3) -- e.g. to
+    record CUDA events around the tiles kernel."""
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, q.shape)
+    B, H, N, d = q.shape
+    scale = d ** -0.5 if scale is None else scale
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), device=q.device, dtype=torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    st = _stream(q)
+    seed = int(seed) & (2**64 - 1)
+    ws, wsb = workspace.data_ptr(), workspace.numel()
+    if between:
+        between(0)
+    _raise(lib.fa_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, ws, wsb, st),
+           "fa_bwd_prepare")
+    if between:
+        between(1)
+    _raise(lib.fa_bwd_tiles(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                            B, H, N, d, int(bool(causal)), float(scale), float(p_drop), seed, ws, wsb, st),
+           "fa_bwd_tiles")
+    if between:
+        between(2)
+    _raise(lib.fa_bwd_finish(dq.data_ptr(), B, H, N, d, float(scale), ws, wsb, st), "fa_bwd_finish")
+    if between:
+        between(3)
     return dq, dk, dv
 
 

@@ -129,50 +129,122 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(rows * sizeof(float), 256);
 }
 
-fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                 void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
-                 uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return FA_ERR_INVALID_ARG;
-  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
-      misaligned(LSE, 16) || misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16) ||
-      misaligned(workspace, 256))
+}  // extern "C"
+
+namespace {
+
+// Workspace carve-up shared by the backward entry points.
+void carve_workspace(fa::BwdArgs* a, void* workspace) {
+  char* ws = static_cast<char*>(workspace);
+  const size_t rows = static_cast<size_t>(a->B) * a->H * a->N;
+  const size_t acc_bytes = round_up(rows * a->d * sizeof(float), 256);
+  const size_t vec_bytes = round_up(rows * sizeof(float), 256);
+  a->dQacc = reinterpret_cast<float*>(ws);
+  a->Dvec = reinterpret_cast<float*>(ws + acc_bytes);
+  a->lse2 = reinterpret_cast<float*>(ws + acc_bytes + vec_bytes);
+}
+
+fa_status check_workspace(const void* workspace, size_t workspace_bytes, int B, int H, int N, int d) {
+  if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+void fill_scalars(fa::BwdArgs* a, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                  uint64_t seed) {
+  a->B = B;
+  a->H = H;
+  a->N = N;
+  a->d = d;
+  a->causal = causal ? 1 : 0;
+  a->scale = scale;
+  a->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a->drop_t = drop_threshold(p_drop);
+  a->drop_scale = a->drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
+  a->seed_lo = static_cast<uint32_t>(seed);
+  a->seed_hi = static_cast<uint32_t>(seed >> 32);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!O || !dO || !LSE) return FA_ERR_INVALID_ARG;
+  if (misaligned(O, 16) || misaligned(dO, 16) || misaligned(LSE, 16)) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, 1.0f, 0.0f);
+  if (st != FA_OK) return st;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
+  fa::BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  fill_scalars(&a, B, H, N, d, 0, 1.0f, 0.0f, 0);
+  carve_workspace(&a, workspace);
+  a.O = O;
+  a.dO = dO;
+  a.LSE = LSE;
+  return fa::launch_bwd_prepare(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
+                       int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !dO || !dK || !dV) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) || misaligned(dK, 16) ||
+      misaligned(dV, 16))
     return FA_ERR_INVALID_ARG;
   fa_status st = check_common(B, H, N, d, scale, p_drop);
   if (st != FA_OK) return st;
-  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
-
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
   fa::BwdArgs a;
   memset(&a, 0, sizeof(a));
   const long long rows = static_cast<long long>(B) * H * N;
   if (!encode_rows_map(&a.tmQ, Q, rows, d) || !encode_rows_map(&a.tmK, K, rows, d) ||
       !encode_rows_map(&a.tmV, V, rows, d) || !encode_rows_map(&a.tmDO, dO, rows, d))
     return FA_ERR_CUDA;
-  a.O = O;
+  fill_scalars(&a, B, H, N, d, causal, scale, p_drop, seed);
+  carve_workspace(&a, workspace);
   a.dO = dO;
-  a.LSE = LSE;
-  a.dQ = dQ;
   a.dK = dK;
   a.dV = dV;
-  a.dQacc = static_cast<float*>(workspace);
-  a.Dvec = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                    round_up(static_cast<size_t>(rows) * d * sizeof(float), 256));
   a.err = error_word_ptr();
   if (!a.err) return FA_ERR_CUDA;
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.d = d;
-  a.causal = causal ? 1 : 0;
-  a.scale = scale;
-  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  a.drop_t = drop_threshold(p_drop);
-  a.drop_scale = a.drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
-  a.seed_lo = static_cast<uint32_t>(seed);
-  a.seed_hi = static_cast<uint32_t>(seed >> 32);
-  return fa::launch_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return fa::launch_bwd_tiles(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!dQ || misaligned(dQ, 16)) return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, 0.0f);
+  if (st != FA_OK) return st;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
+  fa::BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  fill_scalars(&a, B, H, N, d, 0, scale, 0.0f, 0);
+  carve_workspace(&a, const_cast<void*>(workspace));
+  a.dQ = dQ;
+  return fa::launch_bwd_finish(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                 void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                 uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  // Validate everything up front so a rejected call launches none of the stages.
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
+      misaligned(LSE, 16) || misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_common(B, H, N, d, scale, p_drop);
+  if (st != FA_OK) return st;
+  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
+  if ((st = fa_bwd_prepare(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK) return st;
+  if ((st = fa_bwd_tiles(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes,
+                         stream)) != FA_OK)
+    return st;
+  return fa_bwd_finish(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed, void* stream) {
@@ -193,7 +265,8 @@ fa_status fa_last_device_error(void) {
   if (v) {
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+    // bit 0: a bounded wait gave up; bit 1: the shared-memory layout did not fit (kernel did nothing)
+    return (v & 1u) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
   }
   return FA_OK;
 }

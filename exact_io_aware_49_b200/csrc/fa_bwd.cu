@@ -1,6 +1,599 @@
-// fa_bwd.cu -- attention backward (placeholder until the kernels land).
+// fa_bwd.cu -- attention backward by recomputation for sm_100a.
+//
+// The backward pass stores no N x N intermediate: it recomputes the scores
+// and probabilities tile by tile from the stored per-row statistic LSE and
+// regenerates the dropout pattern from (seed, b, h, i, j) instead of reading
+// a stored mask ("FlashAttention" glossary, Recomputation; "Flash Attention"
+// glossary, How Flash Attention Works step 6 and Key Components).
+//
+// Gradients of L = sum(dO * O) with O = (P * Z / (1-p)) V, P = softmax(scale S):
+//   dV = (P*Z/(1-p))^T dO            dP = (dO V^T) * Z / (1-p)
+//   D_i = sum_c dO_ic O_ic            dS = P * (dP - D)
+//   dQ = scale * dS K                 dK = scale * dS^T Q
+//
+// Three kernels:
+//   1. preprocess: D_i = rowsum(dO * O) (fp32, from the stored bf16 O),
+//      LSE2_i = LSE_i * log2(e), and zeroing of the fp32 dQ accumulator;
+//   2. main: one CTA per (b, h, 128-key tile j) keeps K_j, V_j in shared
+//      memory and dK_j, dV_j in tensor memory while it streams the query
+//      tiles i (i >= j when causal) through a two-stage TMA ring.  Per tile:
+//        S^T = K_j Q_i^T and dP^T = V_j dO_i^T  (tcgen05, M = 128 keys)
+//        P^T = exp2(S^T scale log2e - LSE2_i), masked, dropout-masked
+//              -> written as bf16 into TMEM over S^T
+//        dV += P^T dO_i                          (A operand read from TMEM)
+//        dS^T = P^T (dP^T Z/(1-p) - D_i)  -> bf16, 128B-swizzled in smem
+//        dK += dS^T Q_i ;  dQ_i = dS K_j  (the same smem tile read K-major
+//              for dK and MN-major for dQ)
+//        dQ_i is read out of TMEM by a dedicated warpgroup and added to the
+//        fp32 accumulator with vector reductions.
+//      Warp roles: warpgroups 0/1 do the elementwise work for query columns
+//      0-63 / 64-127 (one thread per key row, the TMEM lane); warp 8 issues
+//      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
+//   3. convert: dQ = bf16(scale * dQacc).
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
 #include "fa_internal.h"
+#include "philox.cuh"
+#include "sm100.cuh"
+
 namespace fa {
-cudaError_t launch_bwd(const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+// ============================================================ preprocess
+
+// One warp per row: D = sum(dO * O), LSE2 = LSE * log2(e), dQacc row = 0.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ O,
+                                                                const __nv_bfloat16* __restrict__ dO,
+                                                                const float* __restrict__ LSE,
+                                                                float* __restrict__ Dvec,
+                                                                float* __restrict__ lse2,
+                                                                float* __restrict__ dQacc, long long rows) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long row = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    // D / 8 lanes active per 16-byte chunk: lane covers elements [8*lane, 8*lane+8) when 8*lane < D
+    float acc = 0.f;
+    if (lane * 8 < D) {
+      const uint4 a = *reinterpret_cast<const uint4*>(O + row * D + lane * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + lane * 8);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+        const float2 fb2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+        acc = fmaf(fa2.x, fb2.x, acc);
+        acc = fmaf(fa2.y, fb2.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    float4* zq = reinterpret_cast<float4*>(dQacc + row * D);
+    for (int c = lane; c < D / 4; c += 32) zq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0) {
+      Dvec[row] = acc;
+      lse2[row] = LSE[row] * 1.4426950408889634f;
+    }
+  }
+}
+
+// ============================================================ dQ convert
+
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ dQacc,
+                                                                __nv_bfloat16* __restrict__ dQ, float scale,
+                                                                long long n8) {
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n8;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(dQacc)[2 * idx];
+    const float4 b = reinterpret_cast<const float4*>(dQacc)[2 * idx + 1];
+    uint4 o;
+    o.x = pack_bf16x2(a.x * scale, a.y * scale);
+    o.y = pack_bf16x2(a.z * scale, a.w * scale);
+    o.z = pack_bf16x2(b.x * scale, b.y * scale);
+    o.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dQ)[idx] = o;
+  }
+}
+
+// ============================================================ main kernel
+
+constexpr int kBwdThreads = 512;
+constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdLoadWarp = 9;
+// setmaxnreg split over the launch pool of 512 threads x 128 registers:
+// two elementwise warpgroups, the dQ-drain warpgroup, the control warpgroup.
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kEwRegs = 168;
+constexpr int kDqRegs = 112;
+constexpr int kCtlRegs = 56;
+static_assert(2 * 128 * kEwRegs + 128 * kDqRegs + 128 * kCtlRegs <= kBwdThreads * kBwdLaunchRegs, "register split");
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kTile = 128 * D * 2;  // 128 rows x D bf16
+  static constexpr int kBox = 128 * 128;     // 128 rows x 64 bf16 (one 128-byte swizzle span)
+  static constexpr int kK = 0;
+  static constexpr int kV = kTile;
+  static constexpr int kQ = 2 * kTile;      // 2 stages
+  static constexpr int kDO = 4 * kTile;     // 2 stages
+  static constexpr int kDS = 6 * kTile;     // dS^T: 128 keys x 128 queries bf16 = 2 boxes
+  static constexpr int kVec = kDS + 2 * kBox;  // 2 stages x (LSE2[128], D[128]) fp32
+  static constexpr int kBar = kVec + 2 * 1024;
+  static constexpr int kNumBars = 16;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kUsed = kMisc + 16;
+};
+
+enum BwdBar {
+  kKVFull = 0,
+  kQFull0 = 1,   // +stage
+  kDOFull0 = 3,  // +stage
+  kEmpty0 = 5,   // +stage
+  kSReady = 7,
+  kDPReady = 8,
+  kPReady = 9,
+  kDSReady = 10,
+  kDSFree = 11,
+  kDQReady = 12,
+  kDQFree = 13,
+  kDKDVReady = 14,
+  kDrain = 15,
+};
+
+struct BwdParams {
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  float* dQacc;
+  const float* lse2;
+  const float* Dvec;
+  unsigned* err;
+  int H, N;
+  float scale;
+  float scale_log2;
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
+};
+
+// D[tmem] (+)= A[K-major tile] * B[K-major tile]^T, M = N = 128, K = D.
+template <int D>
+__device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
+    mma_ss(tmem_d, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc, kk > 0);
+  }
+}
+
+// dV (+)= P^T dO : A = P^T (TMEM, bf16 pairs), B = dO tile (MN-major), K = 128 queries, N = D.
+template <int D>
+__device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts(tmem_d, tmem_p + kk * 8, sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// dK (+)= dS^T Q : A = dS^T (smem, K-major over queries), B = Q tile (MN-major), N = D.
+template <int D>
+__device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32_t q_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t a_off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
+    mma_ss(tmem_d, sdesc_sw128(ds_smem + a_off, 16, 1024), sdesc_sw128(q_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
+           idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// dQ_i = dS K : A = dS (the dS^T tile read MN-major, M = queries), B = K tile (MN-major), N = D.
+template <int D>
+__device__ __forceinline__ void mma_dq(uint32_t tmem_d, uint32_t ds_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ss(tmem_d, sdesc_sw128(ds_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
+           sdesc_sw128(k_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, kk > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
+  tc_fence_before();
+  asm volatile("bar.sync 1, %0;" ::"n"(kBwdThreads) : "memory");
+  tc_fence_after();
+  if (dealloc) tmem_dealloc(tmem, 512);
+}
+
+// Keep bits of the dropout mask for one key row and 8 consecutive queries
+// q0..q0+7.  The Philox counter (key >> 3, query, h, b) yields 8 keys x 1
+// query per call, so lane l of each group of 8 consecutive keys evaluates
+// query q0 + l, and 8 warp ballots transpose the 8 x 8 bit block: the result
+// has bit l set when (this lane's key, query q0 + l) is kept.
+__device__ __forceinline__ uint32_t keep_bits_8(uint32_t key_grp, uint32_t q0, uint32_t h, uint32_t b,
+                                                uint32_t seed_lo, uint32_t seed_hi, DropConst dk, int lane) {
+  const int l8 = lane & 7;
+  uint32_t w[4];
+  philox4x32_10(key_grp, q0 + l8, h, b, seed_lo, seed_hi, w);
+  uint32_t mine = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t km = keep_mask_2x16(w[e], dk);
+    const uint32_t b_lo = __ballot_sync(0xffffffffu, (km & 1u) != 0);
+    const uint32_t b_hi = __ballot_sync(0xffffffffu, (km >> 31) != 0);
+    mine = (l8 == 2 * e) ? b_lo : mine;
+    mine = (l8 == 2 * e + 1) ? b_hi : mine;
+  }
+  return (mine >> (lane & ~7)) & 0xFFu;
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  using L = BwdSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (!smem_layout_fits(smem_raw, smem, L::kUsed, p.err)) return;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int N = p.N;
+  const int n_t = N / 128;
+  const int kj = blockIdx.y;                 // key tile (lowest first: the heaviest causal work)
+  const int q_first = CAUSAL ? kj : 0;
+  const int nq = n_t - q_first;              // query tiles visited
+  const int row0 = bh * N;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i)
+      mbar_init(&bars[i], (i == kPReady || i == kDSReady) ? 8u : (i == kDQFree ? 4u : 1u));
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // TMEM columns: S^T [0,128) (P^T over [0,64)), dP^T / dQ [128,256), dK, dV after.
+  constexpr uint32_t kColS = 0, kColDP = 128, kColDK = 256, kColDV = 256 + D;
+  const uint32_t sm_k = smem_u32(smem + L::kK), sm_v = smem_u32(smem + L::kV);
+  const uint32_t sm_q = smem_u32(smem + L::kQ), sm_do = smem_u32(smem + L::kDO);
+  const uint32_t sm_ds = smem_u32(smem + L::kDS);
+
+  if (warp >= 8 && warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
+    if (warp == kBwdLoadWarp && lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      mbar_expect_tx(&bars[kKVFull], 2 * L::kTile);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(smem + L::kK + c * L::kBox, &tmK, c * 64, row0 + kj * 128, &bars[kKVFull]);
+        tma_load_2d(smem + L::kV + c * L::kBox, &tmV, c * 64, row0 + kj * 128, &bars[kKVFull]);
+      }
+      int issued = 0;
+      for (int it = 0; it < nq; ++it) {
+        const int s = it & 1;
+        const int qrow = row0 + (q_first + it) * 128;
+        if (it >= 2 && !mbar_wait(&bars[kEmpty0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
+        mbar_expect_tx(&bars[kQFull0 + s], L::kTile + 1024);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, qrow, &bars[kQFull0 + s]);
+        bulk_load_1d(smem + L::kVec + s * 1024, p.lse2 + qrow, 512, &bars[kQFull0 + s]);
+        bulk_load_1d(smem + L::kVec + s * 1024 + 512, p.Dvec + qrow, 512, &bars[kQFull0 + s]);
+        mbar_expect_tx(&bars[kDOFull0 + s], L::kTile);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, qrow, &bars[kDOFull0 + s]);
+        issued = it + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(&bars[kKVFull], 0);
+        for (int it = max(0, issued - 2); it < issued; ++it) {
+          mbar_wait_drain(&bars[kQFull0 + (it & 1)], (it >> 1) & 1);
+          mbar_wait_drain(&bars[kDOFull0 + (it & 1)], (it >> 1) & 1);
+        }
+      }
+    } else if (warp == kBwdMmaWarp && lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err) &&
+                mbar_wait(&bars[kQFull0], 0, abort_flag, p.err);
+      if (ok) {
+        tc_fence_after();
+        mma_tile_kk<D>(tmem + kColS, sm_k, sm_q);
+        mma_commit(&bars[kSReady]);
+        ok = mbar_wait(&bars[kDOFull0], 0, abort_flag, p.err);
+        if (ok) {
+          tc_fence_after();
+          mma_tile_kk<D>(tmem + kColDP, sm_v, sm_do);
+          mma_commit(&bars[kDPReady]);
+        }
+      }
+      for (int it = 0; ok && it < nq; ++it) {
+        const int s = it & 1, s1 = (it + 1) & 1;
+        const bool more = it + 1 < nq;
+        if (!mbar_wait(&bars[kPReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        mma_dv<D>(tmem + kColDV, tmem + kColS, sm_do + s * L::kTile, it > 0);
+        if (more) {
+          if (!mbar_wait(&bars[kQFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          mma_tile_kk<D>(tmem + kColS, sm_k, sm_q + s1 * L::kTile);
+          mma_commit(&bars[kSReady]);
+        }
+        if (!mbar_wait(&bars[kDSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        mma_dk<D>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
+        mma_commit(&bars[kEmpty0 + s]);
+        mma_dq<D>(tmem + kColDP, sm_ds, sm_k);
+        mma_commit(&bars[kDQReady]);
+        mma_commit(&bars[kDSFree]);
+        if (more) {
+          if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
+              !mbar_wait(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          mma_tile_kk<D>(tmem + kColDP, sm_v, sm_do + s1 * L::kTile);
+          mma_commit(&bars[kDPReady]);
+        }
+      }
+      if (ok) {
+        mma_commit(&bars[kDKDVReady]);
+      } else {
+        mma_commit(&bars[kDrain]);
+        mbar_wait_drain(&bars[kDrain], 0);
+      }
+    }
+    __syncwarp();
+    bwd_teardown(tmem, warp == kBwdMmaWarp);
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------------ dQ drain
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDqRegs));
+    const int wq = warp & 3;
+    const int c = wq * 32 + lane;  // query row within the tile == TMEM lane
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kColDP;
+    for (int it = 0; it < nq; ++it) {
+      if (!mbar_wait(&bars[kDQReady], it & 1, abort_flag, p.err)) break;
+      tc_fence_after();
+      float* dst = p.dQacc + (static_cast<size_t>(row0) + (q_first + it) * 128 + c) * D;
+#pragma unroll
+      for (int half = 0; half < D / 64; ++half) {
+        uint32_t v[64];
+        tmem_ld32(t_row + half * 64, v);
+        tmem_ld32(t_row + half * 64 + 32, v + 32);
+        tmem_ld_wait();
+        reg_fence32(v);
+        reg_fence32(v + 32);
+        if (half == D / 64 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kDQFree]);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          red_add_v4(dst + half * 64 + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+      }
+    }
+    bwd_teardown(tmem, false);
+  } else {
+    // ------------------------------------------------------------------ elementwise
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEwRegs));
+    const int g = warp >> 2;  // query columns [64 g, 64 g + 64)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row within the tile == TMEM lane
+    const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sl2 = p.scale_log2;
+    const DropConst dk = make_drop_const(p.drop_t);
+    const uint32_t hh = static_cast<uint32_t>(bh % p.H), bb = static_cast<uint32_t>(bh / p.H);
+    const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
+    const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
+    bool ok = true;
+    for (int it = 0; it < nq; ++it) {
+      const int s = it & 1;
+      const int qi = q_first + it;
+      if (!mbar_wait(&bars[kQFull0 + s], (it >> 1) & 1, abort_flag, p.err) ||
+          !mbar_wait(&bars[kSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(t_row + kColS + 64 * g, sr);
+      tmem_ld32(t_row + kColS + 64 * g + 32, sr + 32);
+      tmem_ld_wait();
+      reg_fence32(sr);
+      reg_fence32(sr + 32);
+      const float* lse2 = reinterpret_cast<const float*>(smem + L::kVec + s * 1024) + 64 * g;
+      const float* dvec = lse2 + 128;
+      float P[64];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * c4);
+        P[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l4.x));
+        P[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l4.y));
+        P[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l4.z));
+        P[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l4.w));
+      }
+      if (CAUSAL && qi == kj) {
+        // query 64 g + c precedes key r: masked
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (64 * g + c < r) P[c] = 0.f;
+      }
+      uint32_t zb[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+      if (DROPOUT) {
+        const uint32_t q0 = static_cast<uint32_t>(qi * 128 + 64 * g);
+#pragma unroll
+        for (int bq = 0; bq < 8; ++bq) {
+          const uint32_t bits = keep_bits_8(key_grp, q0 + 8 * bq, hh, bb, p.seed_lo, p.seed_hi, dk, lane);
+          if (bq % 4 == 0) zb[bq / 4] = 0;
+          zb[bq / 4] |= bits << (8 * (bq % 4));
+        }
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float a = P[2 * c], b2 = P[2 * c + 1];
+        if (DROPOUT) {
+          a = ((zb[c / 16] >> ((2 * c) % 32)) & 1u) ? a : 0.f;
+          b2 = ((zb[c / 16] >> ((2 * c + 1) % 32)) & 1u) ? b2 : 0.f;
+        }
+        pk[c] = pack_bf16x2(a, b2);
+      }
+      tmem_st32(t_row + kColS + 32 * g, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kPReady]);
+
+      if (!mbar_wait(&bars[kDPReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t dr[64];
+      tmem_ld32(t_row + kColDP + 64 * g, dr);
+      tmem_ld32(t_row + kColDP + 64 * g + 32, dr + 32);
+      tmem_ld_wait();
+      reg_fence32(dr);
+      reg_fence32(dr + 32);
+      uint32_t dsk[32];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(dvec + 4 * c4);
+        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          float dp = __uint_as_float(dr[c]);
+          if (DROPOUT) dp = ((zb[c / 32] >> (c % 32)) & 1u) ? dp * p.drop_scale : 0.f;
+          v[e] = P[c] * (dp - dd[e]);
+        }
+        dsk[2 * c4] = pack_bf16x2(v[0], v[1]);
+        dsk[2 * c4 + 1] = pack_bf16x2(v[2], v[3]);
+      }
+      // the previous dK / dQ MMAs must have finished reading dS^T
+      if (it > 0 && !mbar_wait(&bars[kDSFree], (it - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(ds_row + ((ch ^ (r & 7)) << 4), dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2],
+                     dsk[4 * ch + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kDSReady]);
+    }
+    if (ok && mbar_wait(&bars[kDKDVReady], 0, abort_flag, p.err)) {
+      // -------------------------------------------------------------- dK / dV epilogue
+      tc_fence_after();
+      const uint32_t col = (g == 0) ? kColDK : kColDV;
+      const float mul = (g == 0) ? p.scale : p.drop_scale;
+      __nv_bfloat16* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(row0) + kj * 128 + r) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(t_row + col + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence32(v);
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+      }
+    }
+    bwd_teardown(tmem, false);
+  }
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
+cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
+  auto kern = fa_bwd_kernel<D, CAUSAL, DROPOUT>;
+  const int used = BwdSmem<D>::kUsed;
+  int max_optin = 0, dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  // 1 KB of slack realigns the dynamic shared-memory base to 1024 bytes when
+  // it is not already aligned; where the budget is tighter the base must be.
+  const int smem = (used + 1024 <= max_optin) ? used + 1024 : used;
+  if (smem > max_optin) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes attr;
+  e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  if (attr.numRegs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
+  BwdParams p;
+  p.dK = static_cast<__nv_bfloat16*>(a.dK);
+  p.dV = static_cast<__nv_bfloat16*>(a.dV);
+  p.dQacc = a.dQacc;
+  p.lse2 = a.lse2;
+  p.Dvec = a.Dvec;
+  p.err = a.err;
+  p.H = a.H;
+  p.N = a.N;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale_log2;
+  p.drop_t = a.drop_t;
+  p.drop_scale = a.drop_scale;
+  p.seed_lo = a.seed_lo;
+  p.seed_hi = a.seed_hi;
+  dim3 grid(a.B * a.H, a.N / 128);
+  kern<<<grid, kBwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmDO, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(a.B) * a.H * a.N;
+  long long blocks = (rows + 7) / 8;  // one warp per row, 8 warps per block
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  const __nv_bfloat16* O = static_cast<const __nv_bfloat16*>(a.O);
+  const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(a.dO);
+  if (a.d == 64)
+    fa_bwd_preprocess_kernel<64><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
+                                                                               a.dQacc, rows);
+  else
+    fa_bwd_preprocess_kernel<128><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
+                                                                                a.dQacc, rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream) {
+  const bool drop = a.drop_t != 0;
+  if (a.d == 64) {
+    if (a.causal) return drop ? launch_bwd_main<64, true, true>(a, stream) : launch_bwd_main<64, true, false>(a, stream);
+    return drop ? launch_bwd_main<64, false, true>(a, stream) : launch_bwd_main<64, false, false>(a, stream);
+  }
+  if (a.causal) return drop ? launch_bwd_main<128, true, true>(a, stream) : launch_bwd_main<128, true, false>(a, stream);
+  return drop ? launch_bwd_main<128, false, true>(a, stream) : launch_bwd_main<128, false, false>(a, stream);
+}
+
+cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
+  const long long n8 = static_cast<long long>(a.B) * a.H * a.N * a.d / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  fa_bwd_dq_convert_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, static_cast<__nv_bfloat16*>(a.dQ),
+                                                                        a.scale, n8);
+  return cudaGetLastError();
+}
+
 }  // namespace fa

@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (!smem_layout_fits(smem_raw, smem, L::kMisc + 16, p.err)) return;
   const FwdBars bar = fwd_bars<D>(smem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);

@@ -30,7 +30,8 @@ struct BwdArgs {
   void* dK;
   void* dV;
   float* dQacc;  // fp32 [B, H, N, d] workspace
-  float* Dvec;   // fp32 [B, H, N] workspace
+  float* Dvec;   // fp32 [B, H, N] workspace: rowsum(dO * O)
+  float* lse2;   // fp32 [B, H, N] workspace: LSE * log2(e)
   unsigned* err;
   int B, H, N, d;
   int causal;
@@ -42,7 +43,11 @@ struct BwdArgs {
 };
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+// The three backward stages; fa_bwd runs them in this order.  Only the fields
+// each stage reads need to be set.
+cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream);  // O, dO, LSE -> Dvec, lse2, dQacc = 0
+cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream);    // maps, lse2, Dvec -> dK, dV, dQacc
+cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream);   // dQacc -> dQ
 cudaError_t launch_dropout_mask(uint8_t* mask, int B, int H, int N, uint32_t drop_t, uint32_t seed_lo,
                                 uint32_t seed_hi, cudaStream_t stream);
 

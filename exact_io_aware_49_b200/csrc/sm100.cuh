@@ -24,6 +24,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Error bits recorded in the device error word.
 constexpr unsigned kErrWaitTimeout = 1u;
+constexpr unsigned kErrSmemLayout = 2u;
+
+__device__ __forceinline__ uint32_t dynamic_smem_size() {
+  uint32_t r;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
+
+// The kernels align their shared-memory carve-out to 1024 bytes (128-byte
+// swizzled TMA / UMMA tiles need it).  Returns false -- after recording the
+// error -- when the aligned layout of ``used`` bytes would not fit the dynamic
+// allocation; every thread of the CTA must then return without touching it.
+__device__ __forceinline__ bool smem_layout_fits(const uint8_t* raw, const uint8_t* aligned, uint32_t used,
+                                                 unsigned* err) {
+  const uint32_t pad = static_cast<uint32_t>(aligned - raw);
+  if (pad + used <= dynamic_smem_size()) return true;
+  if (threadIdx.x == 0 && err) atomicOr(err, kErrSmemLayout);
+  return false;
+}
 
 // A pipeline wait gives up after this long.  No legitimate wait inside one
 // CTA lasts more than a few milliseconds; the limit only has to separate a
@@ -108,6 +127,24 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Four fp32 reductions into consecutive global words (16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -84,9 +84,10 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
- * accumulator [B, H, N, d] plus the fp32 row statistic D [B, H, N], each
- * rounded up to 256 bytes.  Linear in N ("FlashAttention" glossary: memory
- * drops from O(N^2) to O(N)).  Returns 0 for non-positive sizes.
+ * accumulator [B, H, N, d], the fp32 row statistic D [B, H, N] and the
+ * fp32 copy of LSE in log2 units [B, H, N], each rounded up to 256 bytes.
+ * Linear in N ("FlashAttention" glossary: memory drops from O(N^2) to O(N)).
+ * Returns 0 for non-positive sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -114,6 +115,27 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  void* stream);
 
 /*
+ * The three stages fa_bwd runs, in order, for callers that schedule or time
+ * them separately.  Same conventions and argument meanings as fa_bwd; each
+ * validates its own arguments and enqueues one kernel.
+ *   fa_bwd_prepare: D_i = sum_c dO_ic O_ic, LSE_i * log2(e), zero the dQ
+ *                   accumulator (all in ``workspace``);
+ *   fa_bwd_tiles:   the fused pass over (key tile, query tile) pairs that
+ *                   recomputes P from the prepared LSE, regenerates the
+ *                   dropout mask, writes dK and dV and adds into the dQ
+ *                   accumulator; needs a workspace fa_bwd_prepare filled on the
+ *                   same stream (or one ordered before it);
+ *   fa_bwd_finish:  dQ = bf16(scale * accumulator).
+ */
+fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
+                       int B, int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed,
+                       void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
  * Test/inspection export: writes the dropout keep mask Z (1 = kept, 0 =
  * dropped) as uint8 [B, H, N, N] into device memory ``mask`` with the same
  * device Philox code the kernels use.  N here only needs to be positive.
@@ -122,9 +144,11 @@ fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint
                           void* stream);
 
 /*
- * Synchronises the device, then reads and clears the device error word that
- * bounded waits set.  FA_OK when no wait gave up since the last call,
- * FA_ERR_TIMEOUT otherwise, FA_ERR_CUDA if the device could not be read.
+ * Synchronises the device, then reads and clears the device error word.
+ * FA_OK when no kernel recorded a problem since the last call; FA_ERR_TIMEOUT
+ * when a bounded wait gave up; FA_ERR_CUDA when a kernel found its shared-
+ * memory layout would not fit and returned without work, or the device could
+ * not be read.
  */
 fa_status fa_last_device_error(void);
 

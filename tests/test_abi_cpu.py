@@ -33,8 +33,8 @@ def _declared_functions():
 
 def test_header_declares_entry_points():
     names = _declared_functions()
-    for want in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_dropout_mask", "fa_last_device_error",
-                 "fa_status_string"):
+    for want in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_tiles", "fa_bwd_finish",
+                 "fa_dropout_mask", "fa_last_device_error", "fa_status_string"):
         assert want in names
 
 
@@ -81,7 +81,7 @@ def _bwd(lib, ws=A, ws_bytes=None, B=1, H=1, N=128, d=64, p=0.0, **ptrs):
 def test_workspace_size_is_linear_in_n(lib):
     s1 = lib.fa_bwd_workspace_size(2, 3, 1024, 128)
     s2 = lib.fa_bwd_workspace_size(2, 3, 2048, 128)
-    assert s1 == 2 * 3 * 1024 * 128 * 4 + 2 * 3 * 1024 * 4
+    assert s1 == 2 * 3 * 1024 * 128 * 4 + 2 * (2 * 3 * 1024 * 4)
     assert s2 == 2 * s1
     assert lib.fa_bwd_workspace_size(0, 1, 128, 64) == 0
 
@@ -92,6 +92,19 @@ def test_workspace_size_is_linear_in_n(lib):
 ])
 def test_bwd_rejects_bad_arguments(lib, kw, want):
     assert _bwd(lib, **kw) == want
+
+
+def test_stage_entry_points_reject_bad_arguments(lib):
+    ws_ok = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert lib.fa_bwd_prepare(0, A, A, 1, 1, 128, 64, A, ws_ok, None) == 1
+    assert lib.fa_bwd_prepare(A, A, A, 1, 1, 128, 64, A, ws_ok - 4, None) == 1
+    assert lib.fa_bwd_prepare(A, A, A, 1, 1, 100, 64, A, ws_ok, None) == 2
+    assert lib.fa_bwd_tiles(A, A, A, A, A, 0, 1, 1, 128, 64, 1, 0.125, 0.0, 0, A, ws_ok, None) == 1
+    assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 1.0, 0, A, ws_ok, None) == 1
+    assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, 96, 1, 0.125, 0.0, 0, A, ws_ok, None) == 2
+    assert lib.fa_bwd_finish(A + 8, 1, 1, 128, 64, 0.125, A, ws_ok, None) == 1
+    assert lib.fa_bwd_finish(A, 1, 1, 128, 64, 0.125, A + 64, ws_ok, None) == 1
+    assert lib.fa_bwd_finish(A, 1, 1, 128, 64, -1.0, A, ws_ok, None) == 1
 
 
 def test_mask_rejects_bad_arguments(lib):
