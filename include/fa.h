@@ -136,6 +136,37 @@ fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const
                         size_t workspace_bytes, void* stream);
 
 /*
+ * Backward pass for callers that cannot allocate device memory.  (The pages
+ * have no counterpart: this is an integration convenience of this library.)
+ * Some callers may not call cudaMalloc at all -- a plugin running inside a
+ * framework whose memory pool owns every device allocation, a latency-critical
+ * loop that cannot take the synchronisation an allocation may cause, or a
+ * deployment with a fixed, audited memory budget.  fa_bwd_noalloc computes
+ * exactly what fa_bwd computes, with the same arguments minus the workspace:
+ * its scratch (fp32 dQ accumulator, D and LSE*log2(e)) lives in a fixed array
+ * of FA_NOALLOC_SCRATCH_BYTES in the library's static device memory, which
+ * every GPU that loads the library holds until the process exits.  The caller
+ * still owns and passes every input and output.
+ *   - Limit: fa_bwd_workspace_size(B, H, N, d) must not exceed
+ *     FA_NOALLOC_SCRATCH_BYTES; larger problems return FA_ERR_UNSUPPORTED
+ *     (use fa_bwd with a caller-provided workspace).  Since N is a multiple
+ *     of 128, that allows B*H*N <= 64512 rows at d = 128 and <= 126976 at
+ *     d = 64.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  It calls no allocating routine.
+ *   - All calls share the one array, and each call's first stage rewrites
+ *     every word of it that the call later reads, so earlier contents do not
+ *     matter; but calls that overlap on the GPU (for example on two streams
+ *     at once) race on it and must be serialised by the caller.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const float* LSE, void* dQ, void* dK, void* dV,
+                         int B, int H, int N, int d, int causal, float scale,
+                         float p_drop, uint64_t seed, void* stream);
+
+/*
  * Test/inspection export: writes the dropout keep mask Z (1 = kept, 0 =
  * dropped) as uint8 [B, H, N, N] into device memory ``mask`` with the same
  * device Philox code the kernels use.  N here only needs to be positive.
