@@ -162,6 +162,7 @@ def oracle_prefix_step(q, k, v, do, w, b, h, n):
 
 
 def cpu_baseline(q, k, v, do, w, n=4096, min_seconds=10.0):
+    n = min(n, w.N)
     flops, reps = 0.0, 0
     t0 = time.perf_counter()
     while time.perf_counter() - t0 < min_seconds or reps == 0:
@@ -179,7 +180,7 @@ def run_reference(args, w, world):
     if world["rank"] != 0:
         return None
     q, k, v, do = wl.draw_inputs(w)
-    n = 2048
+    n = min(2048, w.N)
     for i in range(args.warmup):
         oracle_prefix_step(q, k, v, do, w, 0, i % w.H, n)
     t0 = time.perf_counter()
