@@ -34,18 +34,24 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows, d] bf16 row-major, boxes of 64 columns x 128 rows, 128-byte swizzle.
-bool encode_rows_map(CUtensorMap* tm, const void* base, long long rows, int d) {
+// [rows, d] row-major 2-D map with 128-byte boxes per row (64 bf16 or 32 fp32
+// columns) x 128 rows and 128-byte swizzle.
+bool encode_rows_map_t(CUtensorMap* tm, const void* base, long long rows, int d, bool fp32) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
+  const cuuint64_t esize = fp32 ? 4 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 128};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_rows_map(CUtensorMap* tm, const void* base, long long rows, int d) {
+  return encode_rows_map_t(tm, base, rows, d, false);
 }
 
 unsigned* error_word_ptr() {
@@ -207,6 +213,7 @@ fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* 
     return FA_ERR_CUDA;
   fill_scalars(&a, B, H, N, d, causal, scale, p_drop, seed);
   carve_workspace(&a, workspace);
+  if (!encode_rows_map_t(&a.tmDQacc, a.dQacc, rows, d, true)) return FA_ERR_CUDA;
   a.dO = dO;
   a.dK = dK;
   a.dV = dV;

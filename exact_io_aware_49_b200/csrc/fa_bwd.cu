@@ -24,8 +24,8 @@
 //        dS^T = P^T (dP^T Z/(1-p) - D_i)  -> bf16, 128B-swizzled in smem
 //        dK += dS^T Q_i ;  dQ_i = dS K_j  (the same smem tile read K-major
 //              for dK and MN-major for dQ)
-//        dQ_i is read out of TMEM by a dedicated warpgroup and added to the
-//        fp32 accumulator with vector reductions.
+//        dQ_i is read out of TMEM by a dedicated warpgroup, staged through the
+//        dS^T buffer and added to the fp32 accumulator with TMA reduce-add.
 //      Warp roles: warpgroups 0/1 do the elementwise work for query columns
 //      0-63 / 64-127 (one thread per key row, the TMEM lane); warp 8 issues
 //      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
@@ -159,6 +159,7 @@ struct BwdParams {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  int group, BH;
 };
 
 // D[tmem] (+)= A[K-major tile] * B[K-major tile]^T, M = N = 128, K = D.
@@ -237,7 +238,7 @@ template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using L = BwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -248,10 +249,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  // 1-D grid over (head group, key tile, head), heaviest key tiles first
+  // within each group of p.group heads.
   const int N = p.N;
   const int n_t = N / 128;
-  const int kj = blockIdx.y;                 // key tile (lowest first: the heaviest causal work)
+  const int per_group = p.group * n_t;
+  const int grp = blockIdx.x / per_group;
+  const int rr = blockIdx.x - grp * per_group;
+  const int gsz = min(p.group, p.BH - grp * p.group);
+  const int kj = rr / gsz;                   // key tile (lowest first: the heaviest causal work)
+  const int bh = grp * p.group + (rr - kj * gsz);
   const int q_first = CAUSAL ? kj : 0;
   const int nq = n_t - q_first;              // query tiles visited
   const int row0 = bh * N;
@@ -344,7 +351,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(&bars[kEmpty0 + s]);
         mma_dq<D>(tmem + kColDP, sm_ds, sm_k);
         mma_commit(&bars[kDQReady]);
-        mma_commit(&bars[kDSFree]);
         if (more) {
           if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
               !mbar_wait(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -364,33 +370,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_teardown(tmem, warp == kBwdMmaWarp);
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain
+    // dQ_i leaves TMEM 64 columns at a time: staged as two 32-column fp32
+    // boxes in the dS^T buffer (free once dK_i and dQ_i have read it) and added
+    // into the fp32 accumulator by TMA reduce-add.  TMEM is released right after
+    // the last load, so the next dP^T MMA does not wait for the reductions.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDqRegs));
     const int wq = warp & 3;
     const int c = wq * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kColDP;
+    const bool leader = threadIdx.x == 12 * 32;
+    volatile int* go = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+    const uint32_t st_row = sm_ds + c * 128;
     for (int it = 0; it < nq; ++it) {
-      if (!mbar_wait(&bars[kDQReady], it & 1, abort_flag, p.err)) break;
+      // one thread waits (bounded); the named barrier hands its verdict to all 128
+      if (leader) *go = mbar_wait(&bars[kDQReady], it & 1, abort_flag, p.err) ? 1 : 0;
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (!*go) break;
       tc_fence_after();
-      float* dst = p.dQacc + (static_cast<size_t>(row0) + (q_first + it) * 128 + c) * D;
+      const int qrow = row0 + (q_first + it) * 128;
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
+      for (int ch = 0; ch < D / 64; ++ch) {
         uint32_t v[64];
-        tmem_ld32(t_row + half * 64, v);
-        tmem_ld32(t_row + half * 64 + 32, v + 32);
+        tmem_ld32(t_row + ch * 64, v);
+        tmem_ld32(t_row + ch * 64 + 32, v + 32);
         tmem_ld_wait();
         reg_fence32(v);
         reg_fence32(v + 32);
-        if (half == D / 64 - 1) {
+        if (ch == D / 64 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[kDQFree]);
         }
+        // the previous chunk's reduce has finished reading the staging buffer
+        if (ch > 0) asm volatile("bar.sync 2, 128;" ::: "memory");
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          red_add_v4(dst + half * 64 + 4 * e, __uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            st_shared_v4(st_row + bx * L::kBox + ((q4 ^ (c & 7)) << 4), v[32 * bx + 4 * q4],
+                         v[32 * bx + 4 * q4 + 1], v[32 * bx + 4 * q4 + 2], v[32 * bx + 4 * q4 + 3]);
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (leader) {
+          tma_reduce_add_2d(&tmDQ, smem + L::kDS, ch * 64, qrow);
+          tma_reduce_add_2d(&tmDQ, smem + L::kDS + L::kBox, ch * 64 + 32, qrow);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
       }
+      if (leader) mbar_arrive(&bars[kDSFree]);  // staging done: dS^T of the next tile may be written
     }
+    if (leader) bulk_wait_group0();
     bwd_teardown(tmem, false);
   } else {
     // ------------------------------------------------------------------ elementwise
@@ -484,7 +514,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dsk[2 * c4] = pack_bf16x2(v[0], v[1]);
         dsk[2 * c4 + 1] = pack_bf16x2(v[2], v[3]);
       }
-      // the previous dK / dQ MMAs must have finished reading dS^T
+      // the dS^T buffer is free once the previous tile's dK / dQ MMAs have read it
+      // and the dQ drain has finished staging through it
       if (it > 0 && !mbar_wait(&bars[kDSFree], (it - 1) & 1, abort_flag, p.err)) { ok = false; break; }
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
@@ -554,8 +585,18 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.drop_scale = a.drop_scale;
   p.seed_lo = a.seed_lo;
   p.seed_hi = a.seed_hi;
-  dim3 grid(a.B * a.H, a.N / 128);
-  kern<<<grid, kBwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmDO, p);
+  p.BH = a.B * a.H;
+  {
+    // heads per group: about 512 key-tile units per group; the CTAs running
+    // together then stream the same Q / dO tiles and add into the same dQ
+    // rows through L2, heaviest (lowest) key tiles first
+    const int n_t = a.N / 128;
+    p.group = (512 + n_t / 2) / n_t;
+    if (p.group < 1) p.group = 1;
+    if (p.group > p.BH) p.group = p.BH;
+  }
+  dim3 grid(a.B * a.H * (a.N / 128));
+  kern<<<grid, kBwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmDO, a.tmDQacc, p);
   return cudaGetLastError();
 }
 

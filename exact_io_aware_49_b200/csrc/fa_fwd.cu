@@ -108,6 +108,7 @@ struct FwdParams {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  int group, BH;
 };
 
 // S_q = Q_q * K^T : M = 128 query rows, N = 128 keys, K = D (both K-major).
@@ -156,10 +157,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;  // b * H + h
+  // 1-D grid over (head group, query block, head): within a group of
+  // p.group heads the heaviest causal blocks come first, and the blocks that
+  // run together share their heads' K and V through L2.
   const int N = p.N;
   const int n_qt = N / kBM;
-  const int qb = CAUSAL ? (gridDim.y - 1 - blockIdx.y) : blockIdx.y;
+  const int n_qb = (n_qt + 1) / 2;
+  // groups of p.group heads; inside a group, all heads' heaviest blocks first
+  const int per_group = p.group * n_qb;
+  const int grp = blockIdx.x / per_group;
+  const int r = blockIdx.x - grp * per_group;
+  const int gsz = min(p.group, p.BH - grp * p.group);
+  const int qb_lin = r / gsz;
+  const int bh = grp * p.group + (r - qb_lin * gsz);  // b * H + h
+  const int qb = CAUSAL ? (n_qb - 1 - qb_lin) : qb_lin;
   const int qt0 = 2 * qb;
   const int nq = min(2, n_qt - qt0);
   // key tiles each query tile visits (causal: up to and including its diagonal)
@@ -314,14 +325,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < kBN; ++c)
             if (c > r) s[c] = -CUDART_INF_F;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max over the 128 columns: four independent 3-input max chains
+        float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
+        float mx2 = fmaxf(s[4], s[5]), mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-        for (int c = 4; c < kBN; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 8; c < kBN; c += 8) {
+          mx0 = max3f(mx0, s[c], s[c + 1]);
+          mx1 = max3f(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3f(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3f(mx3, s[c + 6], s[c + 7]);
         }
+        static_assert(kBN % 8 == 0, "row max covers the tile in steps of 8");
         const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
         const float m_new = fmaxf(m, m_tile);
         if (__any_sync(0xffffffffu, m_new > m + kRescaleTau)) {
@@ -342,18 +356,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           m = m_new;
         }
-        const float neg_m = -m;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(-m, -m);
         uint32_t pk[64];
-        float rs0 = 0.f, rs1 = 0.f;
+        uint64_t rs0 = 0ull, rs1 = 0ull;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
-          rs0 += p0;
-          rs1 += p1;
+          float x0, x1;
+          f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          if (c & 1)
+            rs1 = add_f2(rs1, f2_pack(p0, p1));
+          else
+            rs0 = add_f2(rs0, f2_pack(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }
-        l += rs0 + rs1;
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(add_f2(rs0, rs1), a0, a1);
+          l += a0 + a1;
+          (void)b0;
+          (void)b1;
+        }
         if (DROPOUT) {
 #pragma unroll
           for (int g = 0; g < kBN / 8; ++g) {
@@ -420,8 +445,18 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   p.drop_scale = a.drop_scale;
   p.seed_lo = a.seed_lo;
   p.seed_hi = a.seed_hi;
+  p.BH = a.B * a.H;
+  {
+    // heads per group: about 256 work units (~2 waves on 148 SMs) per group,
+    // so the blocks running together share their heads' K and V in L2 while
+    // the heaviest causal blocks of the group still start first
+    const int n_qb = (a.N / kBM + 1) / 2;
+    p.group = (256 + n_qb / 2) / n_qb;
+    if (p.group < 1) p.group = 1;
+    if (p.group > p.BH) p.group = p.BH;
+  }
   const int n_qt = a.N / kBM;
-  dim3 grid(a.B * a.H, (n_qt + 1) / 2);
+  dim3 grid(a.B * a.H * ((n_qt + 1) / 2));
   kern<<<grid, kFwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
   return cudaGetLastError();
 }

@@ -23,6 +23,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // same layout as the forward maps
+  CUtensorMap tmDQacc;               // fp32 [B*H*N, d], 32-column x 128-row boxes, 128B swizzle
   const void* O;
   const void* dO;
   const float* LSE;
