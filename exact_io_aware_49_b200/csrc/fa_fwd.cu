@@ -24,9 +24,11 @@
 //  * the O rescale is lazy: the stale maximum is kept until a row's maximum
 //    grows by more than 8 (log2 units).  l and O share the stale maximum, so
 //    the result is unchanged; P stays <= 2^8;
-//  * dropout never stores a mask: keep bits come from Philox keyed on
-//    (seed, b, h, i, j); kept P are left unscaled and 1/(1-p) is folded into
-//    the final normalisation.
+//  * dropout never stores a mask: keep decisions come from Philox keyed on
+//    (seed, b, h, i, j), computed as 0.0 / 1.0 multipliers with one byte
+//    permute and one saturating add per element (the integer ALU pipe, which
+//    runs at half rate, is the bottleneck of this path); kept P are left
+//    unscaled and 1/(1-p) is folded into the final normalisation.
 //  * a causal CTA processes only key tiles up to its diagonal; the grid puts
 //    the heaviest query blocks first.
 #include <cuda.h>
@@ -302,7 +304,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t t_s = t_lane + q * 128;
       const uint32_t t_o = t_lane + 256 + q * D;
       const float sl2 = p.scale_log2;
-      const DropConst dk = make_drop_const(p.drop_t);
+      // keep test on the FMA pipe: for a 16-bit draw u, the float 2^23 + u is
+      // exact, and sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0
+      const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
       const int h = bh % p.H;
       const int b = bh / p.H;
       float m = -CUDART_INF_F;  // running max of scale*log2(e)*S, possibly stale
@@ -361,33 +365,41 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float x0, x1;
-          f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          if (c & 1)
-            rs1 = add_f2(rs1, f2_pack(p0, p1));
-          else
-            rs0 = add_f2(rs0, f2_pack(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        {
-          float a0, a1, b0, b1;
-          f2_unpack(add_f2(rs0, rs1), a0, a1);
-          l += a0 + a1;
-          (void)b0;
-          (void)b1;
-        }
-        if (DROPOUT) {
-#pragma unroll
-          for (int g = 0; g < kBN / 8; ++g) {
-            uint32_t w[4];
+        for (int g = 0; g < kBN / 8; ++g) {
+          uint32_t w[4];
+          if (DROPOUT)
             philox4x32_10(static_cast<uint32_t>(t * (kBN / 8) + g), static_cast<uint32_t>(i),
                           static_cast<uint32_t>(h), static_cast<uint32_t>(b), p.seed_lo, p.seed_hi, w);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) pk[g * 4 + e] &= keep_mask_2x16(w[e], dk);
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * g + e;
+            float x0, x1;
+            f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            uint64_t pp = f2_pack(p0, p1);
+            if (e & 1)
+              rs1 = add_f2(rs1, pp);
+            else
+              rs0 = add_f2(rs0, pp);
+            if (DROPOUT) {
+              // keep = sat((2^23 + u16) - (2^23 + t - 1)): exactly 1.0 if u16 >= t, else 0.0
+              const float u0 = __uint_as_float(prmt(w[e], 0x4B000000u, 0x7610u));
+              const float u1 = __uint_as_float(prmt(w[e], 0x4B000000u, 0x7632u));
+              float k0, k1;
+              asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k0) : "f"(u0), "f"(drop_bias));
+              asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(u1), "f"(drop_bias));
+              pp = mul_f2(pp, f2_pack(k0, k1));
+            }
+            float q0, q1;
+            f2_unpack(pp, q0, q1);
+            pk[c] = pack_bf16x2(q0, q1);
           }
+        }
+        {
+          float a0, a1;
+          f2_unpack(add_f2(rs0, rs1), a0, a1);
+          l += a0 + a1;
         }
         tmem_st32(t_s, pk);
         tmem_st32(t_s + 32, pk + 32);
