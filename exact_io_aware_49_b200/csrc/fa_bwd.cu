@@ -212,26 +212,55 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
   if (dealloc) tmem_dealloc(tmem, 512);
 }
 
-// Keep bits of the dropout mask for one key row and 8 consecutive queries
-// q0..q0+7.  The Philox counter (key >> 3, query, h, b) yields 8 keys x 1
-// query per call, so lane l of each group of 8 consecutive keys evaluates
-// query q0 + l, and 8 warp ballots transpose the 8 x 8 bit block: the result
-// has bit l set when (this lane's key, query q0 + l) is kept.
-__device__ __forceinline__ uint32_t keep_bits_8(uint32_t key_grp, uint32_t q0, uint32_t h, uint32_t b,
-                                                uint32_t seed_lo, uint32_t seed_hi, DropConst dk, int lane) {
-  const int l8 = lane & 7;
-  uint32_t w[4];
-  philox4x32_10(key_grp, q0 + l8, h, b, seed_lo, seed_hi, w);
-  uint32_t mine = 0;
+// Keep bits of the dropout mask for this lane's key row and 32 consecutive
+// queries q0 .. q0+31: bit l of the result is keep(key, q0 + l).
+//
+// The Philox counter (key >> 3, query, h, b) yields 8 keys x 1 query per call,
+// so lane l8 of each group of 8 consecutive keys evaluates queries
+// q0 + 8 j + l8 (j = 0..3).  Per output word the two 16-bit draws are tested
+// against t with three integer ops (the same two-lane test as the mask
+// export), and a multiply-high on the FMA pipe moves the two keep bits to
+// bits 2e and 16 + 2e of an accumulator.  That gives, per lane, four bytes
+// whose bit k' is keep(key 8 g + k', query q0 + 8 j + l8); a three-stage
+// butterfly of lane shuffles then transposes each 8 x 8 bit block so that lane
+// k' holds bit l = keep(its key, query q0 + 8 j + l).
+template <bool kHighT>
+__device__ __forceinline__ uint32_t keep_bits_32(uint32_t key_grp, uint32_t q0, uint32_t h, uint32_t b,
+                                                 uint32_t seed_lo, uint32_t seed_hi, uint32_t c2, int lane) {
+  const uint32_t l8 = static_cast<uint32_t>(lane & 7);
+  uint32_t W = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t w[4];
+    philox4x32_10(key_grp, q0 + 8 * j + l8, h, b, seed_lo, seed_hi, w);
+    uint32_t acc = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t y = (w[e] & 0x7FFF7FFFu) + c2;
+      const uint32_t zm = (kHighT ? (w[e] & y) : (w[e] | y)) & 0x80008000u;  // keep bits at 15 and 31
+      acc = mad_hi_u32(zm, 1u << (17 + 2 * e), acc);                          // -> bits 2e and 16 + 2e
+    }
+    W |= ((acc | (acc >> 15)) & 0xFFu) << (8 * j);
+  }
+#pragma unroll
+  for (int sh = 4; sh >= 1; sh >>= 1) {
+    const uint32_t lo = (sh == 4) ? 0x0F0F0F0Fu : ((sh == 2) ? 0x33333333u : 0x55555555u);
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, W, sh);
+    W = (l8 & sh) ? ((W & ~lo) | ((y >> sh) & lo)) : ((W & lo) | ((y << sh) & ~lo));
+  }
+  return W;
+}
+
+// Marks dropped entries by setting the sign bit of P: for 4 columns whose keep
+// bits are the low nibble of ``nib``, spreads the bits to the byte signs with
+// one multiply and turns each into a full-word mask with PRMT's sign mode.
+__device__ __forceinline__ void mark_dropped4(float* P, uint32_t nib) {
+  const uint32_t sp = (nib & 0xFu) * 0x10204080u;  // bit e -> bit 8 e + 7
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const uint32_t km = keep_mask_2x16(w[e], dk);
-    const uint32_t b_lo = __ballot_sync(0xffffffffu, (km & 1u) != 0);
-    const uint32_t b_hi = __ballot_sync(0xffffffffu, (km >> 31) != 0);
-    mine = (l8 == 2 * e) ? b_lo : mine;
-    mine = (l8 == 2 * e + 1) ? b_hi : mine;
+    const uint32_t keep = prmt(sp, 0u, 0x8888u + 0x1111u * e);
+    P[e] = __uint_as_float(__float_as_uint(P[e]) ^ (~keep & 0x80000000u));
   }
-  return (mine >> (lane & ~7)) & 0xFFu;
 }
 
 template <int D, bool CAUSAL, bool DROPOUT>
@@ -388,21 +417,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!*go) break;
       tc_fence_after();
       const int qrow = row0 + (q_first + it) * 128;
+      // chunk 0 is staged into shared memory before chunk 1 leaves TMEM, so
+      // TMEM is released after two loads and one set of stores -- before any
+      // wait on the reduce engine.
+      uint32_t v[64];
+      tmem_ld32(t_row, v);
+      tmem_ld32(t_row + 32, v + 32);
+      tmem_ld_wait();
+      reg_fence32(v);
+      reg_fence32(v + 32);
+      if (D == 64) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kDQFree]);  // all of dQ is out of TMEM
+      }
 #pragma unroll
       for (int ch = 0; ch < D / 64; ++ch) {
-        uint32_t v[64];
-        tmem_ld32(t_row + ch * 64, v);
-        tmem_ld32(t_row + ch * 64 + 32, v + 32);
-        tmem_ld_wait();
-        reg_fence32(v);
-        reg_fence32(v + 32);
-        if (ch == D / 64 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[kDQFree]);
-        }
-        // the previous chunk's reduce has finished reading the staging buffer
-        if (ch > 0) asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (ch > 0) asm volatile("bar.sync 2, 128;" ::: "memory");  // previous reduce has read the buffer
 #pragma unroll
         for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
@@ -410,6 +441,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             st_shared_v4(st_row + bx * L::kBox + ((q4 ^ (c & 7)) << 4), v[32 * bx + 4 * q4],
                          v[32 * bx + 4 * q4 + 1], v[32 * bx + 4 * q4 + 2], v[32 * bx + 4 * q4 + 3]);
         fence_proxy_async_smem();
+        if (ch + 1 < D / 64) {
+          tmem_ld32(t_row + (ch + 1) * 64, v);
+          tmem_ld32(t_row + (ch + 1) * 64 + 32, v + 32);
+          tmem_ld_wait();
+          reg_fence32(v);
+          reg_fence32(v + 32);
+          if (ch + 2 == D / 64) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[kDQFree]);  // all of dQ is out of TMEM
+          }
+        }
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader) {
           tma_reduce_add_2d(&tmDQ, smem + L::kDS, ch * 64, qrow);
@@ -431,6 +474,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
     const DropConst dk = make_drop_const(p.drop_t);
+    const bool hi_t = p.drop_t > 0x8000u;
     const uint32_t hh = static_cast<uint32_t>(bh % p.H), bb = static_cast<uint32_t>(bh / p.H);
     const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
     const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
@@ -464,26 +508,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < 64; ++c)
           if (64 * g + c < r) P[c] = 0.f;
       }
-      uint32_t zb[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
       if (DROPOUT) {
+        // dropped entries get the sign bit set; dS and the bf16 pack read it
         const uint32_t q0 = static_cast<uint32_t>(qi * 128 + 64 * g);
 #pragma unroll
-        for (int bq = 0; bq < 8; ++bq) {
-          const uint32_t bits = keep_bits_8(key_grp, q0 + 8 * bq, hh, bb, p.seed_lo, p.seed_hi, dk, lane);
-          if (bq % 4 == 0) zb[bq / 4] = 0;
-          zb[bq / 4] |= bits << (8 * (bq % 4));
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t zb = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane)
+                                   : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane);
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) mark_dropped4(P + 32 * half + 4 * k4, zb >> (4 * k4));
         }
       }
       uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float a = P[2 * c], b2 = P[2 * c + 1];
-        if (DROPOUT) {
-          a = ((zb[c / 16] >> ((2 * c) % 32)) & 1u) ? a : 0.f;
-          b2 = ((zb[c / 16] >> ((2 * c + 1) % 32)) & 1u) ? b2 : 0.f;
-        }
-        pk[c] = pack_bf16x2(a, b2);
-      }
+      for (int c = 0; c < 32; ++c)
+        pk[c] = DROPOUT ? pack_bf16x2_relu(P[2 * c], P[2 * c + 1]) : pack_bf16x2(P[2 * c], P[2 * c + 1]);
       tmem_st32(t_row + kColS + 32 * g, pk);
       tmem_st_wait();
       tc_fence_before();
@@ -507,9 +546,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = 4 * c4 + e;
-          float dp = __uint_as_float(dr[c]);
-          if (DROPOUT) dp = ((zb[c / 32] >> (c % 32)) & 1u) ? dp * p.drop_scale : 0.f;
-          v[e] = P[c] * (dp - dd[e]);
+          const float dp = __uint_as_float(dr[c]);
+          // kept: P (dP / (1-p) - D); dropped (sign set): -|P| D
+          v[e] = DROPOUT ? fmaxf(P[c], 0.f) * (dp * p.drop_scale) - fabsf(P[c]) * dd[e] : P[c] * (dp - dd[e]);
         }
         dsk[2 * c4] = pack_bf16x2(v[0], v[1]);
         dsk[2 * c4 + 1] = pack_bf16x2(v[2], v[3]);
