@@ -50,6 +50,8 @@ def load_library(path=None):
     lib.fa_bwd_finish.restype = i
     lib.fa_dropout_mask.argtypes = [vp, i, i, i, f, u64, vp]
     lib.fa_dropout_mask.restype = i
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+    lib.fa_selftest_wait_timeout.restype = i
     lib.fa_last_device_error.argtypes = []
     lib.fa_last_device_error.restype = i
     lib.fa_status_string.argtypes = [i]
@@ -164,6 +166,13 @@ def fa_dropout_mask(B, H, N, p_drop, seed, device="cuda"):
     st = lib.fa_dropout_mask(mask.data_ptr(), B, H, N, float(p_drop), int(seed) & (2**64 - 1), _stream(mask))
     _raise(st, "fa_dropout_mask")
     return mask
+
+
+def fa_selftest_wait_timeout(limit_us=1000, device="cuda"):
+    """Runs the bounded-wait self-test kernel (a wait that can only time out)."""
+    lib = load_library()
+    st = torch.cuda.current_stream(torch.device(device))
+    _raise(lib.fa_selftest_wait_timeout(int(limit_us), ctypes.c_void_p(st.cuda_stream)), "fa_selftest_wait_timeout")
 
 
 def fa_last_device_error():

@@ -265,6 +265,15 @@ fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint
              : FA_ERR_CUDA;
 }
 
+fa_status fa_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return FA_ERR_INVALID_ARG;
+  unsigned* err = error_word_ptr();
+  if (!err) return FA_ERR_CUDA;
+  return fa::launch_wait_timeout_probe(err, 1000ull * limit_us, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
 fa_status fa_last_device_error(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
   unsigned v = 0;

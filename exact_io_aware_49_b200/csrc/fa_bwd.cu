@@ -25,7 +25,8 @@
 //        dK += dS^T Q_i ;  dQ_i = dS K_j  (the same smem tile read K-major
 //              for dK and MN-major for dQ)
 //        dQ_i is read out of TMEM by a dedicated warpgroup, staged through the
-//        dS^T buffer and added to the fp32 accumulator with TMA reduce-add.
+//        tile's dO buffer (idle by then) and added to the fp32 accumulator
+//        with TMA reduce-add.
 //      Warp roles: warpgroups 0/1 do the elementwise work for query columns
 //      0-63 / 64-127 (one thread per key row, the TMEM lane); warp 8 issues
 //      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
@@ -125,7 +126,7 @@ struct BwdSmem {
   static constexpr int kDS = 6 * kTile;     // dS^T: 128 keys x 128 queries bf16 = 2 boxes
   static constexpr int kVec = kDS + 2 * kBox;  // 2 stages x (LSE2[128], D[128]) fp32
   static constexpr int kBar = kVec + 2 * 1024;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 18;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kUsed = kMisc + 16;
 };
@@ -144,6 +145,7 @@ enum BwdBar {
   kDQFree = 13,
   kDKDVReady = 14,
   kDrain = 15,
+  kDOStage0 = 16,  // +stage: the dQ drain has finished staging through that dO buffer
 };
 
 struct BwdParams {
@@ -335,10 +337,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tma_load_2d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, qrow, &bars[kQFull0 + s]);
         bulk_load_1d(smem + L::kVec + s * 1024, p.lse2 + qrow, 512, &bars[kQFull0 + s]);
         bulk_load_1d(smem + L::kVec + s * 1024 + 512, p.Dvec + qrow, 512, &bars[kQFull0 + s]);
+        issued = it + 1;
+        // the dO buffer doubles as the dQ drain's staging area two tiles back
+        if (it >= 2 && !mbar_wait(&bars[kDOStage0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kDOFull0 + s], L::kTile);
         for (int c = 0; c < D / 64; ++c)
           tma_load_2d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, qrow, &bars[kDOFull0 + s]);
-        issued = it + 1;
       }
       if (*abort_flag) {
         mbar_wait_drain(&bars[kKVFull], 0);
@@ -380,6 +384,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(&bars[kEmpty0 + s]);
         mma_dq<D>(tmem + kColDP, sm_ds, sm_k);
         mma_commit(&bars[kDQReady]);
+        mma_commit(&bars[kDSFree]);
         if (more) {
           if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
               !mbar_wait(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -399,69 +404,64 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_teardown(tmem, warp == kBwdMmaWarp);
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain
-    // dQ_i leaves TMEM 64 columns at a time: staged as two 32-column fp32
-    // boxes in the dS^T buffer (free once dK_i and dQ_i have read it) and added
-    // into the fp32 accumulator by TMA reduce-add.  TMEM is released right after
-    // the last load, so the next dP^T MMA does not wait for the reductions.
+    // dQ_i leaves TMEM in two rounds of D/2 columns.  Each round is staged as
+    // 32-column fp32 boxes (128-byte swizzled rows) in the dO buffer of this
+    // tile -- idle since dV_i and dP^T_i read it, and not refilled until the
+    // drain releases it -- and added into the fp32 accumulator by TMA
+    // reduce-add.  TMEM is released right after the second load.
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kDqRegs));
+    constexpr int kCols = D / 2;       // columns per round
+    constexpr int kBoxes = kCols / 32;  // 32-column fp32 boxes per round
     const int wq = warp & 3;
     const int c = wq * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kColDP;
     const bool leader = threadIdx.x == 12 * 32;
     volatile int* go = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-    const uint32_t st_row = sm_ds + c * 128;
     for (int it = 0; it < nq; ++it) {
       // one thread waits (bounded); the named barrier hands its verdict to all 128
       if (leader) *go = mbar_wait(&bars[kDQReady], it & 1, abort_flag, p.err) ? 1 : 0;
       asm volatile("bar.sync 2, 128;" ::: "memory");
       if (!*go) break;
       tc_fence_after();
+      const int s = it & 1;
       const int qrow = row0 + (q_first + it) * 128;
-      // chunk 0 is staged into shared memory before chunk 1 leaves TMEM, so
-      // TMEM is released after two loads and one set of stores -- before any
-      // wait on the reduce engine.
-      uint32_t v[64];
-      tmem_ld32(t_row, v);
-      tmem_ld32(t_row + 32, v + 32);
+      uint8_t* stage = smem + L::kDO + s * L::kTile;
+      const uint32_t st_row = smem_u32(stage) + c * 128;
+      uint32_t v[kCols];
+#pragma unroll
+      for (int k = 0; k < kCols / 32; ++k) tmem_ld32(t_row + 32 * k, v + 32 * k);
       tmem_ld_wait();
-      reg_fence32(v);
-      reg_fence32(v + 32);
-      if (D == 64) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kDQFree]);  // all of dQ is out of TMEM
-      }
 #pragma unroll
-      for (int ch = 0; ch < D / 64; ++ch) {
-        if (ch > 0) asm volatile("bar.sync 2, 128;" ::: "memory");  // previous reduce has read the buffer
+      for (int k = 0; k < kCols / 32; ++k) reg_fence32(v + 32 * k);
 #pragma unroll
-        for (int bx = 0; bx < 2; ++bx)
+      for (int r = 0; r < 2; ++r) {
+        if (r > 0) asm volatile("bar.sync 2, 128;" ::: "memory");  // round 0's reduce has read the buffer
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx)
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4)
             st_shared_v4(st_row + bx * L::kBox + ((q4 ^ (c & 7)) << 4), v[32 * bx + 4 * q4],
                          v[32 * bx + 4 * q4 + 1], v[32 * bx + 4 * q4 + 2], v[32 * bx + 4 * q4 + 3]);
         fence_proxy_async_smem();
-        if (ch + 1 < D / 64) {
-          tmem_ld32(t_row + (ch + 1) * 64, v);
-          tmem_ld32(t_row + (ch + 1) * 64 + 32, v + 32);
+        if (r == 0) {
+#pragma unroll
+          for (int k = 0; k < kCols / 32; ++k) tmem_ld32(t_row + kCols + 32 * k, v + 32 * k);
           tmem_ld_wait();
-          reg_fence32(v);
-          reg_fence32(v + 32);
-          if (ch + 2 == D / 64) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[kDQFree]);  // all of dQ is out of TMEM
-          }
+#pragma unroll
+          for (int k = 0; k < kCols / 32; ++k) reg_fence32(v + 32 * k);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[kDQFree]);  // all of dQ is out of TMEM
         }
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader) {
-          tma_reduce_add_2d(&tmDQ, smem + L::kDS, ch * 64, qrow);
-          tma_reduce_add_2d(&tmDQ, smem + L::kDS + L::kBox, ch * 64 + 32, qrow);
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) tma_reduce_add_2d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, qrow);
           bulk_commit_group();
           bulk_wait_group_read0();
         }
       }
-      if (leader) mbar_arrive(&bars[kDSFree]);  // staging done: dS^T of the next tile may be written
+      if (leader) mbar_arrive(&bars[kDOStage0 + s]);  // the dO buffer may be refilled
     }
     if (leader) bulk_wait_group0();
     bwd_teardown(tmem, false);
@@ -554,7 +554,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         dsk[2 * c4 + 1] = pack_bf16x2(v[2], v[3]);
       }
       // the dS^T buffer is free once the previous tile's dK / dQ MMAs have read it
-      // and the dQ drain has finished staging through it
       if (it > 0 && !mbar_wait(&bars[kDSFree], (it - 1) & 1, abort_flag, p.err)) { ok = false; break; }
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)

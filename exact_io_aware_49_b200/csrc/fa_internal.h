@@ -49,6 +49,7 @@ cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream);  // O, dO, LSE -> Dvec, lse2, dQacc = 0
 cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream);    // maps, lse2, Dvec -> dK, dV, dQacc
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream);   // dQacc -> dQ
+cudaError_t launch_wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_dropout_mask(uint8_t* mask, int B, int H, int N, uint32_t drop_t, uint32_t seed_lo,
                                 uint32_t seed_hi, cudaStream_t stream);
 

@@ -37,7 +37,28 @@ __global__ void fa_dropout_mask_kernel(uint8_t* mask, int H, int N, uint32_t t, 
   }
 }
 
+// Failure-detection self-test: one warp waits on an mbarrier that nothing will
+// ever arrive on, with a wait limit of ``limit_ns``; the bounded wait gives up,
+// records the timeout bit in the device error word and returns.
+__global__ void fa_wait_timeout_probe_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, limit_ns);
+  __syncthreads();
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream) {
+  fa_wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dropout_mask(uint8_t* mask, int B, int H, int N, uint32_t drop_t, uint32_t seed_lo,
                                 uint32_t seed_hi, cudaStream_t stream) {

@@ -183,6 +183,17 @@ fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint
  */
 fa_status fa_last_device_error(void);
 
+/*
+ * Failure-detection self-test: enqueues one tiny kernel whose single bounded
+ * wait is on a barrier that nothing ever completes, with a limit of
+ * ``limit_us`` microseconds (1 .. 1000000).  The wait gives up, records a
+ * timeout in the device error word and the kernel returns normally, so the
+ * next fa_last_device_error() reports FA_ERR_TIMEOUT and the CUDA context
+ * stays usable.  It exercises the same bounded-wait code the attention
+ * kernels use; it never faults or hangs the device.
+ */
+fa_status fa_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status status);
 

@@ -107,6 +107,11 @@ def test_stage_entry_points_reject_bad_arguments(lib):
     assert lib.fa_bwd_finish(A, 1, 1, 128, 64, -1.0, A, ws_ok, None) == 1
 
 
+def test_selftest_rejects_bad_limits_before_any_cuda_call(lib):
+    assert lib.fa_selftest_wait_timeout(0, None) == 1
+    assert lib.fa_selftest_wait_timeout(1000001, None) == 1
+
+
 def test_mask_rejects_bad_arguments(lib):
     assert lib.fa_dropout_mask(None, 1, 1, 8, 0.1, 0, None) == 1
     assert lib.fa_dropout_mask(A, 0, 1, 8, 0.1, 0, None) == 1
