@@ -478,6 +478,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t hh = static_cast<uint32_t>(bh % p.H), bb = static_cast<uint32_t>(bh / p.H);
     const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
     const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
+    // keep bits of this thread's 64 query columns for the coming query tile;
+    // computed one tile ahead, while the warp would otherwise wait for S^T
+    uint32_t zb[2] = {0u, 0u};
+    auto keep_bits_tile = [&](int qi_next) {
+      const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g);
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        zb[half] = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane)
+                        : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane);
+    };
+    if (DROPOUT) keep_bits_tile(q_first);
     bool ok = true;
     for (int it = 0; it < nq; ++it) {
       const int s = it & 1;
@@ -510,14 +521,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (DROPOUT) {
         // dropped entries get the sign bit set; dS and the bf16 pack read it
-        const uint32_t q0 = static_cast<uint32_t>(qi * 128 + 64 * g);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t zb = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane)
-                                   : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane);
+        for (int half = 0; half < 2; ++half)
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) mark_dropped4(P + 32 * half + 4 * k4, zb >> (4 * k4));
-        }
+          for (int k4 = 0; k4 < 8; ++k4) mark_dropped4(P + 32 * half + 4 * k4, zb[half] >> (4 * k4));
       }
       uint32_t pk[32];
 #pragma unroll
@@ -563,6 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kDSReady]);
+      if (DROPOUT && it + 1 < nq) keep_bits_tile(qi + 1);
     }
     if (ok && mbar_wait(&bars[kDKDVReady], 0, abort_flag, p.err)) {
       // -------------------------------------------------------------- dK / dV epilogue
