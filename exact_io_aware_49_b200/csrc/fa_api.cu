@@ -34,24 +34,21 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows, d] row-major 2-D map with 128-byte boxes per row (64 bf16 or 32 fp32
-// columns) x 128 rows and 128-byte swizzle.
-bool encode_rows_map_t(CUtensorMap* tm, const void* base, long long rows, int d, bool fp32) {
+// [BH, N, d] row-major 3-D map with 128-byte boxes per row (64 bf16 or 32
+// fp32 columns) x 128 rows x 1 head and 128-byte swizzle.  Rows past N of a
+// head are outside the tensor: loads zero-fill them, reductions skip them.
+bool encode_head_map(CUtensorMap* tm, const void* base, long long BH, int N, int d, bool fp32) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t esize = fp32 ? 4 : 2;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * esize};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(N) * d * esize};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
-}
-
-bool encode_rows_map(CUtensorMap* tm, const void* base, long long rows, int d) {
-  return encode_rows_map_t(tm, base, rows, d, false);
 }
 
 unsigned* error_word_ptr() {
@@ -75,7 +72,6 @@ fa_status check_common(int B, int H, int N, int d, float scale, float p_drop) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * H * N;
   if (rows >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
@@ -111,9 +107,9 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 
   fa::FwdArgs a;
   memset(&a, 0, sizeof(a));
-  const long long rows = static_cast<long long>(B) * H * N;
-  if (!encode_rows_map(&a.tmQ, Q, rows, d) || !encode_rows_map(&a.tmK, K, rows, d) ||
-      !encode_rows_map(&a.tmV, V, rows, d))
+  const long long BH = static_cast<long long>(B) * H;
+  if (!encode_head_map(&a.tmQ, Q, BH, N, d, false) || !encode_head_map(&a.tmK, K, BH, N, d, false) ||
+      !encode_head_map(&a.tmV, V, BH, N, d, false))
     return FA_ERR_CUDA;
   a.O = O;
   a.LSE = LSE;
@@ -135,7 +131,8 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
-  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(rows * sizeof(float), 256);
+  const size_t rows_pad = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
+  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(rows_pad * sizeof(float), 256);
 }
 
 }  // extern "C"
@@ -146,8 +143,9 @@ namespace {
 void carve_workspace(fa::BwdArgs* a, void* workspace) {
   char* ws = static_cast<char*>(workspace);
   const size_t rows = static_cast<size_t>(a->B) * a->H * a->N;
+  const size_t rows_pad = static_cast<size_t>(a->B) * a->H * ((static_cast<size_t>(a->N) + 127) / 128 * 128);
   const size_t acc_bytes = round_up(rows * a->d * sizeof(float), 256);
-  const size_t vec_bytes = round_up(rows * sizeof(float), 256);
+  const size_t vec_bytes = round_up(rows_pad * sizeof(float), 256);
   a->dQacc = reinterpret_cast<float*>(ws);
   a->Dvec = reinterpret_cast<float*>(ws + acc_bytes);
   a->lse2 = reinterpret_cast<float*>(ws + acc_bytes + vec_bytes);
@@ -207,13 +205,13 @@ fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* 
   if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
   fa::BwdArgs a;
   memset(&a, 0, sizeof(a));
-  const long long rows = static_cast<long long>(B) * H * N;
-  if (!encode_rows_map(&a.tmQ, Q, rows, d) || !encode_rows_map(&a.tmK, K, rows, d) ||
-      !encode_rows_map(&a.tmV, V, rows, d) || !encode_rows_map(&a.tmDO, dO, rows, d))
+  const long long BH = static_cast<long long>(B) * H;
+  if (!encode_head_map(&a.tmQ, Q, BH, N, d, false) || !encode_head_map(&a.tmK, K, BH, N, d, false) ||
+      !encode_head_map(&a.tmV, V, BH, N, d, false) || !encode_head_map(&a.tmDO, dO, BH, N, d, false))
     return FA_ERR_CUDA;
   fill_scalars(&a, B, H, N, d, causal, scale, p_drop, seed);
   carve_workspace(&a, workspace);
-  if (!encode_rows_map_t(&a.tmDQacc, a.dQacc, rows, d, true)) return FA_ERR_CUDA;
+  if (!encode_head_map(&a.tmDQacc, a.dQacc, BH, N, d, true)) return FA_ERR_CUDA;
   a.dO = dO;
   a.dK = dK;
   a.dV = dV;

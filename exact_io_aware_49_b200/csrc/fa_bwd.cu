@@ -46,19 +46,32 @@ namespace {
 
 // ============================================================ preprocess
 
-// One warp per row: D = sum(dO * O), LSE2 = LSE * log2(e), dQacc row = 0.
+// One warp per padded row (b*H + h, i < Npad): for i < N, D = sum(dO * O),
+// LSE2 = LSE * log2(e) and the dQ accumulator row is zeroed; for the padding
+// rows of a partial last tile, D = 0 and LSE2 = +inf (so exp2(x - LSE2) = 0).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ O,
                                                                 const __nv_bfloat16* __restrict__ dO,
                                                                 const float* __restrict__ LSE,
                                                                 float* __restrict__ Dvec,
                                                                 float* __restrict__ lse2,
-                                                                float* __restrict__ dQacc, long long rows) {
+                                                                float* __restrict__ dQacc, long long rows_pad,
+                                                                int N, int Npad) {
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long row = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
-       row += warps) {
-    // D / 8 lanes active per 16-byte chunk: lane covers elements [8*lane, 8*lane+8) when 8*lane < D
+  for (long long prow = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); prow < rows_pad;
+       prow += warps) {
+    const long long bh = prow / Npad;
+    const int i = static_cast<int>(prow - bh * Npad);
+    if (i >= N) {
+      if (lane == 0) {
+        Dvec[prow] = 0.f;
+        lse2[prow] = CUDART_INF_F;
+      }
+      continue;
+    }
+    const long long row = bh * N + i;
+    // lane covers elements [8*lane, 8*lane+8) when 8*lane < D
     float acc = 0.f;
     if (lane * 8 < D) {
       const uint4 a = *reinterpret_cast<const uint4*>(O + row * D + lane * 8);
@@ -78,8 +91,8 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
     float4* zq = reinterpret_cast<float4*>(dQacc + row * D);
     for (int c = lane; c < D / 4; c += 32) zq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane == 0) {
-      Dvec[row] = acc;
-      lse2[row] = LSE[row] * 1.4426950408889634f;
+      Dvec[prow] = acc;
+      lse2[prow] = LSE[row] * 1.4426950408889634f;
     }
   }
 }
@@ -283,7 +296,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // 1-D grid over (head group, key tile, head), heaviest key tiles first
   // within each group of p.group heads.
   const int N = p.N;
-  const int n_t = N / 128;
+  const int n_t = (N + 127) / 128;  // the last tile may be partial
+  const int Npad = n_t * 128;
   const int per_group = p.group * n_t;
   const int grp = blockIdx.x / per_group;
   const int rr = blockIdx.x - grp * per_group;
@@ -292,7 +306,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int bh = grp * p.group + (rr - kj * gsz);
   const int q_first = CAUSAL ? kj : 0;
   const int nq = n_t - q_first;              // query tiles visited
-  const int row0 = bh * N;
+  const size_t vrow0 = static_cast<size_t>(bh) * Npad;  // this head's rows in the padded LSE2 / D vectors
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -324,25 +338,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(&bars[kKVFull], 2 * L::kTile);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(smem + L::kK + c * L::kBox, &tmK, c * 64, row0 + kj * 128, &bars[kKVFull]);
-        tma_load_2d(smem + L::kV + c * L::kBox, &tmV, c * 64, row0 + kj * 128, &bars[kKVFull]);
+        tma_load_3d(smem + L::kK + c * L::kBox, &tmK, c * 64, kj * 128, bh, &bars[kKVFull]);
+        tma_load_3d(smem + L::kV + c * L::kBox, &tmV, c * 64, kj * 128, bh, &bars[kKVFull]);
       }
       int issued = 0;
       for (int it = 0; it < nq; ++it) {
         const int s = it & 1;
-        const int qrow = row0 + (q_first + it) * 128;
+        const int qrow = (q_first + it) * 128;  // first query row of the tile within the head
         if (it >= 2 && !mbar_wait(&bars[kEmpty0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kQFull0 + s], L::kTile + 1024);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, qrow, &bars[kQFull0 + s]);
-        bulk_load_1d(smem + L::kVec + s * 1024, p.lse2 + qrow, 512, &bars[kQFull0 + s]);
-        bulk_load_1d(smem + L::kVec + s * 1024 + 512, p.Dvec + qrow, 512, &bars[kQFull0 + s]);
+          tma_load_3d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, qrow, bh, &bars[kQFull0 + s]);
+        bulk_load_1d(smem + L::kVec + s * 1024, p.lse2 + vrow0 + qrow, 512, &bars[kQFull0 + s]);
+        bulk_load_1d(smem + L::kVec + s * 1024 + 512, p.Dvec + vrow0 + qrow, 512, &bars[kQFull0 + s]);
         issued = it + 1;
         // the dO buffer doubles as the dQ drain's staging area two tiles back
         if (it >= 2 && !mbar_wait(&bars[kDOStage0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kDOFull0 + s], L::kTile);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, qrow, &bars[kDOFull0 + s]);
+          tma_load_3d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, qrow, bh, &bars[kDOFull0 + s]);
       }
       if (*abort_flag) {
         mbar_wait_drain(&bars[kKVFull], 0);
@@ -424,7 +438,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!*go) break;
       tc_fence_after();
       const int s = it & 1;
-      const int qrow = row0 + (q_first + it) * 128;
+      const int qrow = (q_first + it) * 128;
       uint8_t* stage = smem + L::kDO + s * L::kTile;
       const uint32_t st_row = smem_u32(stage) + c * 128;
       uint32_t v[kCols];
@@ -456,7 +470,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader) {
 #pragma unroll
-          for (int bx = 0; bx < kBoxes; ++bx) tma_reduce_add_2d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, qrow);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, qrow, bh);  // rows past N skipped
           bulk_commit_group();
           bulk_wait_group_read0();
         }
@@ -477,6 +492,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool hi_t = p.drop_t > 0x8000u;
     const uint32_t hh = static_cast<uint32_t>(bh % p.H), bb = static_cast<uint32_t>(bh / p.H);
     const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
+    const bool key_valid = kj * 128 + r < N;
     const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
     // keep bits of this thread's 64 query columns for the coming query tile;
     // computed one tile ahead, while the warp would otherwise wait for S^T
@@ -513,11 +529,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         P[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l4.z));
         P[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l4.w));
       }
-      if (CAUSAL && qi == kj) {
-        // query 64 g + c precedes key r: masked
+      // masked: queries before this key on the diagonal tile (causal), and the
+      // whole row for a key past N (queries past N already get LSE2 = +inf)
+      if ((CAUSAL && qi == kj) || !key_valid) {
+        const int lo = key_valid ? r : 128;  // columns 64 g + c < lo are zeroed
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (64 * g + c < r) P[c] = 0.f;
+          if (64 * g + c < lo) P[c] = 0.f;
       }
       if (DROPOUT) {
         // dropped entries get the sign bit set; dS and the bf16 pack read it
@@ -577,7 +595,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint32_t col = (g == 0) ? kColDK : kColDV;
       const float mul = (g == 0) ? p.scale : p.drop_scale;
-      __nv_bfloat16* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(row0) + kj * 128 + r) * D;
+      __nv_bfloat16* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(bh) * N + kj * 128 + r) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -588,9 +606,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+        if (key_valid) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+        }
       }
     }
     bwd_teardown(tmem, false);
@@ -636,12 +656,12 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
     // heads per group: about 512 key-tile units per group; the CTAs running
     // together then stream the same Q / dO tiles and add into the same dQ
     // rows through L2, heaviest (lowest) key tiles first
-    const int n_t = a.N / 128;
+    const int n_t = (a.N + 127) / 128;
     p.group = (512 + n_t / 2) / n_t;
     if (p.group < 1) p.group = 1;
     if (p.group > p.BH) p.group = p.BH;
   }
-  dim3 grid(a.B * a.H * (a.N / 128));
+  dim3 grid(a.B * a.H * ((a.N + 127) / 128));
   kern<<<grid, kBwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmDO, a.tmDQacc, p);
   return cudaGetLastError();
 }
@@ -649,17 +669,18 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
-  const long long rows = static_cast<long long>(a.B) * a.H * a.N;
-  long long blocks = (rows + 7) / 8;  // one warp per row, 8 warps per block
+  const int Npad = (a.N + 127) / 128 * 128;
+  const long long rows_pad = static_cast<long long>(a.B) * a.H * Npad;
+  long long blocks = (rows_pad + 7) / 8;  // one warp per row, 8 warps per block
   if (blocks > 148 * 16) blocks = 148 * 16;
   const __nv_bfloat16* O = static_cast<const __nv_bfloat16*>(a.O);
   const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(a.dO);
   if (a.d == 64)
     fa_bwd_preprocess_kernel<64><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                               a.dQacc, rows);
+                                                                               a.dQacc, rows_pad, a.N, Npad);
   else
     fa_bwd_preprocess_kernel<128><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                a.dQacc, rows);
+                                                                                a.dQacc, rows_pad, a.N, Npad);
   return cudaGetLastError();
 }
 

@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // p.group heads the heaviest causal blocks come first, and the blocks that
   // run together share their heads' K and V through L2.
   const int N = p.N;
-  const int n_qt = N / kBM;
+  const int n_qt = (N + kBM - 1) / kBM;  // the last tile may be partial
   const int n_qb = (n_qt + 1) / 2;
   // groups of p.group heads; inside a group, all heads' heaviest blocks first
   const int per_group = p.group * n_qb;
@@ -218,11 +218,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int row0 = bh * N;
+      // 3-D coordinates (column, row within the head, head): rows past N read as zeros
       mbar_expect_tx(bar.q, nq * L::kTileBytes);
       for (int q = 0; q < nq; ++q)
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(smem + L::kQ + q * L::kTileBytes + c * L::kBoxBytes, &tmQ, c * 64, row0 + (qt0 + q) * kBM,
+          tma_load_3d(smem + L::kQ + q * L::kTileBytes + c * L::kBoxBytes, &tmQ, c * 64, (qt0 + q) * kBM, bh,
                       bar.q);
       int issued = 0;
       for (int t = 0; t < nt_all; ++t) {
@@ -230,11 +230,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (t >= S && !mbar_wait(&bar.kvempty[s], ((t / S) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bar.kfull[s], L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(smem + L::kK + s * L::kTileBytes + c * L::kBoxBytes, &tmK, c * 64, row0 + t * kBN,
+          tma_load_3d(smem + L::kK + s * L::kTileBytes + c * L::kBoxBytes, &tmK, c * 64, t * kBN, bh,
                       &bar.kfull[s]);
         mbar_expect_tx(&bar.vfull[s], L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(smem + L::kV + s * L::kTileBytes + c * L::kBoxBytes, &tmV, c * 64, row0 + t * kBN,
+          tma_load_3d(smem + L::kV + s * L::kTileBytes + c * L::kBoxBytes, &tmV, c * 64, t * kBN, bh,
                       &bar.vfull[s]);
         issued = t + 1;
       }
@@ -324,10 +324,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float s[kBN];
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
-        if (CAUSAL && t == ntile[q] - 1) {
+        // masked columns: keys after this row on the diagonal tile (causal) and
+        // keys past N on a partial last tile; both are c > lim for one limit
+        const int jv = N - t * kBN;  // keys of this tile inside the sequence
+        if ((CAUSAL && t == ntile[q] - 1) || jv < kBN) {
+          const int lim = min((CAUSAL && t == ntile[q] - 1) ? r : kBN - 1, jv - 1);
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
-            if (c > r) s[c] = -CUDART_INF_F;
+            if (c > lim) s[c] = -CUDART_INF_F;
         }
         // row max over the 128 columns: four independent 3-input max chains
         float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
@@ -423,12 +427,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             packed[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
+          if (i < N) {  // rows of a partial last tile past N are computed but not stored
+            uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+          }
         }
-        p.LSE[static_cast<size_t>(bh) * N + i] = (m + lg2_approx(l)) * 0.69314718055994531f;
+        if (i < N) p.LSE[static_cast<size_t>(bh) * N + i] = (m + lg2_approx(l)) * 0.69314718055994531f;
       }
     }
     cta_teardown(tmem, false);
@@ -462,12 +468,12 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
     // heads per group: about 256 work units (~2 waves on 148 SMs) per group,
     // so the blocks running together share their heads' K and V in L2 while
     // the heaviest causal blocks of the group still start first
-    const int n_qb = (a.N / kBM + 1) / 2;
+    const int n_qb = ((a.N + kBM - 1) / kBM + 1) / 2;
     p.group = (256 + n_qb / 2) / n_qb;
     if (p.group < 1) p.group = 1;
     if (p.group > p.BH) p.group = p.BH;
   }
-  const int n_qt = a.N / kBM;
+  const int n_qt = (a.N + kBM - 1) / kBM;
   dim3 grid(a.B * a.H * ((n_qt + 1) / 2));
   kern<<<grid, kFwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
   return cudaGetLastError();

@@ -9,7 +9,7 @@
 namespace fa {
 
 struct FwdArgs {
-  CUtensorMap tmQ, tmK, tmV;  // 2-D maps over [B*H*N, d] bf16, 64 x 128 boxes, 128B swizzle
+  CUtensorMap tmQ, tmK, tmV;  // 3-D maps over [B*H, N, d] bf16, 64 x 128 x 1 boxes, 128B swizzle
   void* O;                    // bf16 [B, H, N, d]
   float* LSE;                 // fp32 [B, H, N]
   unsigned* err;              // device error word
@@ -23,7 +23,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // same layout as the forward maps
-  CUtensorMap tmDQacc;               // fp32 [B*H*N, d], 32-column x 128-row boxes, 128B swizzle
+  CUtensorMap tmDQacc;               // fp32 [B*H, N, d], 32-column x 128-row boxes, 128B swizzle
   const void* O;
   const void* dO;
   const float* LSE;
@@ -31,8 +31,8 @@ struct BwdArgs {
   void* dK;
   void* dV;
   float* dQacc;  // fp32 [B, H, N, d] workspace
-  float* Dvec;   // fp32 [B, H, N] workspace: rowsum(dO * O)
-  float* lse2;   // fp32 [B, H, N] workspace: LSE * log2(e)
+  float* Dvec;   // fp32 [B, H, Npad] workspace: rowsum(dO * O); 0 past N
+  float* lse2;   // fp32 [B, H, Npad] workspace: LSE * log2(e); +inf past N
   unsigned* err;
   int B, H, N, d;
   int causal;

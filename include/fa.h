@@ -27,7 +27,8 @@
  *    statistics (LSE) are fp32 [B, H, N].
  *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
  *    aligned.  The library allocates nothing and keeps no per-call state.
- *  - Supported: d in {64, 128}; N a positive multiple of 128; B*H*N < 2^31.
+ *  - Supported: d in {64, 128}; any N >= 1 (a partial last 128-row tile is
+ *    handled inside the kernels); B*H*N < 2^31.
  *  - ``stream`` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call only enqueues work on it and returns; results are
  *    ready when the stream reaches that point.
@@ -61,7 +62,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, p_drop outside [0,1), ... */
-  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d not in {64,128}, N % 128 != 0, too large */
+  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d not in {64,128}, B*H*N too large */
   FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor-map encoding, ...) */
   FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by fa_last_device_error) */
 } fa_status;
@@ -84,8 +85,9 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
- * accumulator [B, H, N, d], the fp32 row statistic D [B, H, N] and the
- * fp32 copy of LSE in log2 units [B, H, N], each rounded up to 256 bytes.
+ * accumulator [B, H, N, d], the fp32 row statistic D and the fp32 copy of
+ * LSE in log2 units, both [B, H, Npad] with Npad = N rounded up to a multiple
+ * of 128, each part rounded up to 256 bytes.
  * Linear in N ("FlashAttention" glossary: memory drops from O(N^2) to O(N)).
  * Returns 0 for non-positive sizes.
  */
@@ -149,8 +151,8 @@ fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const
  * still owns and passes every input and output.
  *   - Limit: fa_bwd_workspace_size(B, H, N, d) must not exceed
  *     FA_NOALLOC_SCRATCH_BYTES; larger problems return FA_ERR_UNSUPPORTED
- *     (use fa_bwd with a caller-provided workspace).  Since N is a multiple
- *     of 128, that allows B*H*N <= 64512 rows at d = 128 and <= 126976 at
+ *     (use fa_bwd with a caller-provided workspace); for N a multiple of
+ *     128 that allows B*H*N <= 64512 rows at d = 128 and <= 126976 at
  *     d = 64.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call

@@ -53,7 +53,10 @@ def check_lse(got, want, what=""):
 
 
 def check_grad(got, want, what=""):
-    rel = rel_fro(got, want)
+    """Relative Frobenius error <= 2e-2, with the reference norm floored at 1e-3
+    for gradients that are identically zero (N = 1: a single key gets P = 1,
+    so dS = 0 and dQ = dK = 0 exactly)."""
+    rel = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-3))
     assert rel <= GRAD_REL_FRO, f"{what}: rel-fro {rel:.3e}"
     return rel
 

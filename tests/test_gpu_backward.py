@@ -85,6 +85,12 @@ def test_long_context_full_size_sampled(idx):
     (1, 2, 384, 128, False, 0.1),   # non-causal with dropout
     (2, 1, 512, 128, True, 0.7),    # threshold above 0x8000
     (1, 3, 640, 64, False, 0.3),
+    # ragged tails: N not a multiple of the 128-row tile
+    (1, 1, 1, 128, True, 0.0),
+    (1, 2, 77, 64, False, 0.1),
+    (2, 1, 200, 128, True, 0.1),
+    (1, 2, 1000, 64, True, 0.0),
+    (1, 1, 2049, 128, False, 0.0),
 ])
 def test_edge_shapes(B, H, N, d, causal, p):
     w = wl.Workload("edge", B, H, N, d, causal, p, 99)

@@ -80,6 +80,13 @@ def test_long_context_full_size_sampled_rows(idx):
     (1, 1, 1024, 128, True, 0.5),    # threshold exactly 0x8000
     (1, 1, 512, 64, True, 0.7),      # threshold above 0x8000
     (1, 2, 256, 128, False, 0.0),
+    # ragged tails: N not a multiple of the 128-row tile
+    (1, 1, 1, 64, True, 0.0),
+    (1, 2, 77, 128, False, 0.1),
+    (2, 1, 129, 64, True, 0.0),
+    (1, 3, 200, 128, True, 0.1),
+    (1, 2, 1000, 64, False, 0.0),
+    (1, 1, 2049, 128, True, 0.0),
 ])
 def test_edge_shapes(B, H, N, d, causal, p):
     w = wl.Workload("edge", B, H, N, d, causal, p, 77)
