@@ -394,10 +394,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (!mbar_wait(&bars[kDSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
-        mma_dk<D>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
-        mma_commit(&bars[kEmpty0 + s]);
+        // dQ first: the dK MMA runs while the drain lifts dQ out of TMEM
         mma_dq<D>(tmem + kColDP, sm_ds, sm_k);
         mma_commit(&bars[kDQReady]);
+        mma_dk<D>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
+        mma_commit(&bars[kEmpty0 + s]);
         mma_commit(&bars[kDSFree]);
         if (more) {
           if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
