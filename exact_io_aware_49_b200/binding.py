@@ -38,10 +38,14 @@ def load_library(path=None):
     vp, i, f, u64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp]
     lib.fa_fwd.restype = i
+    lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, i, vp]
+    lib.fa_fwd_ex.restype = i
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp, sz, vp]
     lib.fa_bwd.restype = i
+    lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, i, vp, sz, vp]
+    lib.fa_bwd_ex.restype = i
     lib.fa_bwd_prepare.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_prepare.restype = i
     lib.fa_bwd_tiles.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp, sz, vp]
@@ -64,11 +68,17 @@ def _stream(t):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
-def _check_bhnd(name, t, shape=None):
+# element types of the ``_ex`` entry points (fa_dtype)
+FA_DTYPE = {torch.bfloat16: 0, torch.float16: 1}
+
+
+def _check_bhnd(name, t, shape=None, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
-    if t.dtype != torch.bfloat16:
-        raise ValueError(f"{name} must be bf16")
+    if t.dtype not in FA_DTYPE:
+        raise ValueError(f"{name} must be bf16 or fp16")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} is {t.dtype}, expected {dtype} like q")
     if t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -81,19 +91,23 @@ def _raise(st, what):
 
 
 def fa_fwd(q, k, v, causal, scale=None, p_drop=0.0, seed=0, out=None, lse=None):
-    """(O, LSE) of exact attention; q, k, v bf16 [B, H, N, d] on one CUDA device."""
+    """(O, LSE) of exact attention; q, k, v [B, H, N, d] on one CUDA device, all
+    bf16 (fa_fwd) or all fp16 (fa_fwd_ex)."""
     lib = load_library()
     _check_bhnd("q", q)
-    _check_bhnd("k", k, q.shape)
-    _check_bhnd("v", v, q.shape)
+    _check_bhnd("k", k, q.shape, q.dtype)
+    _check_bhnd("v", v, q.shape, q.dtype)
     B, H, N, d = q.shape
     scale = d ** -0.5 if scale is None else scale
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
-    _check_bhnd("out", out, q.shape)
-    st = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, N, d,
-                    int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1), _stream(q))
-    _raise(st, "fa_fwd")
+    _check_bhnd("out", out, q.shape, q.dtype)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, N, d, int(bool(causal)),
+            float(scale), float(p_drop), int(seed) & (2**64 - 1))
+    if q.dtype == torch.bfloat16:
+        _raise(lib.fa_fwd(*args, _stream(q)), "fa_fwd")
+    else:
+        _raise(lib.fa_fwd_ex(*args, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_ex")
     return out, lse
 
 
@@ -103,10 +117,11 @@ def fa_bwd_workspace_size(B, H, N, d):
 
 def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspace=None, dq=None, dk=None,
            dv=None):
-    """(dQ, dK, dV) of sum(dO * O) by recomputation; same arguments as the matching fa_fwd call."""
+    """(dQ, dK, dV) of sum(dO * O) by recomputation; same arguments as the matching fa_fwd call
+    (bf16 tensors go to fa_bwd, fp16 ones to fa_bwd_ex)."""
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _check_bhnd(name, t, q.shape)
+        _check_bhnd(name, t, q.shape, q.dtype)
     B, H, N, d = q.shape
     scale = d ** -0.5 if scale is None else scale
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
@@ -117,10 +132,16 @@ def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspac
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
-    st = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
-                    float(p_drop), int(seed) & (2**64 - 1), workspace.data_ptr(), workspace.numel(), _stream(q))
-    _raise(st, "fa_bwd")
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bhnd(name, t, q.shape, q.dtype)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), float(p_drop),
+            int(seed) & (2**64 - 1))
+    ws = (workspace.data_ptr(), workspace.numel(), _stream(q))
+    if q.dtype == torch.bfloat16:
+        _raise(lib.fa_bwd(*args, *ws), "fa_bwd")
+    else:
+        _raise(lib.fa_bwd_ex(*args, FA_DTYPE[q.dtype], *ws), "fa_bwd_ex")
     return dq, dk, dv
 
 
@@ -131,7 +152,7 @@ def fa_bwd_stages(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, w
     record CUDA events around the tiles kernel."""
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _check_bhnd(name, t, q.shape)
+        _check_bhnd(name, t, q.shape, torch.bfloat16)
     B, H, N, d = q.shape
     scale = d ** -0.5 if scale is None else scale
     if workspace is None:

@@ -34,18 +34,18 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH, N, d] row-major 3-D map with 128-byte boxes per row (64 bf16 or 32
-// fp32 columns) x 128 rows x 1 head and 128-byte swizzle.  Rows past N of a
-// head are outside the tensor: loads zero-fill them, reductions skip them.
-bool encode_head_map(CUtensorMap* tm, const void* base, long long BH, int N, int d, bool fp32) {
+// [BH, N, d] row-major 3-D map with 128-byte boxes per row (64 bf16 / fp16
+// or 32 fp32 columns) x 128 rows x 1 head and 128-byte swizzle.  Rows past N
+// of a head are outside the tensor: loads zero-fill them, reductions skip them.
+bool encode_head_map(CUtensorMap* tm, const void* base, long long BH, int N, int d, CUtensorMapDataType dt) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t esize = fp32 ? 4 : 2;
+  const cuuint64_t esize = (dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 4 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(N) * d * esize};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(tm, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  CUresult r = enc(tm, dt, 3,
                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -60,6 +60,10 @@ unsigned* error_word_ptr() {
   if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return nullptr;
   if (dev < 128) cache[dev] = static_cast<unsigned*>(p);
   return static_cast<unsigned*>(p);
+}
+
+CUtensorMapDataType elem_type(bool f16) {
+  return f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 }
 
 bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
@@ -97,8 +101,12 @@ const char* fa_status_string(fa_status s) {
   return "unknown fa_status";
 }
 
-fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
-                 int causal, float scale, float p_drop, uint64_t seed, void* stream) {
+}  // extern "C"
+
+namespace {
+
+fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                   int causal, float scale, float p_drop, uint64_t seed, bool f16, void* stream) {
   if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
   if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(LSE, 16))
     return FA_ERR_INVALID_ARG;
@@ -108,9 +116,11 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   fa::FwdArgs a;
   memset(&a, 0, sizeof(a));
   const long long BH = static_cast<long long>(B) * H;
-  if (!encode_head_map(&a.tmQ, Q, BH, N, d, false) || !encode_head_map(&a.tmK, K, BH, N, d, false) ||
-      !encode_head_map(&a.tmV, V, BH, N, d, false))
+  const CUtensorMapDataType dt = elem_type(f16);
+  if (!encode_head_map(&a.tmQ, Q, BH, N, d, dt) || !encode_head_map(&a.tmK, K, BH, N, d, dt) ||
+      !encode_head_map(&a.tmV, V, BH, N, d, dt))
     return FA_ERR_CUDA;
+  a.f16 = f16 ? 1 : 0;
   a.O = O;
   a.LSE = LSE;
   a.err = error_word_ptr();
@@ -126,6 +136,23 @@ fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LS
   a.seed_lo = static_cast<uint32_t>(seed);
   a.seed_hi = static_cast<uint32_t>(seed >> 32);
   return fa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+bool dtype_ok(fa_dtype dtype) { return dtype == FA_DTYPE_BF16 || dtype == FA_DTYPE_F16; }
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                 int causal, float scale, float p_drop, uint64_t seed, void* stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, causal, scale, p_drop, seed, false, stream);
+}
+
+fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+                    int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -172,12 +199,8 @@ void fill_scalars(fa::BwdArgs* a, int B, int H, int N, int d, int causal, float 
   a->seed_hi = static_cast<uint32_t>(seed >> 32);
 }
 
-}  // namespace
-
-extern "C" {
-
-fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+fa_status prepare_impl(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
+                       void* workspace, size_t workspace_bytes, bool f16, void* stream) {
   if (!O || !dO || !LSE) return FA_ERR_INVALID_ARG;
   if (misaligned(O, 16) || misaligned(dO, 16) || misaligned(LSE, 16)) return FA_ERR_INVALID_ARG;
   fa_status st = check_common(B, H, N, d, 1.0f, 0.0f);
@@ -187,15 +210,16 @@ fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B,
   memset(&a, 0, sizeof(a));
   fill_scalars(&a, B, H, N, d, 0, 1.0f, 0.0f, 0);
   carve_workspace(&a, workspace);
+  a.f16 = f16 ? 1 : 0;
   a.O = O;
   a.dO = dO;
   a.LSE = LSE;
   return fa::launch_bwd_prepare(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
-                       int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+fa_status tiles_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
+                     int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
+                     size_t workspace_bytes, bool f16, void* stream) {
   if (!Q || !K || !V || !dO || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) || misaligned(dK, 16) ||
       misaligned(dV, 16))
@@ -206,12 +230,14 @@ fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* 
   fa::BwdArgs a;
   memset(&a, 0, sizeof(a));
   const long long BH = static_cast<long long>(B) * H;
-  if (!encode_head_map(&a.tmQ, Q, BH, N, d, false) || !encode_head_map(&a.tmK, K, BH, N, d, false) ||
-      !encode_head_map(&a.tmV, V, BH, N, d, false) || !encode_head_map(&a.tmDO, dO, BH, N, d, false))
+  const CUtensorMapDataType dt = elem_type(f16);
+  if (!encode_head_map(&a.tmQ, Q, BH, N, d, dt) || !encode_head_map(&a.tmK, K, BH, N, d, dt) ||
+      !encode_head_map(&a.tmV, V, BH, N, d, dt) || !encode_head_map(&a.tmDO, dO, BH, N, d, dt))
     return FA_ERR_CUDA;
   fill_scalars(&a, B, H, N, d, causal, scale, p_drop, seed);
   carve_workspace(&a, workspace);
-  if (!encode_head_map(&a.tmDQacc, a.dQacc, BH, N, d, true)) return FA_ERR_CUDA;
+  if (!encode_head_map(&a.tmDQacc, a.dQacc, BH, N, d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)) return FA_ERR_CUDA;
+  a.f16 = f16 ? 1 : 0;
   a.dO = dO;
   a.dK = dK;
   a.dV = dV;
@@ -220,8 +246,8 @@ fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* 
   return fa::launch_bwd_tiles(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
-                        size_t workspace_bytes, void* stream) {
+fa_status finish_impl(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
+                      size_t workspace_bytes, bool f16, void* stream) {
   if (!dQ || misaligned(dQ, 16)) return FA_ERR_INVALID_ARG;
   fa_status st = check_common(B, H, N, d, scale, 0.0f);
   if (st != FA_OK) return st;
@@ -230,13 +256,14 @@ fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const
   memset(&a, 0, sizeof(a));
   fill_scalars(&a, B, H, N, d, 0, scale, 0.0f, 0);
   carve_workspace(&a, const_cast<void*>(workspace));
+  a.f16 = f16 ? 1 : 0;
   a.dQ = dQ;
   return fa::launch_bwd_finish(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                 void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
-                 uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                   void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                   uint64_t seed, void* workspace, size_t workspace_bytes, bool f16, void* stream) {
   // Validate everything up front so a rejected call launches none of the stages.
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
@@ -245,11 +272,47 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
   fa_status st = check_common(B, H, N, d, scale, p_drop);
   if (st != FA_OK) return st;
   if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
-  if ((st = fa_bwd_prepare(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK) return st;
-  if ((st = fa_bwd_tiles(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes,
-                         stream)) != FA_OK)
+  if ((st = prepare_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, f16, stream)) != FA_OK) return st;
+  if ((st = tiles_impl(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes, f16,
+                       stream)) != FA_OK)
     return st;
-  return fa_bwd_finish(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  return finish_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, f16, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  return prepare_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, false, stream);
+}
+
+fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
+                       int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return tiles_impl(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes, false,
+                    stream);
+}
+
+fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  return finish_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, false, stream);
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                 void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                 uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace,
+                  workspace_bytes, false, stream);
+}
+
+fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                    void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
+                    uint64_t seed, fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace,
+                  workspace_bytes, dtype == FA_DTYPE_F16, stream);
 }
 
 fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed, void* stream) {

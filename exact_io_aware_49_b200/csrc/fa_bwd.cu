@@ -12,16 +12,16 @@
 //   dQ = scale * dS K                 dK = scale * dS^T Q
 //
 // Three kernels:
-//   1. preprocess: D_i = rowsum(dO * O) (fp32, from the stored bf16 O),
+//   1. preprocess: D_i = rowsum(dO * O) (fp32, from the stored 16-bit O),
 //      LSE2_i = LSE_i * log2(e), and zeroing of the fp32 dQ accumulator;
 //   2. main: one CTA per (b, h, 128-key tile j) keeps K_j, V_j in shared
 //      memory and dK_j, dV_j in tensor memory while it streams the query
 //      tiles i (i >= j when causal) through a two-stage TMA ring.  Per tile:
 //        S^T = K_j Q_i^T and dP^T = V_j dO_i^T  (tcgen05, M = 128 keys)
 //        P^T = exp2(S^T scale log2e - LSE2_i), masked, dropout-masked
-//              -> written as bf16 into TMEM over S^T
+//              -> written in the input type into TMEM over S^T
 //        dV += P^T dO_i                          (A operand read from TMEM)
-//        dS^T = P^T (dP^T Z/(1-p) - D_i)  -> bf16, 128B-swizzled in smem
+//        dS^T = P^T (dP^T Z/(1-p) - D_i)  -> 16-bit, 128B-swizzled in smem
 //        dK += dS^T Q_i ;  dQ_i = dS K_j  (the same smem tile read K-major
 //              for dK and MN-major for dQ)
 //        dQ_i is read out of TMEM by a dedicated warpgroup, staged through the
@@ -30,7 +30,9 @@
 //      Warp roles: warpgroups 0/1 do the elementwise work for query columns
 //      0-63 / 64-127 (one thread per key row, the TMEM lane); warp 8 issues
 //      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
-//   3. convert: dQ = bf16(scale * dQacc).
+//   3. convert: dQ = scale * dQacc, rounded to the input type.
+// Inputs and outputs are all bf16 or all fp16 (the F16 template flag); every
+// accumulation is fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -49,9 +51,9 @@ namespace {
 // One warp per padded row (b*H + h, i < Npad): for i < N, D = sum(dO * O),
 // LSE2 = LSE * log2(e) and the dQ accumulator row is zeroed; for the padding
 // rows of a partial last tile, D = 0 and LSE2 = +inf (so exp2(x - LSE2) = 0).
-template <int D>
-__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ O,
-                                                                const __nv_bfloat16* __restrict__ dO,
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* __restrict__ O,
+                                                                const uint16_t* __restrict__ dO,
                                                                 const float* __restrict__ LSE,
                                                                 float* __restrict__ Dvec,
                                                                 float* __restrict__ lse2,
@@ -80,8 +82,8 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
       const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 fa2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
-        const float2 fb2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+        const float2 fa2 = unpack2<F16>(av[e]);
+        const float2 fb2 = unpack2<F16>(bv[e]);
         acc = fmaf(fa2.x, fb2.x, acc);
         acc = fmaf(fa2.y, fb2.y, acc);
       }
@@ -99,18 +101,19 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
 
 // ============================================================ dQ convert
 
+template <bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ dQacc,
-                                                                __nv_bfloat16* __restrict__ dQ, float scale,
+                                                                uint16_t* __restrict__ dQ, float scale,
                                                                 long long n8) {
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n8;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 a = reinterpret_cast<const float4*>(dQacc)[2 * idx];
     const float4 b = reinterpret_cast<const float4*>(dQacc)[2 * idx + 1];
     uint4 o;
-    o.x = pack_bf16x2(a.x * scale, a.y * scale);
-    o.y = pack_bf16x2(a.z * scale, a.w * scale);
-    o.z = pack_bf16x2(b.x * scale, b.y * scale);
-    o.w = pack_bf16x2(b.z * scale, b.w * scale);
+    o.x = pack2<F16>(a.x * scale, a.y * scale);
+    o.y = pack2<F16>(a.z * scale, a.w * scale);
+    o.z = pack2<F16>(b.x * scale, b.y * scale);
+    o.w = pack2<F16>(b.z * scale, b.w * scale);
     reinterpret_cast<uint4*>(dQ)[idx] = o;
   }
 }
@@ -130,13 +133,13 @@ static_assert(2 * 128 * kEwRegs + 128 * kDqRegs + 128 * kCtlRegs <= kBwdThreads 
 
 template <int D>
 struct BwdSmem {
-  static constexpr int kTile = 128 * D * 2;  // 128 rows x D bf16
-  static constexpr int kBox = 128 * 128;     // 128 rows x 64 bf16 (one 128-byte swizzle span)
+  static constexpr int kTile = 128 * D * 2;  // 128 rows x D 16-bit elements
+  static constexpr int kBox = 128 * 128;     // 128 rows x 64 16-bit (one 128-byte swizzle span)
   static constexpr int kK = 0;
   static constexpr int kV = kTile;
   static constexpr int kQ = 2 * kTile;      // 2 stages
   static constexpr int kDO = 4 * kTile;     // 2 stages
-  static constexpr int kDS = 6 * kTile;     // dS^T: 128 keys x 128 queries bf16 = 2 boxes
+  static constexpr int kDS = 6 * kTile;     // dS^T: 128 keys x 128 queries 16-bit = 2 boxes
   static constexpr int kVec = kDS + 2 * kBox;  // 2 stages x (LSE2[128], D[128]) fp32
   static constexpr int kBar = kVec + 2 * 1024;
   static constexpr int kNumBars = 18;
@@ -162,8 +165,8 @@ enum BwdBar {
 };
 
 struct BwdParams {
-  __nv_bfloat16* dK;
-  __nv_bfloat16* dV;
+  uint16_t* dK;  // bf16 or fp16 bits
+  uint16_t* dV;
   float* dQacc;
   const float* lse2;
   const float* Dvec;
@@ -178,9 +181,9 @@ struct BwdParams {
 };
 
 // D[tmem] (+)= A[K-major tile] * B[K-major tile]^T, M = N = 128, K = D.
-template <int D>
+template <int D, bool F16>
 __device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+  constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
@@ -188,10 +191,10 @@ __device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, ui
   }
 }
 
-// dV (+)= P^T dO : A = P^T (TMEM, bf16 pairs), B = dO tile (MN-major), K = 128 queries, N = D.
-template <int D>
+// dV (+)= P^T dO : A = P^T (TMEM, 16-bit pairs), B = dO tile (MN-major), K = 128 queries, N = D.
+template <int D, bool F16>
 __device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
     mma_ts(tmem_d, tmem_p + kk * 8, sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc,
@@ -199,9 +202,9 @@ __device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_
 }
 
 // dK (+)= dS^T Q : A = dS^T (smem, K-major over queries), B = Q tile (MN-major), N = D.
-template <int D>
+template <int D, bool F16>
 __device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32_t q_smem, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t a_off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
@@ -211,9 +214,9 @@ __device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32
 }
 
 // dQ_i = dS K : A = dS (the dS^T tile read MN-major, M = queries), B = K tile (MN-major), N = D.
-template <int D>
+template <int D, bool F16>
 __device__ __forceinline__ void mma_dq(uint32_t tmem_d, uint32_t ds_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+  constexpr uint32_t idesc = idesc_f32acc(128, D, true, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
     mma_ss(tmem_d, sdesc_sw128(ds_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
@@ -278,7 +281,7 @@ __device__ __forceinline__ void mark_dropped4(float* P, uint32_t nib) {
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -371,12 +374,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mbar_wait(&bars[kQFull0], 0, abort_flag, p.err);
       if (ok) {
         tc_fence_after();
-        mma_tile_kk<D>(tmem + kColS, sm_k, sm_q);
+        mma_tile_kk<D, F16>(tmem + kColS, sm_k, sm_q);
         mma_commit(&bars[kSReady]);
         ok = mbar_wait(&bars[kDOFull0], 0, abort_flag, p.err);
         if (ok) {
           tc_fence_after();
-          mma_tile_kk<D>(tmem + kColDP, sm_v, sm_do);
+          mma_tile_kk<D, F16>(tmem + kColDP, sm_v, sm_do);
           mma_commit(&bars[kDPReady]);
         }
       }
@@ -385,26 +388,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const bool more = it + 1 < nq;
         if (!mbar_wait(&bars[kPReady], it & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
-        mma_dv<D>(tmem + kColDV, tmem + kColS, sm_do + s * L::kTile, it > 0);
+        mma_dv<D, F16>(tmem + kColDV, tmem + kColS, sm_do + s * L::kTile, it > 0);
         if (more) {
           if (!mbar_wait(&bars[kQFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
-          mma_tile_kk<D>(tmem + kColS, sm_k, sm_q + s1 * L::kTile);
+          mma_tile_kk<D, F16>(tmem + kColS, sm_k, sm_q + s1 * L::kTile);
           mma_commit(&bars[kSReady]);
         }
         if (!mbar_wait(&bars[kDSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         // dQ first: the dK MMA runs while the drain lifts dQ out of TMEM
-        mma_dq<D>(tmem + kColDP, sm_ds, sm_k);
+        mma_dq<D, F16>(tmem + kColDP, sm_ds, sm_k);
         mma_commit(&bars[kDQReady]);
-        mma_dk<D>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
+        mma_dk<D, F16>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
         mma_commit(&bars[kEmpty0 + s]);
         mma_commit(&bars[kDSFree]);
         if (more) {
           if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
               !mbar_wait(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
-          mma_tile_kk<D>(tmem + kColDP, sm_v, sm_do + s1 * L::kTile);
+          mma_tile_kk<D, F16>(tmem + kColDP, sm_v, sm_do + s1 * L::kTile);
           mma_commit(&bars[kDPReady]);
         }
       }
@@ -539,7 +542,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (64 * g + c < lo) P[c] = 0.f;
       }
       if (DROPOUT) {
-        // dropped entries get the sign bit set; dS and the bf16 pack read it
+        // dropped entries get the sign bit set; dS and the 16-bit pack read it
 #pragma unroll
         for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -548,7 +551,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        pk[c] = DROPOUT ? pack_bf16x2_relu(P[2 * c], P[2 * c + 1]) : pack_bf16x2(P[2 * c], P[2 * c + 1]);
+        pk[c] = DROPOUT ? pack2_relu<F16>(P[2 * c], P[2 * c + 1]) : pack2<F16>(P[2 * c], P[2 * c + 1]);
       tmem_st32(t_row + kColS + 32 * g, pk);
       tmem_st_wait();
       tc_fence_before();
@@ -576,8 +579,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // kept: P (dP / (1-p) - D); dropped (sign set): -|P| D
           v[e] = DROPOUT ? fmaxf(P[c], 0.f) * (dp * p.drop_scale) - fabsf(P[c]) * dd[e] : P[c] * (dp - dd[e]);
         }
-        dsk[2 * c4] = pack_bf16x2(v[0], v[1]);
-        dsk[2 * c4 + 1] = pack_bf16x2(v[2], v[3]);
+        dsk[2 * c4] = pack2<F16>(v[0], v[1]);
+        dsk[2 * c4 + 1] = pack2<F16>(v[2], v[3]);
       }
       // the dS^T buffer is free once the previous tile's dK / dQ MMAs have read it
       if (it > 0 && !mbar_wait(&bars[kDSFree], (it - 1) & 1, abort_flag, p.err)) { ok = false; break; }
@@ -596,7 +599,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint32_t col = (g == 0) ? kColDK : kColDV;
       const float mul = (g == 0) ? p.scale : p.drop_scale;
-      __nv_bfloat16* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(bh) * N + kj * 128 + r) * D;
+      uint16_t* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(bh) * N + kj * 128 + r) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -606,7 +609,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t o[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          o[e] = pack2<F16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
         if (key_valid) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
@@ -618,9 +621,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
-  auto kern = fa_bwd_kernel<D, CAUSAL, DROPOUT>;
+  auto kern = fa_bwd_kernel<D, CAUSAL, DROPOUT, F16>;
   const int used = BwdSmem<D>::kUsed;
   int max_optin = 0, dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -638,8 +641,8 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (attr.numRegs < kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
   BwdParams p;
-  p.dK = static_cast<__nv_bfloat16*>(a.dK);
-  p.dV = static_cast<__nv_bfloat16*>(a.dV);
+  p.dK = static_cast<uint16_t*>(a.dK);
+  p.dV = static_cast<uint16_t*>(a.dV);
   p.dQacc = a.dQacc;
   p.lse2 = a.lse2;
   p.Dvec = a.Dvec;
@@ -667,6 +670,31 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <bool F16>
+void launch_preprocess_typed(const BwdArgs& a, long long blocks, long long rows_pad, int Npad, cudaStream_t stream) {
+  const uint16_t* O = static_cast<const uint16_t*>(a.O);
+  const uint16_t* dO = static_cast<const uint16_t*>(a.dO);
+  if (a.d == 64)
+    fa_bwd_preprocess_kernel<64, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
+                                                                                    a.dQacc, rows_pad, a.N, Npad);
+  else
+    fa_bwd_preprocess_kernel<128, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
+                                                                                     a.dQacc, rows_pad, a.N, Npad);
+}
+
+template <bool F16>
+cudaError_t launch_bwd_tiles_typed(const BwdArgs& a, cudaStream_t stream) {
+  const bool drop = a.drop_t != 0;
+  if (a.d == 64) {
+    if (a.causal)
+      return drop ? launch_bwd_main<64, true, true, F16>(a, stream) : launch_bwd_main<64, true, false, F16>(a, stream);
+    return drop ? launch_bwd_main<64, false, true, F16>(a, stream) : launch_bwd_main<64, false, false, F16>(a, stream);
+  }
+  if (a.causal)
+    return drop ? launch_bwd_main<128, true, true, F16>(a, stream) : launch_bwd_main<128, true, false, F16>(a, stream);
+  return drop ? launch_bwd_main<128, false, true, F16>(a, stream) : launch_bwd_main<128, false, false, F16>(a, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
@@ -674,25 +702,15 @@ cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
   const long long rows_pad = static_cast<long long>(a.B) * a.H * Npad;
   long long blocks = (rows_pad + 7) / 8;  // one warp per row, 8 warps per block
   if (blocks > 148 * 16) blocks = 148 * 16;
-  const __nv_bfloat16* O = static_cast<const __nv_bfloat16*>(a.O);
-  const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(a.dO);
-  if (a.d == 64)
-    fa_bwd_preprocess_kernel<64><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                               a.dQacc, rows_pad, a.N, Npad);
+  if (a.f16)
+    launch_preprocess_typed<true>(a, blocks, rows_pad, Npad, stream);
   else
-    fa_bwd_preprocess_kernel<128><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                a.dQacc, rows_pad, a.N, Npad);
+    launch_preprocess_typed<false>(a, blocks, rows_pad, Npad, stream);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream) {
-  const bool drop = a.drop_t != 0;
-  if (a.d == 64) {
-    if (a.causal) return drop ? launch_bwd_main<64, true, true>(a, stream) : launch_bwd_main<64, true, false>(a, stream);
-    return drop ? launch_bwd_main<64, false, true>(a, stream) : launch_bwd_main<64, false, false>(a, stream);
-  }
-  if (a.causal) return drop ? launch_bwd_main<128, true, true>(a, stream) : launch_bwd_main<128, true, false>(a, stream);
-  return drop ? launch_bwd_main<128, false, true>(a, stream) : launch_bwd_main<128, false, false>(a, stream);
+  return a.f16 ? launch_bwd_tiles_typed<true>(a, stream) : launch_bwd_tiles_typed<false>(a, stream);
 }
 
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
@@ -700,8 +718,11 @@ cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  fa_bwd_dq_convert_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, static_cast<__nv_bfloat16*>(a.dQ),
-                                                                        a.scale, n8);
+  uint16_t* dQ = static_cast<uint16_t*>(a.dQ);
+  if (a.f16)
+    fa_bwd_dq_convert_kernel<true><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, n8);
+  else
+    fa_bwd_dq_convert_kernel<false><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, n8);
   return cudaGetLastError();
 }
 

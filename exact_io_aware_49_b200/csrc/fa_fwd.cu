@@ -13,9 +13,9 @@
 //  * one CTA owns two 128-row query tiles (Q0, Q1) of one (b, h) and streams
 //    128-key K/V tiles through a multi-stage TMA + mbarrier ring;
 //  * S_q = Q_q K_t^T and O_q += P_q V_t run on the 5th-generation tensor cores
-//    (tcgen05.mma, bf16 in, fp32 accumulators in tensor memory).  TMEM holds
-//    S0 | S1 | O0 | O1 (512 columns); P_q (bf16) is written back over S_q and
-//    read by the PV MMA directly from TMEM;
+//    (tcgen05.mma, bf16 or fp16 in, fp32 accumulators in tensor memory).
+//    TMEM holds S0 | S1 | O0 | O1 (512 columns); P_q (in the input type) is
+//    written back over S_q and read by the PV MMA directly from TMEM;
 //  * warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q0 and Q1
 //    (one thread per query row: causal mask on the diagonal tile, running
 //    max / sum, exp2, Philox dropout, P to TMEM, and the epilogue); warp 8
@@ -62,7 +62,7 @@ constexpr float kRescaleTau = 8.0f;  // lazy-rescale threshold, log2 units
 template <int D>
 struct FwdSmem {
   static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kTileBytes = kBN * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kTileBytes = kBN * D * 2;  // one 128 x D tile of 16-bit elements
   static constexpr int kBoxBytes = 128 * 128;     // one 128-row x 64-col box (128B rows)
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + 2 * kTileBytes;
@@ -102,7 +102,7 @@ __device__ __forceinline__ FwdBars fwd_bars(uint8_t* smem) {
 }
 
 struct FwdParams {
-  __nv_bfloat16* O;
+  uint16_t* O;  // bf16 or fp16 bits
   float* LSE;
   unsigned* err;
   int H, N;
@@ -114,9 +114,9 @@ struct FwdParams {
 };
 
 // S_q = Q_q * K^T : M = 128 query rows, N = 128 keys, K = D (both K-major).
-template <int D>
+template <int D, bool F16>
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+  constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * FwdSmem<D>::kBoxBytes + (kk % 4) * 32;
@@ -124,11 +124,11 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint3
   }
 }
 
-// O_q (+)= P_q * V : M = 128, N = D, K = 128 keys.  P (bf16, packed in pairs)
-// lives in TMEM over S_q; V is MN-major in shared memory (D contiguous).
-template <int D>
+// O_q (+)= P_q * V : M = 128, N = D, K = 128 keys.  P (16-bit, packed in
+// pairs) lives in TMEM over S_q; V is MN-major in shared memory (D contiguous).
+template <int D, bool F16>
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
     const uint64_t bdesc = sdesc_sw128(v_smem + kk * 2048, FwdSmem<D>::kBoxBytes, 1024);
@@ -144,7 +144,7 @@ __device__ __forceinline__ void cta_teardown(uint32_t tmem, bool dealloc) {
   if (dealloc) tmem_dealloc(tmem, 512);
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok) {
         tc_fence_after();
         for (int q = 0; q < nq; ++q) {
-          issue_qk<D>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k);
+          issue_qk<D, F16>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k);
           mma_commit(&bar.s_ready[q]);
         }
       }
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (t >= ntile[q]) continue;
           if (!mbar_wait(&bar.p_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tmem + 256 + q * D, tmem + q * 128, sm_v + s * L::kTileBytes, t > 0);
+          issue_pv<D, F16>(tmem + 256 + q * D, tmem + q * 128, sm_v + s * L::kTileBytes, t > 0);
           if (t == ntile[q] - 1) {
             mma_commit(&bar.o_ready[q]);
           } else {
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tc_fence_after();
               next_k_ready = true;
             }
-            issue_qk<D>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k + s1 * L::kTileBytes);
+            issue_qk<D, F16>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k + s1 * L::kTileBytes);
             mma_commit(&bar.s_ready[q]);
           }
         }
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             float q0, q1;
             f2_unpack(pp, q0, q1);
-            pk[c] = pack_bf16x2(q0, q1);
+            pk[c] = pack2<F16>(q0, q1);
           }
         }
         {
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ---------------------------------------------------------- epilogue
         tc_fence_after();
         const float inv = p.drop_scale / l;
-        __nv_bfloat16* orow_g = p.O + (static_cast<size_t>(bh) * N + i) * D;
+        uint16_t* orow_g = p.O + (static_cast<size_t>(bh) * N + i) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           uint32_t packed[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            packed[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+            packed[e] = pack2<F16>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
           if (i < N) {  // rows of a partial last tile past N are computed but not stored
             uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
 #pragma unroll
@@ -441,9 +441,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
-  auto kern = fa_fwd_kernel<D, CAUSAL, DROPOUT>;
+  auto kern = fa_fwd_kernel<D, CAUSAL, DROPOUT, F16>;
   const int smem = FwdSmem<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -453,7 +453,7 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (attr.numRegs < kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
   FwdParams p;
-  p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.O = static_cast<uint16_t*>(a.O);
   p.LSE = a.LSE;
   p.err = a.err;
   p.H = a.H;
@@ -479,16 +479,23 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <bool F16>
+cudaError_t launch_fwd_typed(const FwdArgs& a, cudaStream_t stream) {
+  const bool drop = a.drop_t != 0;
+  if (a.d == 64) {
+    if (a.causal)
+      return drop ? launch_fwd_t<64, true, true, F16>(a, stream) : launch_fwd_t<64, true, false, F16>(a, stream);
+    return drop ? launch_fwd_t<64, false, true, F16>(a, stream) : launch_fwd_t<64, false, false, F16>(a, stream);
+  }
+  if (a.causal)
+    return drop ? launch_fwd_t<128, true, true, F16>(a, stream) : launch_fwd_t<128, true, false, F16>(a, stream);
+  return drop ? launch_fwd_t<128, false, true, F16>(a, stream) : launch_fwd_t<128, false, false, F16>(a, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream) {
-  const bool drop = a.drop_t != 0;
-  if (a.d == 64) {
-    if (a.causal) return drop ? launch_fwd_t<64, true, true>(a, stream) : launch_fwd_t<64, true, false>(a, stream);
-    return drop ? launch_fwd_t<64, false, true>(a, stream) : launch_fwd_t<64, false, false>(a, stream);
-  }
-  if (a.causal) return drop ? launch_fwd_t<128, true, true>(a, stream) : launch_fwd_t<128, true, false>(a, stream);
-  return drop ? launch_fwd_t<128, false, true>(a, stream) : launch_fwd_t<128, false, false>(a, stream);
+  return a.f16 ? launch_fwd_typed<true>(a, stream) : launch_fwd_typed<false>(a, stream);
 }
 
 }  // namespace fa

@@ -9,8 +9,9 @@
 namespace fa {
 
 struct FwdArgs {
-  CUtensorMap tmQ, tmK, tmV;  // 3-D maps over [B*H, N, d] bf16, 64 x 128 x 1 boxes, 128B swizzle
-  void* O;                    // bf16 [B, H, N, d]
+  CUtensorMap tmQ, tmK, tmV;  // 3-D maps over [B*H, N, d] 16-bit, 64 x 128 x 1 boxes, 128B swizzle
+  void* O;                    // [B, H, N, d], same type as Q
+  int f16;                    // element type of Q, K, V, O: 0 bf16, 1 fp16
   float* LSE;                 // fp32 [B, H, N]
   unsigned* err;              // device error word
   int B, H, N, d;
@@ -24,6 +25,7 @@ struct FwdArgs {
 struct BwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // same layout as the forward maps
   CUtensorMap tmDQacc;               // fp32 [B*H, N, d], 32-column x 128-row boxes, 128B swizzle
+  int f16;  // element type of Q, K, V, O, dO, dQ, dK, dV: 0 bf16, 1 fp16
   const void* O;
   const void* dO;
   const float* LSE;

@@ -60,8 +60,9 @@ WORKLOADS = [
 BY_NAME = {w.name: w for w in WORKLOADS}
 
 
-def draw_inputs(w: Workload, B=None, H=None, N=None):
-    """(Q, K, V, dO) as bf16 CPU tensors [B, H, N, d] drawn by the recipe above.
+def draw_inputs(w: Workload, B=None, H=None, N=None, dtype=torch.bfloat16):
+    """(Q, K, V, dO) as CPU tensors [B, H, N, d] drawn by the recipe above,
+    rounded to ``dtype`` (bf16 unless asked for fp16).
 
     B, H, N may be overridden to draw a reduced case with the same recipe.
     """
@@ -77,7 +78,7 @@ def draw_inputs(w: Workload, B=None, H=None, N=None):
     if w.qk_std != 1.0:
         q = q * w.qk_std
         k = k * w.qk_std
-    return tuple(x.to(torch.bfloat16) for x in (q, k, v, do))
+    return tuple(x.to(dtype) for x in (q, k, v, do))
 
 
 def sample_rows(w: Workload, n_rows=None, B=None, H=None, N=None):

@@ -23,8 +23,10 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Tensors are dense, row-major [B, H, N, d] (strides H*N*d, N*d, d, 1) with
- *    elements of type bf16 (IEEE bfloat16, passed as void*).  Per-row
- *    statistics (LSE) are fp32 [B, H, N].
+ *    16-bit elements passed as void*: bfloat16 for the plain entry points;
+ *    bfloat16 or IEEE fp16 (binary16), as the ``dtype`` argument says, for
+ *    the ``_ex`` ones.  All tensors of one call share the type.  Per-row
+ *    statistics (LSE) are fp32 [B, H, N]; every sum inside the kernels is fp32.
  *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
  *    aligned.  The library allocates nothing and keeps no per-call state.
  *  - Supported: d in {64, 128}; any N >= 1 (a partial last 128-row tile is
@@ -67,6 +69,12 @@ typedef enum {
   FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by fa_last_device_error) */
 } fa_status;
 
+/* Element type of the 16-bit tensors of an ``_ex`` call. */
+typedef enum {
+  FA_DTYPE_BF16 = 0, /* bfloat16: 8 exponent bits, 7 stored mantissa bits */
+  FA_DTYPE_F16 = 1   /* IEEE binary16: 5 exponent bits, 10 stored mantissa bits */
+} fa_dtype;
+
 /*
  * Forward pass.
  *   Q, K, V : in,  bf16 [B, H, N, d]
@@ -82,6 +90,16 @@ typedef enum {
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
                  int B, int H, int N, int d, int causal, float scale,
                  float p_drop, uint64_t seed, void* stream);
+
+/*
+ * fa_fwd for either 16-bit input type: Q, K, V and O are all of ``dtype``
+ * (FA_DTYPE_BF16 gives exactly fa_fwd).  The probabilities fed to the second
+ * product are rounded to ``dtype`` too; LSE stays fp32.  An unknown dtype
+ * returns FA_ERR_INVALID_ARG.
+ */
+fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                    int B, int H, int N, int d, int causal, float scale,
+                    float p_drop, uint64_t seed, fa_dtype dtype, void* stream);
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
@@ -115,6 +133,19 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
                  int B, int H, int N, int d, int causal, float scale,
                  float p_drop, uint64_t seed, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/*
+ * fa_bwd for either 16-bit input type: Q, K, V, O, dO, dQ, dK and dV are all
+ * of ``dtype`` (FA_DTYPE_BF16 gives exactly fa_bwd); the workspace is the
+ * same fp32 scratch of fa_bwd_workspace_size() bytes.  The recomputed P and
+ * dS are rounded to ``dtype`` before their products.  An unknown dtype
+ * returns FA_ERR_INVALID_ARG.
+ */
+fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV,
+                    int B, int H, int N, int d, int causal, float scale,
+                    float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 /*
  * The three stages fa_bwd runs, in order, for callers that schedule or time

@@ -22,15 +22,16 @@ def rel_fro(got, want):
     return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
 
 
-def bf16_half_ulp(x):
-    """Half a bf16 unit in the last place at |x| (8 significant bits): the largest
-    error that rounding the exact value to the bf16 output can introduce."""
+def bf16_half_ulp(x, bits=8):
+    """Half a unit in the last place at |x| of a format with ``bits`` significant
+    bits (8 for bf16, 11 for fp16): the largest error that rounding the exact
+    value to the 16-bit output can introduce (normal range)."""
     ax = np.abs(np.asarray(x, dtype=np.float64))
     e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
-    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+    return np.where(ax > 0, np.exp2(e - bits), 0.0)
 
 
-def check_o(got, want, what=""):
+def check_o(got, want, what="", bits=8):
     """O max-abs <= 1e-2 on top of the bf16 output rounding, rel-Frobenius <= 5e-3.
 
     O is returned in bf16, so even the exact result rounded to bf16 differs from
@@ -38,7 +39,7 @@ def check_o(got, want, what=""):
     (near one-hot rows of wide-logit inputs, or 1/(1-p) at large p).  The
     max-abs bound therefore applies to the error beyond that rounding:
     |got - want| <= 1e-2 + half_ulp_bf16(want)."""
-    excess = float((np.abs(got - want) - bf16_half_ulp(want)).max())
+    excess = float((np.abs(got - want) - bf16_half_ulp(want, bits)).max())
     err = float(np.abs(got - want).max())
     rel = rel_fro(got, want)
     assert excess <= O_MAX_ABS and rel <= O_REL_FRO, \

@@ -33,7 +33,7 @@ def _declared_functions():
 
 def test_header_declares_entry_points():
     names = _declared_functions()
-    for want in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_tiles", "fa_bwd_finish",
+    for want in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_workspace_size", "fa_bwd_prepare", "fa_bwd_tiles", "fa_bwd_finish",
                  "fa_dropout_mask", "fa_last_device_error", "fa_status_string"):
         assert want in names
 
@@ -95,6 +95,26 @@ def test_workspace_size_is_linear_in_n(lib):
 ])
 def test_bwd_rejects_bad_arguments(lib, kw, want):
     assert _bwd(lib, **kw) == want
+
+
+@pytest.mark.parametrize("dtype", [-1, 2, 7])
+def test_ex_entry_points_reject_unknown_dtype(lib, dtype):
+    # every other argument is valid: only the element type stops the call
+    assert lib.fa_fwd_ex(A, A, A, A, A, 1, 1, 128, 64, 0, 0.125, 0.0, 0, dtype, None) == 1
+    ws_ok = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 0.0, 0, dtype, A, ws_ok, None) == 1
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+def test_ex_entry_points_validate_like_the_plain_ones(lib, dtype):
+    ws_ok = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert lib.fa_fwd_ex(0, A, A, A, A, 1, 1, 128, 64, 0, 0.125, 0.0, 0, dtype, None) == 1
+    assert lib.fa_fwd_ex(A, A, A, A, A, 1, 1, 128, 96, 0, 0.125, 0.0, 0, dtype, None) == 2
+    assert lib.fa_fwd_ex(A, A, A, A + 8, A, 1, 1, 128, 64, 0, 0.125, 0.0, 0, dtype, None) == 1
+    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 1.0, 0, dtype, A, ws_ok, None) == 1
+    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 0.0, 0, dtype, A, ws_ok - 4,
+                         None) == 1
+    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 32, 1, 0.125, 0.0, 0, dtype, A, ws_ok, None) == 2
 
 
 def test_stage_entry_points_reject_bad_arguments(lib):
