@@ -9,6 +9,7 @@
 
 #include "../../include/fa.h"
 #include "fa_internal.h"
+#include "philox.cuh"
 
 namespace {
 
@@ -135,6 +136,7 @@ fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* 
   a.drop_scale = a.drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
   a.seed_lo = static_cast<uint32_t>(seed);
   a.seed_hi = static_cast<uint32_t>(seed >> 32);
+  fa::philox_round_keys(seed, a.philox_rk);
   return fa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -197,6 +199,7 @@ void fill_scalars(fa::BwdArgs* a, int B, int H, int N, int d, int causal, float 
   a->drop_scale = a->drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
   a->seed_lo = static_cast<uint32_t>(seed);
   a->seed_hi = static_cast<uint32_t>(seed >> 32);
+  fa::philox_round_keys(seed, a->philox_rk);
 }
 
 fa_status prepare_impl(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,

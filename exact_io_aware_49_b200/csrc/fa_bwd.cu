@@ -176,7 +176,7 @@ struct BwdParams {
   float scale_log2;
   uint32_t drop_t;
   float drop_scale;
-  uint32_t seed_lo, seed_hi;
+  uint32_t philox_rk[20];  // Philox round keys (read from the constant bank)
   int group, BH;
 };
 
@@ -244,13 +244,13 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
 // k' holds bit l = keep(its key, query q0 + 8 j + l).
 template <bool kHighT>
 __device__ __forceinline__ uint32_t keep_bits_32(uint32_t key_grp, uint32_t q0, uint32_t h, uint32_t b,
-                                                 uint32_t seed_lo, uint32_t seed_hi, uint32_t c2, int lane) {
+                                                 const uint32_t* rk, uint32_t c2, int lane) {
   const uint32_t l8 = static_cast<uint32_t>(lane & 7);
   uint32_t W = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     uint32_t w[4];
-    philox4x32_10(key_grp, q0 + 8 * j + l8, h, b, seed_lo, seed_hi, w);
+    philox4x32_10_rk(key_grp, q0 + 8 * j + l8, h, b, rk, w);
     uint32_t acc = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -285,7 +285,7 @@ template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ BwdParams p) {
   using L = BwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -505,8 +505,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g);
 #pragma unroll
       for (int half = 0; half < 2; ++half)
-        zb[half] = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane)
-                        : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.seed_lo, p.seed_hi, dk.c2, lane);
+        zb[half] = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane)
+                        : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane);
     };
     if (DROPOUT) keep_bits_tile(q_first);
     bool ok = true;
@@ -653,8 +653,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
-  p.seed_lo = a.seed_lo;
-  p.seed_hi = a.seed_hi;
+  for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
   p.BH = a.B * a.H;
   {
     // heads per group: about 512 key-tile units per group; the CTAs running

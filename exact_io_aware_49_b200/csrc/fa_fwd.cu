@@ -109,7 +109,7 @@ struct FwdParams {
   float scale_log2;
   uint32_t drop_t;
   float drop_scale;
-  uint32_t seed_lo, seed_hi;
+  uint32_t philox_rk[20];  // Philox round keys (read from the constant bank)
   int group, BH;
 };
 
@@ -147,7 +147,7 @@ __device__ __forceinline__ void cta_teardown(uint32_t tmem, bool dealloc) {
 template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
   using L = FwdSmem<D>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -372,8 +372,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int g = 0; g < kBN / 8; ++g) {
           uint32_t w[4];
           if (DROPOUT)
-            philox4x32_10(static_cast<uint32_t>(t * (kBN / 8) + g), static_cast<uint32_t>(i),
-                          static_cast<uint32_t>(h), static_cast<uint32_t>(b), p.seed_lo, p.seed_hi, w);
+            philox4x32_10_rk(static_cast<uint32_t>(t * (kBN / 8) + g), static_cast<uint32_t>(i),
+                             static_cast<uint32_t>(h), static_cast<uint32_t>(b), p.philox_rk, w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = 4 * g + e;
@@ -461,8 +461,7 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
-  p.seed_lo = a.seed_lo;
-  p.seed_hi = a.seed_hi;
+  for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
   p.BH = a.B * a.H;
   {
     // heads per group: about 256 work units (~2 waves on 148 SMs) per group,

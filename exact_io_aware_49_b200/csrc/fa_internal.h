@@ -20,6 +20,7 @@ struct FwdArgs {
   uint32_t drop_t;    // keep <=> u16 >= drop_t (0: no dropout)
   float drop_scale;   // 1 / (1 - p)
   uint32_t seed_lo, seed_hi;
+  uint32_t philox_rk[20];  // Philox round keys of the seed (rounds 0..9, k0 / k1 interleaved)
 };
 
 struct BwdArgs {
@@ -43,6 +44,7 @@ struct BwdArgs {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  uint32_t philox_rk[20];  // Philox round keys of the seed (rounds 0..9, k0 / k1 interleaved)
 };
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
