@@ -2,13 +2,19 @@
 
 TEST INFRASTRUCTURE ONLY -- see ``oracle/__init__.py``.
 
-Definition followed (per head; Q, K, V, dO are [N, d]):
+Definition followed (per head):
 
 * S_ij = scale * Q_i . K_j  ("DL0056 FlashAttention", "Where:" after the
   Mathematical Formulation, with scale = 1/sqrt(d) there; here ``scale`` is an
   argument and the workloads pass 1/sqrt(d)).
-* causal: S_ij = -inf for j > i, square and top-left aligned ("FlashAttention"
-  glossary, Causal Masking bullet: no token attends to a future token).
+* causal: S_ij = -inf for j > i + (Nk - Nq) ("FlashAttention" glossary,
+  Causal Masking bullet: no token attends to a future token).  For Nq = Nk
+  this is the square, top-left aligned mask; for Nq != Nk the queries are the
+  LAST Nq positions of the key sequence (bottom-right alignment), the reading
+  under which query i sits at position i + Nk - Nq.
+* a query row that sees no key at all (only possible when Nk < Nq under the
+  causal mask) has an empty softmax: its sum l_i is the empty sum 0, so
+  LSE_i = ln 0 = -inf, O_i = 0, and it contributes nothing to any gradient.
 * P = softmax over each row of S ("Flash Attention" glossary, "Why Regular
   Attention Becomes a Bottleneck": scores, softmax weights, combine values).
 * stored statistic LSE_i = m_i + ln(l_i) with m_i = max_j S_ij and
@@ -20,6 +26,8 @@ Definition followed (per head; Q, K, V, dO are [N, d]):
   the normalised probabilities after the softmax ("FlashAttention" glossary,
   Dropout bullet; reading recorded in the design notes).
 * O = P_d V.
+
+Q and dO are [Nq, d]; K and V are [Nk, d].
 
 Backward: the analytic gradient of O = P_d V for an upstream gradient dO,
     dV = P_d^T dO,   dP_d = dO V^T,   dP = dP_d * Z / (1 - p),
@@ -46,15 +54,31 @@ def _as64(x):
 
 
 def scores(q, k, scale, causal, rows=None, cols=None):
-    """S[rows, cols] = scale * Q[rows] K[cols]^T with the causal mask (-inf above the diagonal)."""
+    """S[rows, cols] = scale * Q[rows] K[cols]^T with the causal mask: -inf where
+    key j lies after query i's position i + Nk - Nq."""
     q, k = _as64(q), _as64(k)
     n = k.shape[0]
+    offset = n - q.shape[0]
     rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
     cols = np.arange(n) if cols is None else np.asarray(cols, dtype=np.int64)
     s = scale * (q[rows] @ k[cols].T)
     if causal:
-        s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+        s = np.where(cols[None, :] > rows[:, None] + offset, -np.inf, s)
     return s
+
+
+def softmax_rows(s):
+    """(P, LSE) of each row of S.  A row with no finite entry (no visible key)
+    gets P = 0 and LSE = -inf: the empty sum is 0 and ln 0 = -inf."""
+    m = s.max(axis=1)
+    seen = np.isfinite(m)
+    m_safe = np.where(seen, m, 0.0)
+    e = np.exp(s - m_safe[:, None])
+    l = e.sum(axis=1)
+    p = e / np.where(seen, l, 1.0)[:, None]
+    with np.errstate(divide="ignore"):
+        lse = np.where(seen, m_safe + np.log(np.where(seen, l, 1.0)), -np.inf)
+    return p, lse
 
 
 def dropout_factor(seed, b, h, rows, cols, p_drop):
@@ -76,11 +100,7 @@ def forward(q, k, v, *, causal, scale, p_drop=0.0, seed=0, b=0, h=0, rows=None, 
     rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows, dtype=np.int64)
     cols = np.arange(n)
     s = scores(q, k, scale, causal, rows, cols)
-    m = s.max(axis=1)
-    e = np.exp(s - m[:, None])
-    l = e.sum(axis=1)
-    p = e / l[:, None]
-    lse = m + np.log(l)
+    p, lse = softmax_rows(s)
     pd = p * dropout_factor(seed, b, h, rows, cols, p_drop)
     o = pd @ v
     if return_p:
@@ -91,13 +111,11 @@ def forward(q, k, v, *, causal, scale, p_drop=0.0, seed=0, b=0, h=0, rows=None, 
 def backward(q, k, v, do, *, causal, scale, p_drop=0.0, seed=0, b=0, h=0):
     """(dQ, dK, dV, D) of one head for the loss gradient dO, full materialisation."""
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
-    n = q.shape[0]
-    rows = np.arange(n)
-    s = scores(q, k, scale, causal, rows, rows)
-    m = s.max(axis=1)
-    e = np.exp(s - m[:, None])
-    p = e / e.sum(axis=1)[:, None]
-    f = dropout_factor(seed, b, h, rows, rows, p_drop)
+    rows = np.arange(q.shape[0])
+    cols = np.arange(k.shape[0])
+    s = scores(q, k, scale, causal, rows, cols)
+    p, _ = softmax_rows(s)
+    f = dropout_factor(seed, b, h, rows, cols, p_drop)
     pd = p * f
     dv = pd.T @ do
     dpd = do @ v.T
@@ -126,12 +144,8 @@ def row_stats(q, k, v, do, *, causal, scale, p_drop=0.0, seed=0, b=0, h=0, rows=
     for a in range(0, len(rows), block):
         rb = rows[a:a + block]
         s = scores(q, k, scale, causal, rb, cols)
-        m = s.max(axis=1)
-        e = np.exp(s - m[:, None])
-        l = e.sum(axis=1)
-        p = e / l[:, None]
+        p, lse[a:a + block] = softmax_rows(s)
         f = dropout_factor(seed, b, h, rb, cols, p_drop)
-        lse[a:a + block] = m + np.log(l)
         o[a:a + block] = (p * f) @ v
         dp = (do[rb] @ v.T) * f
         d_row[a:a + block] = (p * dp).sum(axis=1)
@@ -148,9 +162,7 @@ def grad_rows(q, k, v, do, *, causal, scale, p_drop=0.0, seed=0, b=0, h=0, rows,
     for a in range(0, len(rows), block):
         rb = rows[a:a + block]
         s = scores(q, k, scale, causal, rb, cols)
-        m = s.max(axis=1)
-        e = np.exp(s - m[:, None])
-        p = e / e.sum(axis=1)[:, None]
+        p, _ = softmax_rows(s)
         f = dropout_factor(seed, b, h, rb, cols, p_drop)
         dp = (do[rb] @ v.T) * f
         d_row = (p * dp).sum(axis=1)
@@ -162,7 +174,7 @@ def grad_cols(q, k, v, do, lse_all, d_all, *, causal, scale, p_drop=0.0, seed=0,
     """dK[cols], dV[cols] given LSE_i and D_i of every query row of the head.
 
     dV_j = sum_i P_d,ij dO_i and dK_j = scale * sum_i P_ij (dP_ij - D_i) Q_i with
-    P_ij = exp(S_ij - LSE_i).
+    P_ij = exp(S_ij - LSE_i) (0 for a row with LSE_i = -inf, which sees no key).
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
     n = q.shape[0]
@@ -172,7 +184,8 @@ def grad_cols(q, k, v, do, lse_all, d_all, *, causal, scale, p_drop=0.0, seed=0,
     for a in range(0, n, block):
         rb = np.arange(a, min(n, a + block))
         s = scores(q, k, scale, causal, rb, cols)
-        p = np.exp(s - lse_all[rb][:, None])
+        lse_rb = lse_all[rb]
+        p = np.where(np.isfinite(lse_rb)[:, None], np.exp(s - np.where(np.isfinite(lse_rb), lse_rb, 0.0)[:, None]), 0.0)
         f = dropout_factor(seed, b, h, rb, cols, p_drop)
         dv += (p * f).T @ do[rb]
         dp = (do[rb] @ v[cols].T) * f

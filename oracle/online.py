@@ -41,4 +41,8 @@ def forward_online(q, k, v, *, causal, scale, tile, p_drop=0.0, seed=0, b=0, h=0
         l = alpha * l + e.sum(axis=1)
         acc = alpha[:, None] * acc + (e * dropout_factor(seed, b, h, rows, cols, p_drop)) @ v[cols]
         m = m_new
-    return acc / l[:, None], m + np.log(l)
+    # a row that saw no key keeps l = 0: O = 0 and LSE = ln 0 = -inf (empty softmax)
+    seen = l > 0
+    with np.errstate(divide="ignore"):
+        return (np.where(seen[:, None], acc / np.where(seen, l, 1.0)[:, None], 0.0),
+                np.where(seen, m + np.log(np.where(seen, l, 1.0)), -np.inf))

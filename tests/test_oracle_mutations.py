@@ -120,3 +120,20 @@ def test_keep_tie_break_at_threshold():
     assert eq.any()
     assert z[eq].all()
     assert not z[u == t - 1].any()
+
+
+def test_top_left_alignment_for_rectangular_is_caught():
+    """With Nq < Nk a mask that ignores the offset (top-left alignment) gives
+    prefix means that are too short: the bottom-right closed form rejects it."""
+    rng = np.random.default_rng(8)
+    nq, nk, d = 4, 10, 3
+    q = np.zeros((nq, d))
+    k, v = rng.standard_normal((nk, d)), rng.standard_normal((nk, d))
+    s = np.where(np.arange(nk)[None, :] > np.arange(nq)[:, None], -np.inf, 0.2 * q @ k.T)  # no offset
+    p = np.exp(s - s.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    mutant = p @ v
+    want = np.stack([v[:i + nk - nq + 1].mean(0) for i in range(nq)])
+    assert np.abs(mutant - want).max() > 1e-3
+    got, _ = attention.forward(q, k, v, causal=True, scale=0.2)
+    assert np.abs(got - want).max() < 1e-12
