@@ -46,6 +46,17 @@ def load_library(path=None):
     lib.fa_bwd.restype = i
     lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, i, vp, sz, vp]
     lib.fa_bwd_ex.restype = i
+    lib.fa_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, u64, i, vp]
+    lib.fa_fwd_qk.restype = i
+    lib.fa_bwd_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, u64, i, vp, sz, vp]
+    lib.fa_bwd_qk.restype = i
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, u64, i, vp]
+    lib.fa_fwd_varlen.restype = i
+    lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_varlen_workspace_size.restype = sz
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, u64, i,
+                                  vp, sz, vp]
+    lib.fa_bwd_varlen.restype = i
     lib.fa_bwd_prepare.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_prepare.restype = i
     lib.fa_bwd_tiles.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, u64, vp, sz, vp]
@@ -91,23 +102,29 @@ def _raise(st, what):
 
 
 def fa_fwd(q, k, v, causal, scale=None, p_drop=0.0, seed=0, out=None, lse=None):
-    """(O, LSE) of exact attention; q, k, v [B, H, N, d] on one CUDA device, all
-    bf16 (fa_fwd) or all fp16 (fa_fwd_ex)."""
+    """(O, LSE) of exact attention on one CUDA device: q [B, H, Nq, d], k and v
+    [B, H, Nk, d], all bf16 or all fp16.  Square bf16 problems go to fa_fwd,
+    square fp16 ones to fa_fwd_ex, Nq != Nk to fa_fwd_qk."""
     lib = load_library()
     _check_bhnd("q", q)
-    _check_bhnd("k", k, q.shape, q.dtype)
-    _check_bhnd("v", v, q.shape, q.dtype)
-    B, H, N, d = q.shape
+    B, H, Nq, d = q.shape
+    _check_bhnd("k", k, None, q.dtype)
+    Nk = k.shape[2]
+    if (k.shape[0], k.shape[1], k.shape[3]) != (B, H, d):
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, Nk, {d}]")
+    _check_bhnd("v", v, k.shape, q.dtype)
     scale = d ** -0.5 if scale is None else scale
     out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
     _check_bhnd("out", out, q.shape, q.dtype)
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, N, d, int(bool(causal)),
-            float(scale), float(p_drop), int(seed) & (2**64 - 1))
-    if q.dtype == torch.bfloat16:
-        _raise(lib.fa_fwd(*args, _stream(q)), "fa_fwd")
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
+    tail = (d, int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1))
+    if Nq != Nk:
+        _raise(lib.fa_fwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_qk")
+    elif q.dtype == torch.bfloat16:
+        _raise(lib.fa_fwd(*ptrs, B, H, Nq, *tail, _stream(q)), "fa_fwd")
     else:
-        _raise(lib.fa_fwd_ex(*args, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_ex")
+        _raise(lib.fa_fwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_ex")
     return out, lse
 
 
@@ -118,30 +135,111 @@ def fa_bwd_workspace_size(B, H, N, d):
 def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspace=None, dq=None, dk=None,
            dv=None):
     """(dQ, dK, dV) of sum(dO * O) by recomputation; same arguments as the matching fa_fwd call
-    (bf16 tensors go to fa_bwd, fp16 ones to fa_bwd_ex)."""
+    (square bf16 tensors go to fa_bwd, square fp16 ones to fa_bwd_ex, Nq != Nk to fa_bwd_qk)."""
     lib = load_library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
+    for name, t in (("q", q), ("o", o), ("do", do)):
         _check_bhnd(name, t, q.shape, q.dtype)
-    B, H, N, d = q.shape
+    B, H, Nq, d = q.shape
+    _check_bhnd("k", k, None, q.dtype)
+    Nk = k.shape[2]
+    if (k.shape[0], k.shape[1], k.shape[3]) != (B, H, d):
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, Nk, {d}]")
+    _check_bhnd("v", v, k.shape, q.dtype)
     scale = d ** -0.5 if scale is None else scale
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
-    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Nq] tensor")
+    ws_bytes = fa_bwd_workspace_size(B, H, Nq, d)
     if workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _check_bhnd(name, t, q.shape, q.dtype)
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
-            dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), float(p_drop),
-            int(seed) & (2**64 - 1))
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    _check_bhnd("dq", dq, q.shape, q.dtype)
+    _check_bhnd("dk", dk, k.shape, q.dtype)
+    _check_bhnd("dv", dv, k.shape, q.dtype)
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr())
+    tail = (d, int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1))
     ws = (workspace.data_ptr(), workspace.numel(), _stream(q))
-    if q.dtype == torch.bfloat16:
-        _raise(lib.fa_bwd(*args, *ws), "fa_bwd")
+    if Nq != Nk:
+        _raise(lib.fa_bwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], *ws), "fa_bwd_qk")
+    elif q.dtype == torch.bfloat16:
+        _raise(lib.fa_bwd(*ptrs, B, H, Nq, *tail, *ws), "fa_bwd")
     else:
-        _raise(lib.fa_bwd_ex(*args, FA_DTYPE[q.dtype], *ws), "fa_bwd_ex")
+        _raise(lib.fa_bwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], *ws), "fa_bwd_ex")
+    return dq, dk, dv
+
+
+def _check_packed(name, t, dtype=None, rows=None, H=None, d=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in FA_DTYPE or (dtype is not None and t.dtype != dtype):
+        raise ValueError(f"{name} must be bf16 or fp16, the type of q")
+    if t.dim() != 3 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [total, H, d] tensor")
+    if (rows is not None and t.shape[0] != rows) or (H is not None and t.shape[1] != H) or \
+            (d is not None and t.shape[2] != d):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}")
+
+
+def _check_cu(name, cu, B):
+    if not cu.is_cuda or cu.dtype != torch.int32 or cu.dim() != 1 or cu.numel() != B + 1 or not cu.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B + 1 offsets")
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, scale=None, p_drop=0.0,
+                  seed=0, out=None, lse=None):
+    """(O [total_q, H, d], LSE [H, total_q]) of B packed sequences: q [total_q, H, d],
+    k, v [total_k, H, d], int32 offsets cu_seqlens_q / cu_seqlens_k [B + 1] on the device."""
+    lib = load_library()
+    _check_packed("q", q)
+    total_q, H, d = q.shape
+    _check_packed("k", k, q.dtype, None, H, d)
+    total_k = k.shape[0]
+    _check_packed("v", v, q.dtype, total_k, H, d)
+    B = cu_seqlens_q.numel() - 1
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    scale = d ** -0.5 if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, total_q), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check_packed("out", out, q.dtype, total_q, H, d)
+    _raise(lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q, total_k,
+                             int(max_seqlen_q), int(max_seqlen_k), d, int(bool(causal)), float(scale), float(p_drop),
+                             int(seed) & (2**64 - 1), FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_varlen")
+    return out, lse
+
+
+def fa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, scale=None,
+                  p_drop=0.0, seed=0, workspace=None, dq=None, dk=None, dv=None):
+    """(dQ, dK, dV) of the matching fa_fwd_varlen call, in the same packed layouts."""
+    lib = load_library()
+    _check_packed("q", q)
+    total_q, H, d = q.shape
+    _check_packed("k", k, q.dtype, None, H, d)
+    total_k = k.shape[0]
+    _check_packed("v", v, q.dtype, total_k, H, d)
+    _check_packed("o", o, q.dtype, total_q, H, d)
+    _check_packed("do", do, q.dtype, total_q, H, d)
+    B = cu_seqlens_q.numel() - 1
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (H, total_q) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [H, total_q] tensor")
+    scale = d ** -0.5 if scale is None else scale
+    ws_bytes = int(lib.fa_bwd_varlen_workspace_size(B, H, total_q, int(max_seqlen_q), d))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    _raise(lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(),
+                             cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
+                             int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1),
+                             FA_DTYPE[q.dtype], workspace.data_ptr(), workspace.numel(), _stream(q)),
+           "fa_bwd_varlen")
     return dq, dk, dv
 
 

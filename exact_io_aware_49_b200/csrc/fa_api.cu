@@ -35,19 +35,21 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH, N, d] row-major 3-D map with 128-byte boxes per row (64 bf16 / fp16
-// or 32 fp32 columns) x 128 rows x 1 head and 128-byte swizzle.  Rows past N
-// of a head are outside the tensor: loads zero-fill them, reductions skip them.
-bool encode_head_map(CUtensorMap* tm, const void* base, long long BH, int N, int d, CUtensorMapDataType dt) {
+// 3-D map (d, T, G) over a 16-bit or fp32 tensor: column, token row, head
+// coordinate, with token stride ``tok`` and head stride ``grp`` (elements).
+// Boxes are 128 bytes of a row (64 16-bit or 32 fp32 columns) x 128 rows x 1
+// head with 128-byte swizzle.  Rows past T are outside the tensor: loads
+// zero-fill them, reductions skip them.
+bool encode_map(CUtensorMap* tm, const void* base, int d, long long T, long long G, long long tok, long long grp,
+                CUtensorMapDataType dt) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t esize = (dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 4 : 2;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize, static_cast<cuuint64_t>(N) * d * esize};
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(G)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(tok) * esize, static_cast<cuuint64_t>(grp) * esize};
   cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(tm, dt, 3,
-                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = enc(tm, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -71,14 +73,12 @@ bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Shared validation of sizes / scalars.  Returns FA_OK or the error.
-fa_status check_common(int B, int H, int N, int d, float scale, float p_drop) {
-  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+long long pad128(long long n) { return (n + 127) / 128 * 128; }
+
+fa_status check_scalars(int d, float scale, float p_drop) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  const long long rows = static_cast<long long>(B) * H * N;
-  if (rows >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -86,6 +86,218 @@ uint32_t drop_threshold(float p_drop) {
   // round-half-even(p * 65536) in double precision (default rounding mode)
   return static_cast<uint32_t>(nearbyint(static_cast<double>(p_drop) * 65536.0));
 }
+
+// One validated problem: the sequence layout plus the scalars every stage needs.
+struct Problem {
+  fa::SeqLayout seq;
+  int d;
+  int causal;
+  float scale;
+  float p_drop;
+  uint64_t seed;
+  bool f16;
+  long long groups() const { return seq.cu_q ? seq.H : static_cast<long long>(seq.B) * seq.H; }
+};
+
+// Fixed lengths: [B, H, Nq, d] queries, [B, H, Nk, d] keys.
+fa_status fixed_problem(Problem* pb, int B, int H, int Nq, int Nk, int d, int causal, float scale, float p_drop,
+                        uint64_t seed, bool f16) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  fa_status st = check_scalars(d, scale, p_drop);
+  if (st != FA_OK) return st;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh * (Nq > Nk ? Nq : Nk) >= (1ll << 31) || bh * pad128(Nq) >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  memset(pb, 0, sizeof(*pb));
+  pb->seq.B = B;
+  pb->seq.H = H;
+  pb->seq.Nq = Nq;
+  pb->seq.Nk = Nk;
+  pb->seq.total_q = Nq;
+  pb->seq.total_k = Nk;
+  pb->seq.tok_stride = d;
+  pb->seq.q_head_stride = static_cast<long long>(Nq) * d;
+  pb->seq.k_head_stride = static_cast<long long>(Nk) * d;
+  pb->d = d;
+  pb->causal = causal ? 1 : 0;
+  pb->scale = scale;
+  pb->p_drop = p_drop;
+  pb->seed = seed;
+  pb->f16 = f16;
+  return FA_OK;
+}
+
+// Packed variable lengths: [total_q, H, d] queries, [total_k, H, d] keys,
+// device offsets cu_q / cu_k [B + 1].
+fa_status packed_problem(Problem* pb, const int* cu_q, const int* cu_k, int B, int H, int total_q, int total_k,
+                         int max_q, int max_k, int d, int causal, float scale, float p_drop, uint64_t seed,
+                         bool f16) {
+  if (!cu_q || !cu_k || misaligned(cu_q, 4) || misaligned(cu_k, 4)) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || total_q <= 0 || total_k <= 0 || max_q <= 0 || max_k <= 0 || d <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (max_q > total_q || max_k > total_k) return FA_ERR_INVALID_ARG;
+  fa_status st = check_scalars(d, scale, p_drop);
+  if (st != FA_OK) return st;
+  const long long bh = static_cast<long long>(B) * H;
+  if (static_cast<long long>(H) * (total_q > total_k ? total_q : total_k) >= (1ll << 31) ||
+      bh * pad128(max_q) >= (1ll << 31) || bh * ((max_k + 127) / 128) >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
+  memset(pb, 0, sizeof(*pb));
+  pb->seq.cu_q = cu_q;
+  pb->seq.cu_k = cu_k;
+  pb->seq.B = B;
+  pb->seq.H = H;
+  pb->seq.Nq = max_q;
+  pb->seq.Nk = max_k;
+  pb->seq.total_q = total_q;
+  pb->seq.total_k = total_k;
+  pb->seq.tok_stride = static_cast<long long>(H) * d;
+  pb->seq.q_head_stride = d;
+  pb->seq.k_head_stride = d;
+  pb->d = d;
+  pb->causal = causal ? 1 : 0;
+  pb->scale = scale;
+  pb->p_drop = p_drop;
+  pb->seed = seed;
+  pb->f16 = f16;
+  return FA_OK;
+}
+
+// Workspace: fp32 dQ accumulator [G, total_q, d], then the fp32 D and
+// LSE * log2(e) vectors [B * H, pad128(Nq)], each part rounded to 256 bytes.
+size_t workspace_bytes(const Problem& pb) {
+  const size_t acc = static_cast<size_t>(pb.groups()) * pb.seq.total_q * pb.d * sizeof(float);
+  const size_t vec = static_cast<size_t>(pb.seq.B) * pb.seq.H * pad128(pb.seq.Nq) * sizeof(float);
+  return round_up(acc, 256) + 2 * round_up(vec, 256);
+}
+
+bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base) {
+  return encode_map(tm, base, pb.d, pb.seq.total_q, pb.groups(), pb.seq.tok_stride, pb.seq.q_head_stride,
+                    elem_type(pb.f16));
+}
+
+bool encode_k_like(const Problem& pb, CUtensorMap* tm, const void* base) {
+  return encode_map(tm, base, pb.d, pb.seq.total_k, pb.groups(), pb.seq.tok_stride, pb.seq.k_head_stride,
+                    elem_type(pb.f16));
+}
+
+void fill_common(const Problem& pb, fa::SeqLayout* seq, int* d, int* causal, float* scale_log2, uint32_t* drop_t,
+                 float* drop_scale, uint32_t* seed_lo, uint32_t* seed_hi, uint32_t (&rk)[20]) {
+  *seq = pb.seq;
+  *d = pb.d;
+  *causal = pb.causal;
+  *scale_log2 = static_cast<float>(static_cast<double>(pb.scale) * 1.4426950408889634);
+  *drop_t = drop_threshold(pb.p_drop);
+  *drop_scale = *drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(pb.p_drop))) : 1.0f;
+  *seed_lo = static_cast<uint32_t>(pb.seed);
+  *seed_hi = static_cast<uint32_t>(pb.seed >> 32);
+  fa::philox_round_keys(pb.seed, rk);
+}
+
+fa_status fwd_run(const Problem& pb, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                  void* stream) {
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(LSE, 16))
+    return FA_ERR_INVALID_ARG;
+  fa::FwdArgs a;
+  memset(&a, 0, sizeof(a));
+  if (!encode_q_like(pb, &a.tmQ, Q) || !encode_k_like(pb, &a.tmK, K) || !encode_k_like(pb, &a.tmV, V))
+    return FA_ERR_CUDA;
+  a.f16 = pb.f16 ? 1 : 0;
+  a.O = O;
+  a.LSE = LSE;
+  a.err = error_word_ptr();
+  if (!a.err) return FA_ERR_CUDA;
+  fill_common(pb, &a.seq, &a.d, &a.causal, &a.scale_log2, &a.drop_t, &a.drop_scale, &a.seed_lo, &a.seed_hi,
+              a.philox_rk);
+  return fa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status check_workspace(const Problem& pb, const void* workspace, size_t bytes) {
+  if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
+  if (bytes < workspace_bytes(pb)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+void bwd_args(const Problem& pb, fa::BwdArgs* a, void* workspace) {
+  memset(a, 0, sizeof(*a));
+  float scale_log2;
+  fill_common(pb, &a->seq, &a->d, &a->causal, &scale_log2, &a->drop_t, &a->drop_scale, &a->seed_lo, &a->seed_hi,
+              a->philox_rk);
+  a->scale = pb.scale;
+  a->scale_log2 = scale_log2;
+  a->f16 = pb.f16 ? 1 : 0;
+  char* ws = static_cast<char*>(workspace);
+  const size_t acc = round_up(static_cast<size_t>(pb.groups()) * pb.seq.total_q * pb.d * sizeof(float), 256);
+  const size_t vec = round_up(static_cast<size_t>(pb.seq.B) * pb.seq.H * pad128(pb.seq.Nq) * sizeof(float), 256);
+  a->dQacc = reinterpret_cast<float*>(ws);
+  a->Dvec = reinterpret_cast<float*>(ws + acc);
+  a->lse2 = reinterpret_cast<float*>(ws + acc + vec);
+}
+
+fa_status prepare_run(const Problem& pb, const void* O, const void* dO, const float* LSE, void* workspace,
+                      size_t bytes, void* stream) {
+  if (!O || !dO || !LSE) return FA_ERR_INVALID_ARG;
+  if (misaligned(O, 16) || misaligned(dO, 16) || misaligned(LSE, 16)) return FA_ERR_INVALID_ARG;
+  fa_status st = check_workspace(pb, workspace, bytes);
+  if (st != FA_OK) return st;
+  fa::BwdArgs a;
+  bwd_args(pb, &a, workspace);
+  a.O = O;
+  a.dO = dO;
+  a.LSE = LSE;
+  return fa::launch_bwd_prepare(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status tiles_run(const Problem& pb, const void* Q, const void* K, const void* V, const void* dO, void* dK,
+                    void* dV, void* workspace, size_t bytes, void* stream) {
+  if (!Q || !K || !V || !dO || !dK || !dV) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) || misaligned(dK, 16) ||
+      misaligned(dV, 16))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_workspace(pb, workspace, bytes);
+  if (st != FA_OK) return st;
+  fa::BwdArgs a;
+  bwd_args(pb, &a, workspace);
+  if (!encode_q_like(pb, &a.tmQ, Q) || !encode_k_like(pb, &a.tmK, K) || !encode_k_like(pb, &a.tmV, V) ||
+      !encode_q_like(pb, &a.tmDO, dO))
+    return FA_ERR_CUDA;
+  // the accumulator is [G, total_q, d] fp32, contiguous
+  if (!encode_map(&a.tmDQacc, a.dQacc, pb.d, pb.seq.total_q, pb.groups(), pb.d,
+                  static_cast<long long>(pb.seq.total_q) * pb.d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+    return FA_ERR_CUDA;
+  a.dO = dO;
+  a.dK = dK;
+  a.dV = dV;
+  a.err = error_word_ptr();
+  if (!a.err) return FA_ERR_CUDA;
+  return fa::launch_bwd_tiles(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status finish_run(const Problem& pb, void* dQ, const void* workspace, size_t bytes, void* stream) {
+  if (!dQ || misaligned(dQ, 16)) return FA_ERR_INVALID_ARG;
+  fa_status st = check_workspace(pb, workspace, bytes);
+  if (st != FA_OK) return st;
+  fa::BwdArgs a;
+  bwd_args(pb, &a, const_cast<void*>(workspace));
+  a.dQ = dQ;
+  return fa::launch_bwd_finish(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_run(const Problem& pb, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                  const float* LSE, void* dQ, void* dK, void* dV, void* workspace, size_t bytes, void* stream) {
+  // Validate everything up front so a rejected call launches none of the stages.
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
+      misaligned(LSE, 16) || misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16))
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_workspace(pb, workspace, bytes);
+  if (st != FA_OK) return st;
+  if ((st = prepare_run(pb, O, dO, LSE, workspace, bytes, stream)) != FA_OK) return st;
+  if ((st = tiles_run(pb, Q, K, V, dO, dK, dV, workspace, bytes, stream)) != FA_OK) return st;
+  return finish_run(pb, dQ, workspace, bytes, stream);
+}
+
+bool dtype_ok(fa_dtype dtype) { return dtype == FA_DTYPE_BF16 || dtype == FA_DTYPE_F16; }
 
 }  // namespace
 
@@ -102,221 +314,131 @@ const char* fa_status_string(fa_status s) {
   return "unknown fa_status";
 }
 
-}  // extern "C"
-
-namespace {
-
-fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
-                   int causal, float scale, float p_drop, uint64_t seed, bool f16, void* stream) {
-  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
-  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(LSE, 16))
-    return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, scale, p_drop);
-  if (st != FA_OK) return st;
-
-  fa::FwdArgs a;
-  memset(&a, 0, sizeof(a));
-  const long long BH = static_cast<long long>(B) * H;
-  const CUtensorMapDataType dt = elem_type(f16);
-  if (!encode_head_map(&a.tmQ, Q, BH, N, d, dt) || !encode_head_map(&a.tmK, K, BH, N, d, dt) ||
-      !encode_head_map(&a.tmV, V, BH, N, d, dt))
-    return FA_ERR_CUDA;
-  a.f16 = f16 ? 1 : 0;
-  a.O = O;
-  a.LSE = LSE;
-  a.err = error_word_ptr();
-  if (!a.err) return FA_ERR_CUDA;
-  a.B = B;
-  a.H = H;
-  a.N = N;
-  a.d = d;
-  a.causal = causal ? 1 : 0;
-  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  a.drop_t = drop_threshold(p_drop);
-  a.drop_scale = a.drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
-  a.seed_lo = static_cast<uint32_t>(seed);
-  a.seed_hi = static_cast<uint32_t>(seed >> 32);
-  fa::philox_round_keys(seed, a.philox_rk);
-  return fa::launch_fwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-bool dtype_ok(fa_dtype dtype) { return dtype == FA_DTYPE_BF16 || dtype == FA_DTYPE_F16; }
-
-}  // namespace
-
-extern "C" {
+// ------------------------------------------------------------ forward
 
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
                  int causal, float scale, float p_drop, uint64_t seed, void* stream) {
-  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, causal, scale, p_drop, seed, false, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, causal, scale, p_drop, seed, false);
+  return st != FA_OK ? st : fwd_run(pb, Q, K, V, O, LSE, stream);
 }
 
 fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
                     int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, void* stream) {
   if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
-  return fwd_impl(Q, K, V, O, LSE, B, H, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : fwd_run(pb, Q, K, V, O, LSE, stream);
 }
+
+fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int Nq, int Nk,
+                    int d, int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, Nq, Nk, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : fwd_run(pb, Q, K, V, O, LSE, stream);
+}
+
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q,
+                        int max_seqlen_k, int d, int causal, float scale, float p_drop, uint64_t seed,
+                        fa_dtype dtype, void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  fa_status st = packed_problem(&pb, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                                d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : fwd_run(pb, Q, K, V, O, LSE, stream);
+}
+
+// ------------------------------------------------------------ backward
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  Problem pb;
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  const size_t rows_pad = static_cast<size_t>(B) * H * ((static_cast<size_t>(N) + 127) / 128 * 128);
-  return round_up(rows * d * sizeof(float), 256) + 2 * round_up(rows_pad * sizeof(float), 256);
+  memset(&pb, 0, sizeof(pb));
+  pb.seq.B = B;
+  pb.seq.H = H;
+  pb.seq.Nq = N;
+  pb.seq.total_q = N;
+  pb.d = d;
+  return workspace_bytes(pb);
 }
 
-}  // extern "C"
-
-namespace {
-
-// Workspace carve-up shared by the backward entry points.
-void carve_workspace(fa::BwdArgs* a, void* workspace) {
-  char* ws = static_cast<char*>(workspace);
-  const size_t rows = static_cast<size_t>(a->B) * a->H * a->N;
-  const size_t rows_pad = static_cast<size_t>(a->B) * a->H * ((static_cast<size_t>(a->N) + 127) / 128 * 128);
-  const size_t acc_bytes = round_up(rows * a->d * sizeof(float), 256);
-  const size_t vec_bytes = round_up(rows_pad * sizeof(float), 256);
-  a->dQacc = reinterpret_cast<float*>(ws);
-  a->Dvec = reinterpret_cast<float*>(ws + acc_bytes);
-  a->lse2 = reinterpret_cast<float*>(ws + acc_bytes + vec_bytes);
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d) {
+  Problem pb;
+  if (B <= 0 || H <= 0 || total_q <= 0 || max_seqlen_q <= 0 || d <= 0) return 0;
+  memset(&pb, 0, sizeof(pb));
+  pb.seq.cu_q = reinterpret_cast<const int*>(1);  // packed layout: G = H
+  pb.seq.B = B;
+  pb.seq.H = H;
+  pb.seq.Nq = max_seqlen_q;
+  pb.seq.total_q = total_q;
+  pb.d = d;
+  return workspace_bytes(pb);
 }
-
-fa_status check_workspace(const void* workspace, size_t workspace_bytes, int B, int H, int N, int d) {
-  if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
-  return FA_OK;
-}
-
-void fill_scalars(fa::BwdArgs* a, int B, int H, int N, int d, int causal, float scale, float p_drop,
-                  uint64_t seed) {
-  a->B = B;
-  a->H = H;
-  a->N = N;
-  a->d = d;
-  a->causal = causal ? 1 : 0;
-  a->scale = scale;
-  a->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  a->drop_t = drop_threshold(p_drop);
-  a->drop_scale = a->drop_t ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop))) : 1.0f;
-  a->seed_lo = static_cast<uint32_t>(seed);
-  a->seed_hi = static_cast<uint32_t>(seed >> 32);
-  fa::philox_round_keys(seed, a->philox_rk);
-}
-
-fa_status prepare_impl(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
-                       void* workspace, size_t workspace_bytes, bool f16, void* stream) {
-  if (!O || !dO || !LSE) return FA_ERR_INVALID_ARG;
-  if (misaligned(O, 16) || misaligned(dO, 16) || misaligned(LSE, 16)) return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, 1.0f, 0.0f);
-  if (st != FA_OK) return st;
-  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
-  fa::BwdArgs a;
-  memset(&a, 0, sizeof(a));
-  fill_scalars(&a, B, H, N, d, 0, 1.0f, 0.0f, 0);
-  carve_workspace(&a, workspace);
-  a.f16 = f16 ? 1 : 0;
-  a.O = O;
-  a.dO = dO;
-  a.LSE = LSE;
-  return fa::launch_bwd_prepare(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-fa_status tiles_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
-                     int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
-                     size_t workspace_bytes, bool f16, void* stream) {
-  if (!Q || !K || !V || !dO || !dK || !dV) return FA_ERR_INVALID_ARG;
-  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) || misaligned(dK, 16) ||
-      misaligned(dV, 16))
-    return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, scale, p_drop);
-  if (st != FA_OK) return st;
-  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
-  fa::BwdArgs a;
-  memset(&a, 0, sizeof(a));
-  const long long BH = static_cast<long long>(B) * H;
-  const CUtensorMapDataType dt = elem_type(f16);
-  if (!encode_head_map(&a.tmQ, Q, BH, N, d, dt) || !encode_head_map(&a.tmK, K, BH, N, d, dt) ||
-      !encode_head_map(&a.tmV, V, BH, N, d, dt) || !encode_head_map(&a.tmDO, dO, BH, N, d, dt))
-    return FA_ERR_CUDA;
-  fill_scalars(&a, B, H, N, d, causal, scale, p_drop, seed);
-  carve_workspace(&a, workspace);
-  if (!encode_head_map(&a.tmDQacc, a.dQacc, BH, N, d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)) return FA_ERR_CUDA;
-  a.f16 = f16 ? 1 : 0;
-  a.dO = dO;
-  a.dK = dK;
-  a.dV = dV;
-  a.err = error_word_ptr();
-  if (!a.err) return FA_ERR_CUDA;
-  return fa::launch_bwd_tiles(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-fa_status finish_impl(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
-                      size_t workspace_bytes, bool f16, void* stream) {
-  if (!dQ || misaligned(dQ, 16)) return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, scale, 0.0f);
-  if (st != FA_OK) return st;
-  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
-  fa::BwdArgs a;
-  memset(&a, 0, sizeof(a));
-  fill_scalars(&a, B, H, N, d, 0, scale, 0.0f, 0);
-  carve_workspace(&a, const_cast<void*>(workspace));
-  a.f16 = f16 ? 1 : 0;
-  a.dQ = dQ;
-  return fa::launch_bwd_finish(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
-
-fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                   void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
-                   uint64_t seed, void* workspace, size_t workspace_bytes, bool f16, void* stream) {
-  // Validate everything up front so a rejected call launches none of the stages.
-  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return FA_ERR_INVALID_ARG;
-  if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(O, 16) || misaligned(dO, 16) ||
-      misaligned(LSE, 16) || misaligned(dQ, 16) || misaligned(dK, 16) || misaligned(dV, 16))
-    return FA_ERR_INVALID_ARG;
-  fa_status st = check_common(B, H, N, d, scale, p_drop);
-  if (st != FA_OK) return st;
-  if ((st = check_workspace(workspace, workspace_bytes, B, H, N, d)) != FA_OK) return st;
-  if ((st = prepare_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, f16, stream)) != FA_OK) return st;
-  if ((st = tiles_impl(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes, f16,
-                       stream)) != FA_OK)
-    return st;
-  return finish_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, f16, stream);
-}
-
-}  // namespace
-
-extern "C" {
 
 fa_status fa_bwd_prepare(const void* O, const void* dO, const float* LSE, int B, int H, int N, int d,
                          void* workspace, size_t workspace_bytes, void* stream) {
-  return prepare_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, false, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, 0, 1.0f, 0.0f, 0, false);
+  return st != FA_OK ? st : prepare_run(pb, O, dO, LSE, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_tiles(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int B,
                        int H, int N, int d, int causal, float scale, float p_drop, uint64_t seed, void* workspace,
                        size_t workspace_bytes, void* stream) {
-  return tiles_impl(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace, workspace_bytes, false,
-                    stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, causal, scale, p_drop, seed, false);
+  return st != FA_OK ? st : tiles_run(pb, Q, K, V, dO, dK, dV, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const void* workspace,
                         size_t workspace_bytes, void* stream) {
-  return finish_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, false, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, 0, scale, 0.0f, 0, false);
+  return st != FA_OK ? st : finish_run(pb, dQ, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                  void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
                  uint64_t seed, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace,
-                  workspace_bytes, false, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, causal, scale, p_drop, seed, false);
+  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                     void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale, float p_drop,
                     uint64_t seed, fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
   if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, p_drop, seed, workspace,
-                  workspace_bytes, dtype == FA_DTYPE_F16, stream);
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, N, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
+
+fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                    void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                    float p_drop, uint64_t seed, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  fa_status st = fixed_problem(&pb, B, H, Nq, Nk, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                        void* dQ, void* dK, void* dV, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                        int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                        int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  fa_status st = packed_problem(&pb, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q, max_seqlen_k,
+                                d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------ utilities
 
 fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed, void* stream) {
   if (!mask) return FA_ERR_INVALID_ARG;

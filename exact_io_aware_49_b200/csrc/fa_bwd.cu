@@ -48,36 +48,38 @@ namespace {
 
 // ============================================================ preprocess
 
-// One warp per padded row (b*H + h, i < Npad): for i < N, D = sum(dO * O),
-// LSE2 = LSE * log2(e) and the dQ accumulator row is zeroed; for the padding
-// rows of a partial last tile, D = 0 and LSE2 = +inf (so exp2(x - LSE2) = 0).
+// One warp per padded row (unit b*H + h, i < Npad): for the unit's queries
+// i < nq, D = sum(dO * O) and LSE2 = LSE * log2(e) (+inf for a row that sees
+// no key, LSE = -inf); for the padding rows, D = 0 and LSE2 = +inf (so
+// exp2(x - LSE2) = 0).  Then the whole fp32 dQ accumulator is zeroed.
 template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* __restrict__ O,
                                                                 const uint16_t* __restrict__ dO,
                                                                 const float* __restrict__ LSE,
                                                                 float* __restrict__ Dvec,
                                                                 float* __restrict__ lse2,
-                                                                float* __restrict__ dQacc, long long rows_pad,
-                                                                int N, int Npad) {
+                                                                float* __restrict__ dQacc, const SeqLayout seq,
+                                                                int Npad, long long acc_vec4) {
   const int lane = threadIdx.x & 31;
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long prow = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); prow < rows_pad;
-       prow += warps) {
-    const long long bh = prow / Npad;
-    const int i = static_cast<int>(prow - bh * Npad);
-    if (i >= N) {
+  const int rows_pad = seq.B * seq.H * Npad;  // < 2^31, checked on the host
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int prow = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); prow < rows_pad; prow += warps) {
+    const int unit = prow / Npad;
+    const int i = prow - unit * Npad;
+    const SeqUnit su = resolve_unit(seq, unit);
+    if (i >= su.nq) {
       if (lane == 0) {
         Dvec[prow] = 0.f;
         lse2[prow] = CUDART_INF_F;
       }
       continue;
     }
-    const long long row = bh * N + i;
+    const size_t row = static_cast<size_t>(su.q0 + i) * seq.tok_stride + static_cast<size_t>(su.g) * seq.q_head_stride;
     // lane covers elements [8*lane, 8*lane+8) when 8*lane < D
     float acc = 0.f;
     if (lane * 8 < D) {
-      const uint4 a = *reinterpret_cast<const uint4*>(O + row * D + lane * 8);
-      const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + lane * 8);
+      const uint4 a = *reinterpret_cast<const uint4*>(O + row + lane * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + row + lane * 8);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
       const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -90,23 +92,39 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    float4* zq = reinterpret_cast<float4*>(dQacc + row * D);
-    for (int c = lane; c < D / 4; c += 32) zq[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane == 0) {
+      const float l = LSE[static_cast<size_t>(su.g) * seq.total_q + su.q0 + i];
       Dvec[prow] = acc;
-      lse2[prow] = LSE[row] * 1.4426950408889634f;
+      lse2[prow] = (l == -CUDART_INF_F) ? CUDART_INF_F : l * 1.4426950408889634f;
     }
   }
+  float4* zq = reinterpret_cast<float4*>(dQacc);
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < acc_vec4;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x)
+    zq[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ============================================================ dQ convert
 
+// dQ row (g, t) = scale * accumulator row (g, t), rounded to the input type;
+// 8 elements per thread.
 template <bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ dQacc,
                                                                 uint16_t* __restrict__ dQ, float scale,
-                                                                long long n8) {
+                                                                const SeqLayout seq, int d, long long n8) {
+  const int shift = (d == 128) ? 4 : 3;  // log2(d / 8)
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n8;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    // fixed length: dQ has the accumulator's layout; packed: row g * total_q + t
+    // of the accumulator is token t of head g in [total_q, H, d]
+    long long dst = idx * 8;
+    if (seq.cu_q) {
+      const int row = static_cast<int>(idx >> shift);  // < 2^31 rows
+      const int part = static_cast<int>(idx & ((1 << shift) - 1));
+      const int g = row / seq.total_q;
+      const int t = row - g * seq.total_q;
+      dst = t * seq.tok_stride + g * seq.q_head_stride + part * 8;
+    }
     const float4 a = reinterpret_cast<const float4*>(dQacc)[2 * idx];
     const float4 b = reinterpret_cast<const float4*>(dQacc)[2 * idx + 1];
     uint4 o;
@@ -114,7 +132,7 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
     o.y = pack2<F16>(a.z * scale, a.w * scale);
     o.z = pack2<F16>(b.x * scale, b.y * scale);
     o.w = pack2<F16>(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dQ)[idx] = o;
+    *reinterpret_cast<uint4*>(dQ + dst) = o;
   }
 }
 
@@ -171,7 +189,7 @@ struct BwdParams {
   const float* lse2;
   const float* Dvec;
   unsigned* err;
-  int H, N;
+  SeqLayout seq;
   float scale;
   float scale_log2;
   uint32_t drop_t;
@@ -180,9 +198,20 @@ struct BwdParams {
   int group, BH;
 };
 
+// The MMA issuer rebuilds its shared-memory descriptors from the tile base
+// addresses at each use instead of keeping all of them live across its loop
+// (its warpgroup runs with few registers): an opaque copy of each base stops
+// the compiler from hoisting the descriptors out of the loop.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  asm volatile("mov.b32 %0, %0;" : "+r"(x));
+  return x;
+}
+
 // D[tmem] (+)= A[K-major tile] * B[K-major tile]^T, M = N = 128, K = D.
 template <int D, bool F16>
 __device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+  a_smem = opaque_u32(a_smem);
+  b_smem = opaque_u32(b_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
@@ -194,6 +223,7 @@ __device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, ui
 // dV (+)= P^T dO : A = P^T (TMEM, 16-bit pairs), B = dO tile (MN-major), K = 128 queries, N = D.
 template <int D, bool F16>
 __device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem, bool accumulate) {
+  do_smem = opaque_u32(do_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
@@ -204,6 +234,8 @@ __device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_
 // dK (+)= dS^T Q : A = dS^T (smem, K-major over queries), B = Q tile (MN-major), N = D.
 template <int D, bool F16>
 __device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32_t q_smem, bool accumulate) {
+  ds_smem = opaque_u32(ds_smem);
+  q_smem = opaque_u32(q_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
@@ -216,6 +248,8 @@ __device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32
 // dQ_i = dS K : A = dS (the dS^T tile read MN-major, M = queries), B = K tile (MN-major), N = D.
 template <int D, bool F16>
 __device__ __forceinline__ void mma_dq(uint32_t tmem_d, uint32_t ds_smem, uint32_t k_smem) {
+  ds_smem = opaque_u32(ds_smem);
+  k_smem = opaque_u32(k_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, true, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
@@ -296,20 +330,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // 1-D grid over (head group, key tile, head), heaviest key tiles first
-  // within each group of p.group heads.
-  const int N = p.N;
-  const int n_t = (N + 127) / 128;  // the last tile may be partial
-  const int Npad = n_t * 128;
-  const int per_group = p.group * n_t;
+  // 1-D grid over (unit group, key tile, unit), heaviest key tiles first
+  // within each group of p.group units.
+  const int n_kt_grid = (p.seq.Nk + 127) / 128;
+  const int Npad = (p.seq.Nq + 127) / 128 * 128;  // padded rows per unit in the LSE2 / D vectors
+  const int per_group = p.group * n_kt_grid;
   const int grp = blockIdx.x / per_group;
   const int rr = blockIdx.x - grp * per_group;
   const int gsz = min(p.group, p.BH - grp * p.group);
   const int kj = rr / gsz;                   // key tile (lowest first: the heaviest causal work)
-  const int bh = grp * p.group + (rr - kj * gsz);
-  const int q_first = CAUSAL ? kj : 0;
-  const int nq = n_t - q_first;              // query tiles visited
-  const size_t vrow0 = static_cast<size_t>(bh) * Npad;  // this head's rows in the padded LSE2 / D vectors
+  const int unit = grp * p.group + (rr - kj * gsz);
+  const SeqUnit su = resolve_unit(p.seq, unit);
+  if (kj * 128 >= su.nk) return;             // past this unit's keys: no work
+  const int n_qt = (su.nq + 127) / 128;
+  const int delta = su.nk - su.nq;           // query i sits at key position i + delta
+  // first query tile with a row that sees a key of this tile: i + delta >= kj * 128
+  const int q_first = CAUSAL ? max(0, floor_div(kj * 128 - delta, 128)) : 0;
+  const int nq = n_qt - q_first;             // query tiles visited
+  const bool key_valid = kj * 128 + static_cast<int>(threadIdx.x & 127) < su.nk;
+  if (nq <= 0) {
+    // no query sees these keys: dK = dV = 0 (threads 0-127 take dK, 128-255 dV)
+    if (threadIdx.x < 256 && key_valid) {
+      uint16_t* dst = ((threadIdx.x < 128) ? p.dK : p.dV) +
+                      static_cast<size_t>(su.k0 + kj * 128 + (threadIdx.x & 127)) * p.seq.tok_stride +
+                      static_cast<size_t>(su.g) * p.seq.k_head_stride;
+      uint4* d4 = reinterpret_cast<uint4*>(dst);
+      for (int e = 0; e < D / 8; ++e) d4[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    return;
+  }
+  const size_t vrow0 = static_cast<size_t>(unit) * Npad;  // this unit's rows in the padded LSE2 / D vectors
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -341,17 +391,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch_desc(&tmDO);
       mbar_expect_tx(&bars[kKVFull], 2 * L::kTile);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(smem + L::kK + c * L::kBox, &tmK, c * 64, kj * 128, bh, &bars[kKVFull]);
-        tma_load_3d(smem + L::kV + c * L::kBox, &tmV, c * 64, kj * 128, bh, &bars[kKVFull]);
+        tma_load_3d(smem + L::kK + c * L::kBox, &tmK, c * 64, su.k0 + kj * 128, su.g, &bars[kKVFull]);
+        tma_load_3d(smem + L::kV + c * L::kBox, &tmV, c * 64, su.k0 + kj * 128, su.g, &bars[kKVFull]);
       }
       int issued = 0;
       for (int it = 0; it < nq; ++it) {
         const int s = it & 1;
-        const int qrow = (q_first + it) * 128;  // first query row of the tile within the head
+        const int qrow = (q_first + it) * 128;  // first query row of the tile within the unit
         if (it >= 2 && !mbar_wait(&bars[kEmpty0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kQFull0 + s], L::kTile + 1024);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, qrow, bh, &bars[kQFull0 + s]);
+          tma_load_3d(smem + L::kQ + s * L::kTile + c * L::kBox, &tmQ, c * 64, su.q0 + qrow, su.g,
+                      &bars[kQFull0 + s]);
         bulk_load_1d(smem + L::kVec + s * 1024, p.lse2 + vrow0 + qrow, 512, &bars[kQFull0 + s]);
         bulk_load_1d(smem + L::kVec + s * 1024 + 512, p.Dvec + vrow0 + qrow, 512, &bars[kQFull0 + s]);
         issued = it + 1;
@@ -359,7 +410,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (it >= 2 && !mbar_wait(&bars[kDOStage0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kDOFull0 + s], L::kTile);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, qrow, bh, &bars[kDOFull0 + s]);
+          tma_load_3d(smem + L::kDO + s * L::kTile + c * L::kBox, &tmDO, c * 64, su.q0 + qrow, su.g,
+                      &bars[kDOFull0 + s]);
       }
       if (*abort_flag) {
         mbar_wait_drain(&bars[kKVFull], 0);
@@ -475,7 +527,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) {
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
-            tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, qrow, bh);  // rows past N skipped
+            // rows past the tensor are skipped; rows of the next packed
+            // sequence receive exact zeros (their P is 0 here)
+            tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, su.q0 + qrow, su.g);
           bulk_commit_group();
           bulk_wait_group_read0();
         }
@@ -494,9 +548,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float sl2 = p.scale_log2;
     const DropConst dk = make_drop_const(p.drop_t);
     const bool hi_t = p.drop_t > 0x8000u;
-    const uint32_t hh = static_cast<uint32_t>(bh % p.H), bb = static_cast<uint32_t>(bh / p.H);
+    const uint32_t hh = static_cast<uint32_t>(su.h), bb = static_cast<uint32_t>(su.b);
     const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
-    const bool key_valid = kj * 128 + r < N;
     const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
     // keep bits of this thread's 64 query columns for the coming query tile;
     // computed one tile ahead, while the warp would otherwise wait for S^T
@@ -509,6 +562,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane);
     };
     if (DROPOUT) keep_bits_tile(q_first);
+    // masking: query i = qi * 128 + c sees this thread's key j = kj * 128 + r
+    // iff i + Nk - Nq >= j, i.e. c >= lo0 - qi * 128; query tiles up to qi_mask
+    // hold such pairs for some key of the tile; a tile past the unit's last
+    // key masks whole rows
+    const int lo0 = CAUSAL ? kj * 128 + r - delta : -(1 << 30);
+    const int qi_mask = CAUSAL ? floor_div(kj * 128 + 126 - delta, 128) : -1;
+    const bool tile_past_keys = kj * 128 + 128 > su.nk;
     bool ok = true;
     for (int it = 0; it < nq; ++it) {
       const int s = it & 1;
@@ -533,10 +593,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         P[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 2]), sl2, -l4.z));
         P[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 3]), sl2, -l4.w));
       }
-      // masked: queries before this key on the diagonal tile (causal), and the
-      // whole row for a key past N (queries past N already get LSE2 = +inf)
-      if ((CAUSAL && qi == kj) || !key_valid) {
-        const int lo = key_valid ? r : 128;  // columns 64 g + c < lo are zeroed
+      // masked: (causal) query columns whose position i + Nk - Nq lies before
+      // this key, and the whole row for a key past the unit's keys; queries
+      // past the unit's rows already get LSE2 = +inf
+      if (qi <= qi_mask || tile_past_keys) {  // the same for the whole warp
+        const int lo = key_valid ? lo0 - qi * 128 : 128;  // query columns c < lo are masked
 #pragma unroll
         for (int c = 0; c < 64; ++c)
           if (64 * g + c < lo) P[c] = 0.f;
@@ -599,7 +660,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint32_t col = (g == 0) ? kColDK : kColDV;
       const float mul = (g == 0) ? p.scale : p.drop_scale;
-      uint16_t* dst = ((g == 0) ? p.dK : p.dV) + (static_cast<size_t>(bh) * N + kj * 128 + r) * D;
+      uint16_t* dst = ((g == 0) ? p.dK : p.dV) + static_cast<size_t>(su.k0 + kj * 128 + r) * p.seq.tok_stride +
+                      static_cast<size_t>(su.g) * p.seq.k_head_stride;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -647,38 +709,37 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.lse2 = a.lse2;
   p.Dvec = a.Dvec;
   p.err = a.err;
-  p.H = a.H;
-  p.N = a.N;
+  p.seq = a.seq;
   p.scale = a.scale;
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
   for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
-  p.BH = a.B * a.H;
+  p.BH = a.seq.B * a.seq.H;
+  const int n_kt = (a.seq.Nk + 127) / 128;
   {
-    // heads per group: about 512 key-tile units per group; the CTAs running
-    // together then stream the same Q / dO tiles and add into the same dQ
-    // rows through L2, heaviest (lowest) key tiles first
-    const int n_t = (a.N + 127) / 128;
-    p.group = (512 + n_t / 2) / n_t;
+    // units per group: about 512 key-tile work units per group; the CTAs
+    // running together then stream the same Q / dO tiles and add into the
+    // same dQ rows through L2, heaviest (lowest) key tiles first
+    p.group = (512 + n_kt / 2) / n_kt;
     if (p.group < 1) p.group = 1;
     if (p.group > p.BH) p.group = p.BH;
   }
-  dim3 grid(a.B * a.H * ((a.N + 127) / 128));
+  dim3 grid(static_cast<unsigned>(p.BH) * n_kt);
   kern<<<grid, kBwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmDO, a.tmDQacc, p);
   return cudaGetLastError();
 }
 
 template <bool F16>
-void launch_preprocess_typed(const BwdArgs& a, long long blocks, long long rows_pad, int Npad, cudaStream_t stream) {
+void launch_preprocess_typed(const BwdArgs& a, long long blocks, int Npad, long long acc_vec4, cudaStream_t stream) {
   const uint16_t* O = static_cast<const uint16_t*>(a.O);
   const uint16_t* dO = static_cast<const uint16_t*>(a.dO);
   if (a.d == 64)
     fa_bwd_preprocess_kernel<64, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                    a.dQacc, rows_pad, a.N, Npad);
+                                                                                    a.dQacc, a.seq, Npad, acc_vec4);
   else
     fa_bwd_preprocess_kernel<128, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                     a.dQacc, rows_pad, a.N, Npad);
+                                                                                     a.dQacc, a.seq, Npad, acc_vec4);
 }
 
 template <bool F16>
@@ -697,14 +758,17 @@ cudaError_t launch_bwd_tiles_typed(const BwdArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
-  const int Npad = (a.N + 127) / 128 * 128;
-  const long long rows_pad = static_cast<long long>(a.B) * a.H * Npad;
+  const int Npad = (a.seq.Nq + 127) / 128 * 128;
+  const long long rows_pad = static_cast<long long>(a.seq.B) * a.seq.H * Npad;
+  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.B) * a.seq.H;
+  const long long acc_vec4 = groups * a.seq.total_q * a.d / 4;
   long long blocks = (rows_pad + 7) / 8;  // one warp per row, 8 warps per block
   if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
   if (a.f16)
-    launch_preprocess_typed<true>(a, blocks, rows_pad, Npad, stream);
+    launch_preprocess_typed<true>(a, blocks, Npad, acc_vec4, stream);
   else
-    launch_preprocess_typed<false>(a, blocks, rows_pad, Npad, stream);
+    launch_preprocess_typed<false>(a, blocks, Npad, acc_vec4, stream);
   return cudaGetLastError();
 }
 
@@ -713,15 +777,17 @@ cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
-  const long long n8 = static_cast<long long>(a.B) * a.H * a.N * a.d / 8;
+  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.B) * a.seq.H;
+  const long long n8 = groups * a.seq.total_q * a.d / 8;
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
   uint16_t* dQ = static_cast<uint16_t*>(a.dQ);
   if (a.f16)
-    fa_bwd_dq_convert_kernel<true><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, n8);
+    fa_bwd_dq_convert_kernel<true><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, a.seq, a.d, n8);
   else
-    fa_bwd_dq_convert_kernel<false><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, n8);
+    fa_bwd_dq_convert_kernel<false><<<static_cast<int>(blocks), 256, 0, stream>>>(a.dQacc, dQ, a.scale, a.seq, a.d,
+                                                                                 n8);
   return cudaGetLastError();
 }
 

@@ -30,7 +30,11 @@
 //    runs at half rate, is the bottleneck of this path); kept P are left
 //    unscaled and 1/(1-p) is folded into the final normalisation.
 //  * a causal CTA processes only key tiles up to its diagonal; the grid puts
-//    the heaviest query blocks first.
+//    the heaviest query blocks first;
+//  * queries and keys may differ in number (Nq != Nk, causal alignment
+//    bottom-right: query i sits at key position i + Nk - Nq) and, with
+//    packed sequence offsets, per sequence.  A row that sees no key gets
+//    O = 0 and LSE = -inf.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -70,7 +74,8 @@ struct FwdSmem {
   static constexpr int kBar = kV + kStages * kTileBytes;
   // barriers: q, kfull[S], vfull[S], kvempty[S], s_ready[2], p_ready[2], o_ready[2], drain
   static constexpr int kNumBars = 1 + 3 * kStages + 7;
-  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot (4 B) + abort flag (4 B)
+  // tmem slot (4 B), abort flag (4 B), the unit's first query row and head coordinate (4 B each)
+  static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;   // + slack for 1024-byte alignment
 };
 
@@ -105,7 +110,7 @@ struct FwdParams {
   uint16_t* O;  // bf16 or fp16 bits
   float* LSE;
   unsigned* err;
-  int H, N;
+  SeqLayout seq;
   float scale_log2;
   uint32_t drop_t;
   float drop_scale;
@@ -159,27 +164,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // 1-D grid over (head group, query block, head): within a group of
-  // p.group heads the heaviest causal blocks come first, and the blocks that
-  // run together share their heads' K and V through L2.
-  const int N = p.N;
-  const int n_qt = (N + kBM - 1) / kBM;  // the last tile may be partial
-  const int n_qb = (n_qt + 1) / 2;
-  // groups of p.group heads; inside a group, all heads' heaviest blocks first
-  const int per_group = p.group * n_qb;
+  // 1-D grid over (head group, query block, unit): within a group of
+  // p.group units the heaviest causal blocks come first, and the blocks that
+  // run together share their units' K and V through L2.
+  const int n_qb_grid = ((p.seq.Nq + kBM - 1) / kBM + 1) / 2;
+  const int per_group = p.group * n_qb_grid;
   const int grp = blockIdx.x / per_group;
-  const int r = blockIdx.x - grp * per_group;
+  const int rr = blockIdx.x - grp * per_group;
   const int gsz = min(p.group, p.BH - grp * p.group);
-  const int qb_lin = r / gsz;
-  const int bh = grp * p.group + (r - qb_lin * gsz);  // b * H + h
-  const int qb = CAUSAL ? (n_qb - 1 - qb_lin) : qb_lin;
+  const int qb_lin = rr / gsz;
+  const int unit = grp * p.group + (rr - qb_lin * gsz);  // b * H + h
+  const SeqUnit su = resolve_unit(p.seq, unit);
+  const int N = su.nq;                   // queries of this unit
+  const int n_qt = (N + kBM - 1) / kBM;  // the last tile may be partial
+  const int qb = CAUSAL ? (n_qb_grid - 1 - qb_lin) : qb_lin;
   const int qt0 = 2 * qb;
+  // a block past this unit's queries (shorter packed sequence) has no work
+  if (qt0 >= n_qt) return;
   const int nq = min(2, n_qt - qt0);
-  // key tiles each query tile visits (causal: up to and including its diagonal)
-  int ntile[2];
-  ntile[0] = CAUSAL ? qt0 + 1 : n_qt;
-  ntile[1] = (nq == 2) ? (CAUSAL ? qt0 + 2 : n_qt) : 0;
-  const int nt_all = ntile[nq - 1];
+  // key tiles each query tile visits: all of them, or (causal) up to the one
+  // holding the last valid row's last visible key i + Nk - Nq; possibly none
+  const int n_kt = (su.nk + kBN - 1) / kBN;
+  const int delta = su.nk - su.nq;
+  // (two scalars rather than an indexed array, which would live in local memory)
+  auto key_tiles = [&](int q) {
+    const int last_row = min(N - 1, (qt0 + q) * kBM + kBM - 1);
+    return CAUSAL ? min(n_kt, max(0, floor_div(last_row + delta, kBN) + 1)) : n_kt;
+  };
+  const int nt0 = key_tiles(0);
+  const int nt1 = (nq == 2) ? key_tiles(1) : 0;
+  const int nt_all = (nq == 2) ? nt1 : nt0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q, 1);
@@ -195,6 +209,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(bar.drain, 1);
     *abort_flag = 0;
+    // the epilogue reads these back instead of keeping them in registers
+    // through the softmax loop
+    reinterpret_cast<int*>(smem + L::kMisc)[2] = su.q0;
+    reinterpret_cast<int*>(smem + L::kMisc)[3] = su.g;
     mbar_fence_init();
   }
   if (warp == kMmaWarp) {
@@ -214,27 +232,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
     if (warp == kLoadWarp) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && nt_all > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      // 3-D coordinates (column, row within the head, head): rows past N read as zeros
+      // 3-D coordinates (column, token row, head coordinate): rows past the
+      // tensor read as zeros, rows of the next packed sequence are masked
       mbar_expect_tx(bar.q, nq * L::kTileBytes);
       for (int q = 0; q < nq; ++q)
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::kQ + q * L::kTileBytes + c * L::kBoxBytes, &tmQ, c * 64, (qt0 + q) * kBM, bh,
-                      bar.q);
+          tma_load_3d(smem + L::kQ + q * L::kTileBytes + c * L::kBoxBytes, &tmQ, c * 64,
+                      su.q0 + (qt0 + q) * kBM, su.g, bar.q);
       int issued = 0;
       for (int t = 0; t < nt_all; ++t) {
         const int s = t % S;
         if (t >= S && !mbar_wait(&bar.kvempty[s], ((t / S) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bar.kfull[s], L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::kK + s * L::kTileBytes + c * L::kBoxBytes, &tmK, c * 64, t * kBN, bh,
+          tma_load_3d(smem + L::kK + s * L::kTileBytes + c * L::kBoxBytes, &tmK, c * 64, su.k0 + t * kBN, su.g,
                       &bar.kfull[s]);
         mbar_expect_tx(&bar.vfull[s], L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem + L::kV + s * L::kTileBytes + c * L::kBoxBytes, &tmV, c * 64, t * kBN, bh,
+          tma_load_3d(smem + L::kV + s * L::kTileBytes + c * L::kBoxBytes, &tmV, c * 64, su.k0 + t * kBN, su.g,
                       &bar.vfull[s]);
         issued = t + 1;
       }
@@ -249,11 +268,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && nt_all > 0) {
       bool ok = mbar_wait(bar.q, 0, abort_flag, p.err) && mbar_wait(&bar.kfull[0], 0, abort_flag, p.err);
       if (ok) {
         tc_fence_after();
         for (int q = 0; q < nq; ++q) {
+          if ((q ? nt1 : nt0) == 0) continue;  // a query tile that sees no key
           issue_qk<D, F16>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k);
           mma_commit(&bar.s_ready[q]);
         }
@@ -264,11 +284,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool next_k_ready = false;
         const int s1 = (t + 1) % S;
         for (int q = 0; q < nq; ++q) {
-          if (t >= ntile[q]) continue;
+          const int ntq = q ? nt1 : nt0;
+          if (t >= ntq) continue;
           if (!mbar_wait(&bar.p_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, F16>(tmem + 256 + q * D, tmem + q * 128, sm_v + s * L::kTileBytes, t > 0);
-          if (t == ntile[q] - 1) {
+          if (t == ntq - 1) {
             mma_commit(&bar.o_ready[q]);
           } else {
             if (!next_k_ready) {
@@ -307,12 +328,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // keep test on the FMA pipe: for a 16-bit draw u, the float 2^23 + u is
       // exact, and sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0
       const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
-      const int h = bh % p.H;
-      const int b = bh / p.H;
+      const int h = su.h;
+      const int b = su.b;
+      // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
+      // last key, and under the causal mask the row's position i + Nk - Nq);
+      // tiles from t_mask on are the first that can hold a masked key for
+      // some row of the tile
+      const int lim0 = CAUSAL ? min(su.nk - 1, i + delta) : su.nk - 1;
+      int t_mask = su.nk / kBN;  // first tile running past the keys
+      if (CAUSAL) t_mask = min(t_mask, max(0, floor_div((qt0 + q) * kBM + delta - (kBN - 1), kBN) + 1));
       float m = -CUDART_INF_F;  // running max of scale*log2(e)*S, possibly stale
       float l = 0.f;            // running sum of exp2(x - m)
       bool ok = true;
-      for (int t = 0; t < ntile[q]; ++t) {
+      const int ntq = q ? nt1 : nt0;
+      for (int t = 0; t < ntq; ++t) {
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -324,11 +353,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float s[kBN];
 #pragma unroll
         for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
-        // masked columns: keys after this row on the diagonal tile (causal) and
-        // keys past N on a partial last tile; both are c > lim for one limit
-        const int jv = N - t * kBN;  // keys of this tile inside the sequence
-        if ((CAUSAL && t == ntile[q] - 1) || jv < kBN) {
-          const int lim = min((CAUSAL && t == ntile[q] - 1) ? r : kBN - 1, jv - 1);
+        // masked columns: keys after this row's position i + Nk - Nq (causal)
+        // and keys past the unit's last key; both are c > lim for one limit
+        if (t >= t_mask) {  // the same for the whole warp
+          const int lim = lim0 - t * kBN;
 #pragma unroll
           for (int c = 0; c < kBN; ++c)
             if (c > lim) s[c] = -CUDART_INF_F;
@@ -365,7 +393,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           m = m_new;
         }
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        const uint64_t negm2 = f2_pack(-m, -m);
+        // a row that has seen no key yet keeps m = -inf: its P is exp2(-inf) = 0
+        const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
+        const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
 #pragma unroll
@@ -412,11 +442,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar.p_ready[q]);
       }
-      if (ok && mbar_wait(&bar.o_ready[q], 0, abort_flag, p.err)) {
+      const bool row_ok = i < N;  // rows of a partial last tile past N are computed but not stored
+      const int q0 = reinterpret_cast<const int*>(smem + L::kMisc)[2];
+      const int gq = reinterpret_cast<const int*>(smem + L::kMisc)[3];
+      uint16_t* orow_g = p.O + static_cast<size_t>(q0 + i) * p.seq.tok_stride +
+                         static_cast<size_t>(gq) * p.seq.q_head_stride;
+      float* lse_g = p.LSE + static_cast<size_t>(gq) * p.seq.total_q + q0 + i;
+      if (ntq == 0) {
+        // the whole tile sees no key: O = 0, LSE = -inf
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow_g);
+#pragma unroll
+          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+          *lse_g = -CUDART_INF_F;
+        }
+      } else if (ok && mbar_wait(&bar.o_ready[q], 0, abort_flag, p.err)) {
         // ---------------------------------------------------------- epilogue
         tc_fence_after();
-        const float inv = p.drop_scale / l;
-        uint16_t* orow_g = p.O + (static_cast<size_t>(bh) * N + i) * D;
+        // l = 0: the row saw no key (O = 0, LSE = -inf)
+        const float inv = (l > 0.f) ? p.drop_scale / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -427,14 +471,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             packed[e] = pack2<F16>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          if (i < N) {  // rows of a partial last tile past N are computed but not stored
+          if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
           }
         }
-        if (i < N) p.LSE[static_cast<size_t>(bh) * N + i] = (m + lg2_approx(l)) * 0.69314718055994531f;
+        if (row_ok) *lse_g = (l > 0.f) ? (m + lg2_approx(l)) * 0.69314718055994531f : -CUDART_INF_F;
       }
     }
     cta_teardown(tmem, false);
@@ -456,24 +500,22 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   p.O = static_cast<uint16_t*>(a.O);
   p.LSE = a.LSE;
   p.err = a.err;
-  p.H = a.H;
-  p.N = a.N;
+  p.seq = a.seq;
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
   for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
-  p.BH = a.B * a.H;
+  p.BH = a.seq.B * a.seq.H;
+  const int n_qb = ((a.seq.Nq + kBM - 1) / kBM + 1) / 2;
   {
-    // heads per group: about 256 work units (~2 waves on 148 SMs) per group,
-    // so the blocks running together share their heads' K and V in L2 while
+    // units per group: about 256 work units (~2 waves on 148 SMs) per group,
+    // so the blocks running together share their units' K and V in L2 while
     // the heaviest causal blocks of the group still start first
-    const int n_qb = ((a.N + kBM - 1) / kBM + 1) / 2;
     p.group = (256 + n_qb / 2) / n_qb;
     if (p.group < 1) p.group = 1;
     if (p.group > p.BH) p.group = p.BH;
   }
-  const int n_qt = (a.N + kBM - 1) / kBM;
-  dim3 grid(a.B * a.H * ((n_qt + 1) / 2));
+  dim3 grid(static_cast<unsigned>(p.BH) * n_qb);
   kern<<<grid, kFwdThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
   return cudaGetLastError();
 }

@@ -8,13 +8,74 @@
 
 namespace fa {
 
+// Where the rows of one (sequence, head) unit live.  Units are numbered
+// b * H + h.
+//  * Fixed length (cu_q == nullptr): every unit has Nq queries and Nk keys;
+//    tensors are [B, H, N, d], so a unit's tokens are contiguous rows and the
+//    head coordinate of unit u is u itself.
+//  * Packed variable length: cu_q / cu_k are device int32 offsets [B + 1]
+//    (sequence b owns query rows cu_q[b] .. cu_q[b+1] - 1); tensors are
+//    [total, H, d] and the head coordinate is h.  Nq / Nk are then the
+//    largest lengths (they size the grid and the padded per-row vectors).
+// Row t of head coordinate g of an LSE-like [G, total] array is g * total + t.
+struct SeqLayout {
+  const int* cu_q;
+  const int* cu_k;
+  int B, H;
+  int Nq, Nk;
+  int total_q, total_k;         // rows per head coordinate (fixed: Nq, Nk)
+  long long tok_stride;         // elements between consecutive tokens of one head
+  long long q_head_stride;      // elements between head coordinates of Q, O, dO, dQ
+  long long k_head_stride;      // elements between head coordinates of K, V, dK, dV
+};
+
+struct SeqUnit {
+  int b, h;
+  int q0, nq;  // first query row (within the head coordinate) and query count
+  int k0, nk;
+  int g;       // head coordinate
+};
+
+#ifdef __CUDACC__
+// Offsets and lengths of one unit.  Packed offsets are clamped into the
+// tensors and to the maximum lengths, so inconsistent offsets give wrong
+// rows but never an access outside the tensors or the workspace.
+__device__ __forceinline__ SeqUnit resolve_unit(const SeqLayout& L, int unit) {
+  SeqUnit u;
+  u.b = unit / L.H;
+  u.h = unit - u.b * L.H;
+  if (L.cu_q) {
+    const int qa = min(max(L.cu_q[u.b], 0), L.total_q);
+    const int qb = min(max(L.cu_q[u.b + 1], qa), L.total_q);
+    const int ka = min(max(L.cu_k[u.b], 0), L.total_k);
+    const int kb = min(max(L.cu_k[u.b + 1], ka), L.total_k);
+    u.q0 = qa;
+    u.nq = min(qb - qa, L.Nq);
+    u.k0 = ka;
+    u.nk = min(kb - ka, L.Nk);
+    u.g = u.h;
+  } else {
+    u.q0 = 0;
+    u.nq = L.Nq;
+    u.k0 = 0;
+    u.nk = L.Nk;
+    u.g = unit;
+  }
+  return u;
+}
+
+// floor(a / b) for b > 0 and any sign of a
+__device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
+#endif
+
 struct FwdArgs {
-  CUtensorMap tmQ, tmK, tmV;  // 3-D maps over [B*H, N, d] 16-bit, 64 x 128 x 1 boxes, 128B swizzle
-  void* O;                    // [B, H, N, d], same type as Q
+  CUtensorMap tmQ, tmK, tmV;  // 3-D maps (d, token, head coordinate), 64 x 128 x 1 boxes, 128B swizzle
+  void* O;                    // same layout and type as Q
   int f16;                    // element type of Q, K, V, O: 0 bf16, 1 fp16
-  float* LSE;                 // fp32 [B, H, N]
+  float* LSE;                 // fp32 [G, total_q]
   unsigned* err;              // device error word
-  int B, H, N, d;
+  SeqLayout seq;
+  int d;
   int causal;
   float scale_log2;   // scale * log2(e)
   uint32_t drop_t;    // keep <=> u16 >= drop_t (0: no dropout)
@@ -25,7 +86,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tmQ, tmK, tmV, tmDO;  // same layout as the forward maps
-  CUtensorMap tmDQacc;               // fp32 [B*H, N, d], 32-column x 128-row boxes, 128B swizzle
+  CUtensorMap tmDQacc;               // fp32 [G, total_q, d], 32-column x 128-row boxes, 128B swizzle
   int f16;  // element type of Q, K, V, O, dO, dQ, dK, dV: 0 bf16, 1 fp16
   const void* O;
   const void* dO;
@@ -33,11 +94,12 @@ struct BwdArgs {
   void* dQ;
   void* dK;
   void* dV;
-  float* dQacc;  // fp32 [B, H, N, d] workspace
-  float* Dvec;   // fp32 [B, H, Npad] workspace: rowsum(dO * O); 0 past N
-  float* lse2;   // fp32 [B, H, Npad] workspace: LSE * log2(e); +inf past N
+  float* dQacc;  // fp32 [G, total_q, d] workspace
+  float* Dvec;   // fp32 [B*H, Npad] workspace: rowsum(dO * O); 0 past a unit's queries
+  float* lse2;   // fp32 [B*H, Npad] workspace: LSE * log2(e); +inf past a unit's queries and for rows that see no key
   unsigned* err;
-  int B, H, N, d;
+  SeqLayout seq;
+  int d;
   int causal;
   float scale;
   float scale_log2;

@@ -30,7 +30,12 @@
  *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
  *    aligned.  The library allocates nothing and keeps no per-call state.
  *  - Supported: d in {64, 128}; any N >= 1 (a partial last 128-row tile is
- *    handled inside the kernels); B*H*N < 2^31.
+ *    handled inside the kernels); B*H*N < 2^31.  Queries and keys may differ
+ *    in number (``_qk`` and ``_varlen`` entry points).
+ *  - Causal mask with Nq queries and Nk keys: query i sits at key position
+ *    i + Nk - Nq (bottom-right alignment; top-left when Nq = Nk) and sees the
+ *    keys j <= i + Nk - Nq.  A query row that sees no key (Nk < Nq) gets
+ *    O = 0 and LSE = -inf, and contributes nothing to the gradients.
  *  - ``stream`` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call only enqueues work on it and returns; results are
  *    ready when the stream reaches that point.
@@ -102,6 +107,40 @@ fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float*
                     float p_drop, uint64_t seed, fa_dtype dtype, void* stream);
 
 /*
+ * Forward pass with Nq queries and Nk keys per (b, h): Q, O are [B, H, Nq, d],
+ * K, V are [B, H, Nk, d], LSE is fp32 [B, H, Nq], all 16-bit tensors of
+ * ``dtype``.  Causal alignment as stated above.  Otherwise as fa_fwd_ex.
+ */
+fa_status fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                    int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                    float p_drop, uint64_t seed, fa_dtype dtype, void* stream);
+
+/*
+ * Forward pass over a batch of B sequences of different lengths, packed
+ * without padding ("variable length").
+ *   Q, O     : [total_q, H, d] of ``dtype``; token rows of all sequences back to back
+ *   K, V     : [total_k, H, d]
+ *   LSE      : out, fp32 [H, total_q]
+ *   cu_seqlens_q, cu_seqlens_k : DEVICE int32 [B + 1], 4-byte aligned:
+ *              sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *              and key rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1; offsets start
+ *              at 0, never decrease and end at total_q / total_k
+ *   max_seqlen_q, max_seqlen_k : the largest sequence lengths (they size the
+ *              launch); 1 <= max_seqlen <= total
+ * Each sequence is an independent problem with Nq = its query count and
+ * Nk = its key count (causal alignment as above).  Dropout draws use b = the
+ * sequence index and i, j = positions within the sequence.  The offsets live
+ * on the device, so the library cannot check them: offsets that break the
+ * rules above give wrong results for the rows concerned (every access is still
+ * clamped into the tensors and the workspace).  H*total < 2^31.
+ */
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                        int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int d, int causal, float scale, float p_drop, uint64_t seed,
+                        fa_dtype dtype, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes: an fp32 dQ
  * accumulator [B, H, N, d], the fp32 row statistic D and the fp32 copy of
  * LSE in log2 units, both [B, H, Npad] with Npad = N rounded up to a multiple
@@ -146,6 +185,36 @@ fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, 
                     int B, int H, int N, int d, int causal, float scale,
                     float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass of fa_fwd_qk: Q, O, dO, dQ are [B, H, Nq, d], K, V, dK, dV
+ * are [B, H, Nk, d]; workspace of at least fa_bwd_workspace_size(B, H, Nq, d)
+ * bytes.  Otherwise as fa_bwd_ex.
+ */
+fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV,
+                    int B, int H, int Nq, int Nk, int d, int causal, float scale,
+                    float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace for fa_bwd_varlen: an fp32 dQ accumulator [H, total_q, d] and the
+ * fp32 D and LSE*log2(e) vectors [B, H, pad128(max_seqlen_q)], each part
+ * rounded up to 256 bytes.  Returns 0 for non-positive sizes.
+ */
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d);
+
+/*
+ * Backward pass of fa_fwd_varlen: same packed layouts (dQ like Q, dK and dV
+ * like K), same offsets and scalars; workspace of at least
+ * fa_bwd_varlen_workspace_size() bytes, 256-byte aligned.
+ */
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                        const float* LSE, void* dQ, void* dK, void* dV,
+                        const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                        int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                        int d, int causal, float scale, float p_drop, uint64_t seed,
+                        fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The three stages fa_bwd runs, in order, for callers that schedule or time

@@ -117,6 +117,36 @@ def test_ex_entry_points_validate_like_the_plain_ones(lib, dtype):
     assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 32, 1, 0.125, 0.0, 0, dtype, A, ws_ok, None) == 2
 
 
+def _varlen_fwd(lib, cu_q=A, cu_k=A, B=1, H=1, tq=64, tk=64, mq=64, mk=64, d=64, scale=0.125, p=0.0, dtype=0):
+    return lib.fa_fwd_varlen(A, A, A, A, A, cu_q, cu_k, B, H, tq, tk, mq, mk, d, 1, scale, p, 0, dtype, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(cu_q=0), 1), (dict(cu_k=0), 1), (dict(cu_q=A + 2), 1), (dict(B=0), 1), (dict(tq=0), 1),
+    (dict(mq=65), 1), (dict(mk=0), 1), (dict(p=1.0), 1), (dict(dtype=3), 1), (dict(d=96), 2),
+    (dict(H=1 << 12, tq=1 << 19, tk=1 << 19, mq=1 << 10, mk=1 << 10), 2),
+])
+def test_varlen_rejects_bad_arguments(lib, kw, want):
+    assert _varlen_fwd(lib, **kw) == want
+
+
+def test_varlen_workspace_size(lib):
+    # accumulator H * total_q * d fp32, then two [B, H, pad128(max_q)] fp32 vectors
+    assert lib.fa_bwd_varlen_workspace_size(3, 2, 500, 300, 64) == 2 * 500 * 64 * 4 + 2 * (3 * 2 * 384 * 4)
+    assert lib.fa_bwd_varlen_workspace_size(0, 2, 500, 300, 64) == 0
+    ws = lib.fa_bwd_varlen_workspace_size(1, 1, 64, 64, 64)
+    assert lib.fa_bwd_varlen(A, A, A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 64, 64, 1, 0.125, 0.0, 0, 0, A,
+                             ws - 4, None) == 1
+
+
+def test_qk_entry_points_validate(lib):
+    assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 0, 64, 1, 0.125, 0.0, 0, 0, None) == 1
+    assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 256, 96, 1, 0.125, 0.0, 0, 0, None) == 2
+    ws = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert lib.fa_bwd_qk(A, A, A, A, A, A, A, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, A, ws - 4, None) == 1
+    assert lib.fa_bwd_qk(A, A, A, A, A, A, 0, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, A, ws, None) == 1
+
+
 def test_stage_entry_points_reject_bad_arguments(lib):
     ws_ok = lib.fa_bwd_workspace_size(1, 1, 128, 64)
     assert lib.fa_bwd_prepare(0, A, A, 1, 1, 128, 64, A, ws_ok, None) == 1
