@@ -48,14 +48,16 @@ def load_library(path=None):
     lib.fa_bwd_ex.restype = i
     lib.fa_fwd_qk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, u64, i, vp]
     lib.fa_fwd_qk.restype = i
-    lib.fa_bwd_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, u64, i, vp, sz, vp]
+    lib.fa_bwd_qk_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_qk_workspace_size.restype = sz
+    lib.fa_bwd_qk.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, u64, i, i, vp, sz, vp]
     lib.fa_bwd_qk.restype = i
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, u64, i, vp]
     lib.fa_fwd_varlen.restype = i
-    lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.fa_bwd_varlen_workspace_size.restype = sz
     lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, f, u64, i,
-                                  vp, sz, vp]
+                                  i, vp, sz, vp]
     lib.fa_bwd_varlen.restype = i
     lib.fa_bwd_prepare.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_prepare.restype = i
@@ -133,9 +135,10 @@ def fa_bwd_workspace_size(B, H, N, d):
 
 
 def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspace=None, dq=None, dk=None,
-           dv=None):
+           dv=None, deterministic=False):
     """(dQ, dK, dV) of sum(dO * O) by recomputation; same arguments as the matching fa_fwd call
-    (square bf16 tensors go to fa_bwd, square fp16 ones to fa_bwd_ex, Nq != Nk to fa_bwd_qk)."""
+    (square bf16 tensors go to fa_bwd, square fp16 ones to fa_bwd_ex, Nq != Nk or
+    ``deterministic`` -- a fixed order of the dQ additions -- to fa_bwd_qk)."""
     lib = load_library()
     for name, t in (("q", q), ("o", o), ("do", do)):
         _check_bhnd(name, t, q.shape, q.dtype)
@@ -148,7 +151,8 @@ def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspac
     scale = d ** -0.5 if scale is None else scale
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, Nq] tensor")
-    ws_bytes = fa_bwd_workspace_size(B, H, Nq, d)
+    det = int(bool(deterministic))
+    ws_bytes = int(lib.fa_bwd_qk_workspace_size(B, H, Nq, d, det))
     if workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
@@ -161,8 +165,8 @@ def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspac
             dk.data_ptr(), dv.data_ptr())
     tail = (d, int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1))
     ws = (workspace.data_ptr(), workspace.numel(), _stream(q))
-    if Nq != Nk:
-        _raise(lib.fa_bwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], *ws), "fa_bwd_qk")
+    if Nq != Nk or det:
+        _raise(lib.fa_bwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], det, *ws), "fa_bwd_qk")
     elif q.dtype == torch.bfloat16:
         _raise(lib.fa_bwd(*ptrs, B, H, Nq, *tail, *ws), "fa_bwd")
     else:
@@ -212,8 +216,9 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_
 
 
 def fa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, scale=None,
-                  p_drop=0.0, seed=0, workspace=None, dq=None, dk=None, dv=None):
-    """(dQ, dK, dV) of the matching fa_fwd_varlen call, in the same packed layouts."""
+                  p_drop=0.0, seed=0, workspace=None, dq=None, dk=None, dv=None, deterministic=False):
+    """(dQ, dK, dV) of the matching fa_fwd_varlen call, in the same packed layouts
+    (``deterministic``: fixed order of the dQ additions)."""
     lib = load_library()
     _check_packed("q", q)
     total_q, H, d = q.shape
@@ -228,7 +233,8 @@ def fa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
     if lse.dtype != torch.float32 or tuple(lse.shape) != (H, total_q) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [H, total_q] tensor")
     scale = d ** -0.5 if scale is None else scale
-    ws_bytes = int(lib.fa_bwd_varlen_workspace_size(B, H, total_q, int(max_seqlen_q), d))
+    det = int(bool(deterministic))
+    ws_bytes = int(lib.fa_bwd_varlen_workspace_size(B, H, total_q, int(max_seqlen_q), d, det))
     if workspace is None:
         workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
@@ -238,7 +244,7 @@ def fa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(),
                              cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
                              int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1),
-                             FA_DTYPE[q.dtype], workspace.data_ptr(), workspace.numel(), _stream(q)),
+                             FA_DTYPE[q.dtype], det, workspace.data_ptr(), workspace.numel(), _stream(q)),
            "fa_bwd_varlen")
     return dq, dk, dv
 

@@ -96,6 +96,7 @@ struct Problem {
   float p_drop;
   uint64_t seed;
   bool f16;
+  bool deterministic;  // backward: fixed order of the dQ additions
   long long groups() const { return seq.cu_q ? seq.H : static_cast<long long>(seq.B) * seq.H; }
 };
 
@@ -163,11 +164,13 @@ fa_status packed_problem(Problem* pb, const int* cu_q, const int* cu_k, int B, i
 }
 
 // Workspace: fp32 dQ accumulator [G, total_q, d], then the fp32 D and
-// LSE * log2(e) vectors [B * H, pad128(Nq)], each part rounded to 256 bytes.
+// LSE * log2(e) vectors [B * H, pad128(Nq)], then (deterministic mode only)
+// one uint32 counter per (unit, query tile), each part rounded to 256 bytes.
 size_t workspace_bytes(const Problem& pb) {
   const size_t acc = static_cast<size_t>(pb.groups()) * pb.seq.total_q * pb.d * sizeof(float);
   const size_t vec = static_cast<size_t>(pb.seq.B) * pb.seq.H * pad128(pb.seq.Nq) * sizeof(float);
-  return round_up(acc, 256) + 2 * round_up(vec, 256);
+  const size_t order = pb.deterministic ? static_cast<size_t>(pb.seq.B) * pb.seq.H * (pad128(pb.seq.Nq) / 128) * 4 : 0;
+  return round_up(acc, 256) + 2 * round_up(vec, 256) + round_up(order, 256);
 }
 
 bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base) {
@@ -232,6 +235,7 @@ void bwd_args(const Problem& pb, fa::BwdArgs* a, void* workspace) {
   a->dQacc = reinterpret_cast<float*>(ws);
   a->Dvec = reinterpret_cast<float*>(ws + acc);
   a->lse2 = reinterpret_cast<float*>(ws + acc + vec);
+  a->dq_order = pb.deterministic ? reinterpret_cast<unsigned*>(ws + acc + 2 * vec) : nullptr;
 }
 
 fa_status prepare_run(const Problem& pb, const void* O, const void* dO, const float* LSE, void* workspace,
@@ -364,7 +368,20 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return workspace_bytes(pb);
 }
 
-size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d) {
+size_t fa_bwd_qk_workspace_size(int B, int H, int Nq, int d, int deterministic) {
+  Problem pb;
+  if (B <= 0 || H <= 0 || Nq <= 0 || d <= 0) return 0;
+  memset(&pb, 0, sizeof(pb));
+  pb.seq.B = B;
+  pb.seq.H = H;
+  pb.seq.Nq = Nq;
+  pb.seq.total_q = Nq;
+  pb.d = d;
+  pb.deterministic = deterministic != 0;
+  return workspace_bytes(pb);
+}
+
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d, int deterministic) {
   Problem pb;
   if (B <= 0 || H <= 0 || total_q <= 0 || max_seqlen_q <= 0 || d <= 0) return 0;
   memset(&pb, 0, sizeof(pb));
@@ -374,6 +391,7 @@ size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q,
   pb.seq.Nq = max_seqlen_q;
   pb.seq.total_q = total_q;
   pb.d = d;
+  pb.deterministic = deterministic != 0;
   return workspace_bytes(pb);
 }
 
@@ -418,24 +436,28 @@ fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, 
 
 fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                     void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d, int causal, float scale,
-                    float p_drop, uint64_t seed, fa_dtype dtype, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+                    float p_drop, uint64_t seed, fa_dtype dtype, int deterministic, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
   Problem pb;
   fa_status st = fixed_problem(&pb, B, H, Nq, Nk, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
-  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  pb.deterministic = deterministic != 0;
+  return bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                         void* dQ, void* dK, void* dV, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                         int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
-                        int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
-                        size_t workspace_bytes, void* stream) {
+                        int causal, float scale, float p_drop, uint64_t seed, fa_dtype dtype, int deterministic,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
   Problem pb;
   fa_status st = packed_problem(&pb, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q, max_seqlen_k,
                                 d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
-  return st != FA_OK ? st : bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  pb.deterministic = deterministic != 0;
+  return bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------ utilities

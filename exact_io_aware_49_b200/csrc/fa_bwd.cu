@@ -27,6 +27,12 @@
 //        dQ_i is read out of TMEM by a dedicated warpgroup, staged through the
 //        tile's dO buffer (idle by then) and added to the fp32 accumulator
 //        with TMA reduce-add.
+//      Deterministic mode fixes the order of those fp32 additions: the key
+//      tiles that contribute to a query tile are always 0 .. K, and key tile
+//      kj adds only after a per-(unit, query tile) counter in the workspace
+//      reaches kj, then increments it.  Query tiles are then visited in
+//      descending order, so every key tile meets a given query tile at the
+//      same iteration and each waits only for the previous one's add.
 //      Warp roles: warpgroups 0/1 do the elementwise work for query columns
 //      0-63 / 64-127 (one thread per key row, the TMEM lane); warp 8 issues
 //      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
@@ -59,7 +65,8 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
                                                                 float* __restrict__ Dvec,
                                                                 float* __restrict__ lse2,
                                                                 float* __restrict__ dQacc, const SeqLayout seq,
-                                                                int Npad, long long acc_vec4) {
+                                                                int Npad, long long acc_vec4,
+                                                                unsigned* __restrict__ dq_order, int n_order) {
   const int lane = threadIdx.x & 31;
   const int rows_pad = seq.B * seq.H * Npad;  // < 2^31, checked on the host
   const int warps = gridDim.x * (blockDim.x >> 5);
@@ -102,6 +109,9 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < acc_vec4;
        idx += static_cast<long long>(gridDim.x) * blockDim.x)
     zq[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (dq_order)
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n_order; idx += gridDim.x * blockDim.x)
+      dq_order[idx] = 0u;
 }
 
 // ============================================================ dQ convert
@@ -188,6 +198,7 @@ struct BwdParams {
   float* dQacc;
   const float* lse2;
   const float* Dvec;
+  unsigned* dq_order;  // deterministic mode: per (unit, query tile) count of dQ adds done; else nullptr
   unsigned* err;
   SeqLayout seq;
   float scale;
@@ -360,6 +371,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     return;
   }
   const size_t vrow0 = static_cast<size_t>(unit) * Npad;  // this unit's rows in the padded LSE2 / D vectors
+  // query tile of iteration it: ascending from q_first, or descending from the
+  // last tile in deterministic mode
+  const bool det = p.dq_order != nullptr;
+  auto qi_of = [&](int it) { return det ? n_qt - 1 - it : q_first + it; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -397,7 +412,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int issued = 0;
       for (int it = 0; it < nq; ++it) {
         const int s = it & 1;
-        const int qrow = (q_first + it) * 128;  // first query row of the tile within the unit
+        const int qrow = qi_of(it) * 128;  // first query row of the tile within the unit
         if (it >= 2 && !mbar_wait(&bars[kEmpty0 + s], ((it >> 1) - 1) & 1, abort_flag, p.err)) break;
         mbar_expect_tx(&bars[kQFull0 + s], L::kTile + 1024);
         for (int c = 0; c < D / 64; ++c)
@@ -494,7 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!*go) break;
       tc_fence_after();
       const int s = it & 1;
-      const int qrow = (q_first + it) * 128;
+      const int qrow = qi_of(it) * 128;
       uint8_t* stage = smem + L::kDO + s * L::kTile;
       const uint32_t st_row = smem_u32(stage) + c * 128;
       uint32_t v[kCols];
@@ -525,13 +540,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         asm volatile("bar.sync 2, 128;" ::: "memory");
         if (leader) {
+          // deterministic: the key tiles before this one have added their part
+          unsigned* order = det ? p.dq_order + static_cast<size_t>(unit) * (Npad / 128) + qrow / 128 : nullptr;
+          if (det && r == 0) {
+            counter_wait_eq(order, static_cast<unsigned>(kj), abort_flag, p.err);
+            fence_proxy_async_global();
+          }
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
             // rows past the tensor are skipped; rows of the next packed
             // sequence receive exact zeros (their P is 0 here)
             tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, su.q0 + qrow, su.g);
           bulk_commit_group();
-          bulk_wait_group_read0();
+          if (det && r == 1) {
+            // both halves are in the accumulator before the next key tile may add
+            bulk_wait_group0();
+            fence_proxy_async_global();
+            counter_release_add(order, 1u);
+          } else {
+            bulk_wait_group_read0();
+          }
         }
       }
       if (leader) mbar_arrive(&bars[kDOStage0 + s]);  // the dO buffer may be refilled
@@ -561,7 +589,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         zb[half] = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane)
                         : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane);
     };
-    if (DROPOUT) keep_bits_tile(q_first);
+    if (DROPOUT) keep_bits_tile(qi_of(0));
     // masking: query i = qi * 128 + c sees this thread's key j = kj * 128 + r
     // iff i + Nk - Nq >= j, i.e. c >= lo0 - qi * 128; query tiles up to qi_mask
     // hold such pairs for some key of the tile; a tile past the unit's last
@@ -572,7 +600,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int it = 0; it < nq; ++it) {
       const int s = it & 1;
-      const int qi = q_first + it;
+      const int qi = qi_of(it);
       if (!mbar_wait(&bars[kQFull0 + s], (it >> 1) & 1, abort_flag, p.err) ||
           !mbar_wait(&bars[kSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
       tc_fence_after();
@@ -653,7 +681,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kDSReady]);
-      if (DROPOUT && it + 1 < nq) keep_bits_tile(qi + 1);
+      if (DROPOUT && it + 1 < nq) keep_bits_tile(qi_of(it + 1));
     }
     if (ok && mbar_wait(&bars[kDKDVReady], 0, abort_flag, p.err)) {
       // -------------------------------------------------------------- dK / dV epilogue
@@ -706,6 +734,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.dK = static_cast<uint16_t*>(a.dK);
   p.dV = static_cast<uint16_t*>(a.dV);
   p.dQacc = a.dQacc;
+  p.dq_order = a.dq_order;
   p.lse2 = a.lse2;
   p.Dvec = a.Dvec;
   p.err = a.err;
@@ -732,14 +761,15 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
 
 template <bool F16>
 void launch_preprocess_typed(const BwdArgs& a, long long blocks, int Npad, long long acc_vec4, cudaStream_t stream) {
+  const int n_order = a.dq_order ? a.seq.B * a.seq.H * (Npad / 128) : 0;
   const uint16_t* O = static_cast<const uint16_t*>(a.O);
   const uint16_t* dO = static_cast<const uint16_t*>(a.dO);
   if (a.d == 64)
-    fa_bwd_preprocess_kernel<64, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                    a.dQacc, a.seq, Npad, acc_vec4);
+    fa_bwd_preprocess_kernel<64, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, Npad, acc_vec4, a.dq_order, n_order);
   else
-    fa_bwd_preprocess_kernel<128, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(O, dO, a.LSE, a.Dvec, a.lse2,
-                                                                                     a.dQacc, a.seq, Npad, acc_vec4);
+    fa_bwd_preprocess_kernel<128, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, Npad, acc_vec4, a.dq_order, n_order);
 }
 
 template <bool F16>

@@ -97,6 +97,7 @@ struct BwdArgs {
   float* dQacc;  // fp32 [G, total_q, d] workspace
   float* Dvec;   // fp32 [B*H, Npad] workspace: rowsum(dO * O); 0 past a unit's queries
   float* lse2;   // fp32 [B*H, Npad] workspace: LSE * log2(e); +inf past a unit's queries and for rows that see no key
+  unsigned* dq_order;  // deterministic mode: uint32 [B*H, Npad/128] workspace counters, else nullptr
   unsigned* err;
   SeqLayout seq;
   int d;

@@ -103,6 +103,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits (acquire, GPU scope) until the global counter equals ``want``; bounded
+// like mbar_wait: on timeout it sets the abort flag and the device error word
+// and returns false.
+__device__ __forceinline__ bool counter_wait_eq(const unsigned* ctr, unsigned want, volatile int* abort_flag,
+                                                unsigned* err, uint64_t limit_ns = kWaitLimitNs) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v == want) return true;
+    if ((it & 15u) == 15u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        if (err) atomicOr(err, kErrWaitTimeout);
+        return false;
+      }
+    }
+    __nanosleep(32);
+  }
+}
+
+// Adds ``v`` to a global counter with release semantics at GPU scope.
+__device__ __forceinline__ void counter_release_add(unsigned* ctr, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(v) : "memory");
+}
+
+// Orders this thread's global accesses through the async proxy (bulk tensor
+// copies and reductions) with its generic-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Wait used only while draining after an abort: bounded, never sets flags.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);

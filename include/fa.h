@@ -187,22 +187,46 @@ fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, 
                     size_t workspace_bytes, void* stream);
 
 /*
+ * Deterministic mode (the ``deterministic`` argument of fa_bwd_qk and
+ * fa_bwd_varlen; the pages ask only for exact results, this is an option of
+ * this library).  dQ is a sum over key tiles that many thread blocks add into
+ * an fp32 accumulator; by default the order of those additions depends on
+ * scheduling, so dQ may differ in its last bits from run to run (O, LSE, dK
+ * and dV never do).  With deterministic != 0 the additions into each query
+ * tile happen in increasing key-tile order, enforced with one counter per
+ * (b, h, query tile) in the workspace, so repeated calls on the same inputs
+ * give bitwise-identical dQ.  It needs the slightly larger workspace the
+ * ``_workspace_size`` functions return for deterministic != 0 and may run
+ * somewhat slower.
+ */
+
+/*
+ * Workspace for fa_bwd_qk: fa_bwd_workspace_size(B, H, Nq, d) bytes, plus
+ * (deterministic != 0) one uint32 counter per (b, h, 128-row query tile)
+ * rounded up to 256 bytes.  Returns 0 for non-positive sizes.
+ */
+size_t fa_bwd_qk_workspace_size(int B, int H, int Nq, int d, int deterministic);
+
+/*
  * Backward pass of fa_fwd_qk: Q, O, dO, dQ are [B, H, Nq, d], K, V, dK, dV
- * are [B, H, Nk, d]; workspace of at least fa_bwd_workspace_size(B, H, Nq, d)
- * bytes.  Otherwise as fa_bwd_ex.
+ * are [B, H, Nk, d]; workspace of at least
+ * fa_bwd_qk_workspace_size(B, H, Nq, d, deterministic) bytes.  Otherwise as
+ * fa_bwd_ex.
  */
 fa_status fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                     const float* LSE, void* dQ, void* dK, void* dV,
                     int B, int H, int Nq, int Nk, int d, int causal, float scale,
-                    float p_drop, uint64_t seed, fa_dtype dtype, void* workspace,
-                    size_t workspace_bytes, void* stream);
+                    float p_drop, uint64_t seed, fa_dtype dtype, int deterministic,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Workspace for fa_bwd_varlen: an fp32 dQ accumulator [H, total_q, d] and the
- * fp32 D and LSE*log2(e) vectors [B, H, pad128(max_seqlen_q)], each part
- * rounded up to 256 bytes.  Returns 0 for non-positive sizes.
+ * Workspace for fa_bwd_varlen: an fp32 dQ accumulator [H, total_q, d], the
+ * fp32 D and LSE*log2(e) vectors [B, H, pad128(max_seqlen_q)] and (when
+ * deterministic != 0) the uint32 counters [B, H, pad128(max_seqlen_q)/128],
+ * each part rounded up to 256 bytes.  Returns 0 for non-positive sizes.
  */
-size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d);
+size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d,
+                                    int deterministic);
 
 /*
  * Backward pass of fa_fwd_varlen: same packed layouts (dQ like Q, dK and dV
@@ -214,7 +238,8 @@ fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void*
                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                         int B, int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
                         int d, int causal, float scale, float p_drop, uint64_t seed,
-                        fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+                        fa_dtype dtype, int deterministic, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /*
  * The three stages fa_bwd runs, in order, for callers that schedule or time

@@ -132,19 +132,28 @@ def test_varlen_rejects_bad_arguments(lib, kw, want):
 
 def test_varlen_workspace_size(lib):
     # accumulator H * total_q * d fp32, then two [B, H, pad128(max_q)] fp32 vectors
-    assert lib.fa_bwd_varlen_workspace_size(3, 2, 500, 300, 64) == 2 * 500 * 64 * 4 + 2 * (3 * 2 * 384 * 4)
-    assert lib.fa_bwd_varlen_workspace_size(0, 2, 500, 300, 64) == 0
-    ws = lib.fa_bwd_varlen_workspace_size(1, 1, 64, 64, 64)
-    assert lib.fa_bwd_varlen(A, A, A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 64, 64, 1, 0.125, 0.0, 0, 0, A,
+    assert lib.fa_bwd_varlen_workspace_size(3, 2, 500, 300, 64, 0) == 2 * 500 * 64 * 4 + 2 * (3 * 2 * 384 * 4)
+    # deterministic: plus one uint32 counter per (b, h, query tile), rounded to 256 bytes
+    assert lib.fa_bwd_varlen_workspace_size(3, 2, 500, 300, 64, 1) == \
+        2 * 500 * 64 * 4 + 2 * (3 * 2 * 384 * 4) + 256
+    assert lib.fa_bwd_varlen_workspace_size(0, 2, 500, 300, 64, 0) == 0
+    ws = lib.fa_bwd_varlen_workspace_size(1, 1, 64, 64, 64, 0)
+    assert lib.fa_bwd_varlen(A, A, A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 64, 64, 1, 0.125, 0.0, 0, 0, 0, A,
                              ws - 4, None) == 1
+    # a deterministic call needs the larger workspace
+    assert lib.fa_bwd_varlen(A, A, A, A, A, A, A, A, A, A, A, 1, 1, 64, 64, 64, 64, 64, 1, 0.125, 0.0, 0, 0, 1, A,
+                             ws, None) == 1
 
 
 def test_qk_entry_points_validate(lib):
     assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 0, 64, 1, 0.125, 0.0, 0, 0, None) == 1
     assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 256, 96, 1, 0.125, 0.0, 0, 0, None) == 2
-    ws = lib.fa_bwd_workspace_size(1, 1, 128, 64)
-    assert lib.fa_bwd_qk(A, A, A, A, A, A, A, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, A, ws - 4, None) == 1
-    assert lib.fa_bwd_qk(A, A, A, A, A, A, 0, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, A, ws, None) == 1
+    ws = lib.fa_bwd_qk_workspace_size(1, 1, 128, 64, 0)
+    assert ws == lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert lib.fa_bwd_qk_workspace_size(2, 3, 1000, 64, 1) == lib.fa_bwd_workspace_size(2, 3, 1000, 64) + 256
+    assert lib.fa_bwd_qk(A, A, A, A, A, A, A, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, 0, A, ws - 4, None) == 1
+    assert lib.fa_bwd_qk(A, A, A, A, A, A, 0, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, 0, A, ws, None) == 1
+    assert lib.fa_bwd_qk(A, A, A, A, A, A, A, A, A, 1, 1, 128, 300, 64, 1, 0.125, 0.0, 0, 0, 1, A, ws, None) == 1
 
 
 def test_stage_entry_points_reject_bad_arguments(lib):

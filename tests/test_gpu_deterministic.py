@@ -1,0 +1,100 @@
+"""Deterministic backward (fa_bwd_qk / fa_bwd_varlen with deterministic != 0):
+repeated calls on the same inputs give bitwise-identical dQ, dK and dV, the
+result still matches the fp64 oracle with the usual bounds, and it equals the
+default (atomic-order) backward up to fp32 summation order."""
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_49_b200 import workloads as wl
+from oracle import attention
+from tests import parity_util as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    return t.view(torch.int16)
+
+
+def _grads(q, k, v, o, do, lse, causal, scale, p, seed, det):
+    from exact_io_aware_49_b200 import fa_bwd
+    g = fa_bwd(q, k, v, o, do, lse, causal, scale, p, seed, deterministic=det)
+    torch.cuda.synchronize()
+    return g
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal,p", [
+    (4, 16, 4096, 4096, 128, True, 0.1),   # the N = 4096 benchmark shape
+    (2, 8, 1024, 1024, 64, False, 0.0),
+    (1, 4, 700, 1500, 128, True, 0.1),     # Nq != Nk, bottom-right causal
+    (2, 2, 1500, 700, 64, True, 0.0),      # rows that see no key
+])
+def test_repeatable_and_exact(B, H, Nq, Nk, d, causal, p):
+    from exact_io_aware_49_b200 import fa_fwd
+    gen = torch.Generator().manual_seed(B * 1000 + Nq + Nk)
+    q, do = (torch.randn(B, H, Nq, d, generator=gen).to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn(B, H, Nk, d, generator=gen).to(torch.bfloat16) for _ in range(2))
+    scale, seed = d ** -0.5, 17
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = fa_fwd(qd, kd, vd, causal, scale, p, seed)
+    first = _grads(qd, kd, vd, o, dod, lse, causal, scale, p, seed, True)
+    for _ in range(2):
+        again = _grads(qd, kd, vd, o, dod, lse, causal, scale, p, seed, True)
+        for a, b in zip(first, again):
+            assert torch.equal(_bits(a), _bits(b))
+    default = _grads(qd, kd, vd, o, dod, lse, causal, scale, p, seed, False)
+    for a, b in zip(first, default):
+        assert pu.rel_fro(pu.f64(a), pu.f64(b)) < 1e-3
+    # against the oracle on two heads
+    for b_, h_ in ((0, 0), (B - 1, H - 1)):
+        args = [x[b_, h_].to(torch.float64).numpy() for x in (q, k, v, do)]
+        want = attention.backward(*args, causal=causal, scale=scale, p_drop=p, seed=seed, b=b_, h=h_)[:3]
+        for got, w, name in zip(first, want, ("dQ", "dK", "dV")):
+            pu.check_grad(pu.f64(got[b_, h_].cpu()), w, f"{name} {(b_, h_)}")
+
+
+def test_varlen_repeatable_and_exact():
+    from exact_io_aware_49_b200 import fa_bwd_varlen, fa_fwd_varlen
+    lens, H, d, p, seed = [700, 1, 1300, 129], 2, 128, 0.1, 3
+    gen = torch.Generator().manual_seed(5)
+    total = sum(lens)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    q, k, v, do = (torch.randn(total, H, d, generator=gen).to(torch.bfloat16) for _ in range(4))
+    qd, kd, vd, dod, cud = (x.cuda() for x in (q, k, v, do, cu))
+    o, lse = fa_fwd_varlen(qd, kd, vd, cud, cud, max(lens), max(lens), True, d ** -0.5, p, seed)
+    runs = []
+    for _ in range(3):
+        runs.append(fa_bwd_varlen(qd, kd, vd, o, dod, lse, cud, cud, max(lens), max(lens), True, d ** -0.5, p, seed,
+                                  deterministic=True))
+        torch.cuda.synchronize()
+    for again in runs[1:]:
+        for a, b in zip(runs[0], again):
+            assert torch.equal(_bits(a), _bits(b))
+    dq, dk, dv = (x.cpu() for x in runs[0])
+    s0, s1 = int(cu[2]), int(cu[3])  # the longest sequence
+    for h in range(H):
+        args = [x[s0:s1, h].to(torch.float64).numpy() for x in (q, k, v, do)]
+        want = attention.backward(*args, causal=True, scale=d ** -0.5, p_drop=p, seed=seed, b=2, h=h)[:3]
+        for got, w, name in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+            pu.check_grad(pu.f64(got[s0:s1, h]), w, f"{name} seq 2 head {h}")
+
+
+def test_full_size_benchmark_shape_repeatable():
+    """The long-context shape (1 x 32 x 32768 x 128, causal, p = 0.1): two
+    deterministic runs agree bit for bit."""
+    from exact_io_aware_49_b200 import fa_fwd
+    w = wl.BY_NAME["causal_dropout_N32768_d128"]
+    q, k, v, do = (x.cuda() for x in wl.draw_inputs(w))
+    o, lse = fa_fwd(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    a = _grads(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, True)
+    b = _grads(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, True)
+    for x, y in zip(a, b):
+        assert torch.equal(_bits(x), _bits(y))
+    assert torch.isfinite(a[0].float()).all()
+
+
+def test_no_device_wait_timed_out():
+    from exact_io_aware_49_b200 import fa_last_device_error
+    assert fa_last_device_error() == 0
