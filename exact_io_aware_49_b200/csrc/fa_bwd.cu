@@ -326,7 +326,7 @@ __device__ __forceinline__ void mark_dropped4(float* P, uint32_t nib) {
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT, bool F16>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16, bool DET>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const size_t vrow0 = static_cast<size_t>(unit) * Npad;  // this unit's rows in the padded LSE2 / D vectors
   // query tile of iteration it: ascending from q_first, or descending from the
   // last tile in deterministic mode
-  const bool det = p.dq_order != nullptr;
+  constexpr bool det = DET;
   auto qi_of = [&](int it) { return det ? n_qt - 1 - it : q_first + it; };
 
   if (threadIdx.x == 0) {
@@ -711,9 +711,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT, bool F16>
+template <int D, bool CAUSAL, bool DROPOUT, bool F16, bool DET>
 cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
-  auto kern = fa_bwd_kernel<D, CAUSAL, DROPOUT, F16>;
+  auto kern = fa_bwd_kernel<D, CAUSAL, DROPOUT, F16, DET>;
   const int used = BwdSmem<D>::kUsed;
   int max_optin = 0, dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -772,17 +772,21 @@ void launch_preprocess_typed(const BwdArgs& a, long long blocks, int Npad, long 
         O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, Npad, acc_vec4, a.dq_order, n_order);
 }
 
-template <bool F16>
+template <bool F16, bool DET>
 cudaError_t launch_bwd_tiles_typed(const BwdArgs& a, cudaStream_t stream) {
   const bool drop = a.drop_t != 0;
   if (a.d == 64) {
     if (a.causal)
-      return drop ? launch_bwd_main<64, true, true, F16>(a, stream) : launch_bwd_main<64, true, false, F16>(a, stream);
-    return drop ? launch_bwd_main<64, false, true, F16>(a, stream) : launch_bwd_main<64, false, false, F16>(a, stream);
+      return drop ? launch_bwd_main<64, true, true, F16, DET>(a, stream)
+                  : launch_bwd_main<64, true, false, F16, DET>(a, stream);
+    return drop ? launch_bwd_main<64, false, true, F16, DET>(a, stream)
+                : launch_bwd_main<64, false, false, F16, DET>(a, stream);
   }
   if (a.causal)
-    return drop ? launch_bwd_main<128, true, true, F16>(a, stream) : launch_bwd_main<128, true, false, F16>(a, stream);
-  return drop ? launch_bwd_main<128, false, true, F16>(a, stream) : launch_bwd_main<128, false, false, F16>(a, stream);
+    return drop ? launch_bwd_main<128, true, true, F16, DET>(a, stream)
+                : launch_bwd_main<128, true, false, F16, DET>(a, stream);
+  return drop ? launch_bwd_main<128, false, true, F16, DET>(a, stream)
+              : launch_bwd_main<128, false, false, F16, DET>(a, stream);
 }
 
 }  // namespace
@@ -803,7 +807,11 @@ cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream) {
-  return a.f16 ? launch_bwd_tiles_typed<true>(a, stream) : launch_bwd_tiles_typed<false>(a, stream);
+  // deterministic mode is a separate instantiation, so the default kernel
+  // carries none of its code
+  if (a.dq_order)
+    return a.f16 ? launch_bwd_tiles_typed<true, true>(a, stream) : launch_bwd_tiles_typed<false, true>(a, stream);
+  return a.f16 ? launch_bwd_tiles_typed<true, false>(a, stream) : launch_bwd_tiles_typed<false, false>(a, stream);
 }
 
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
