@@ -19,6 +19,9 @@ exactly to fp64):
   ("DL0056 FlashAttention", Mathematical Formulation) written out step by
   step; it exists only so the tests can show that it equals the two-pass
   definition above.
+* ``paged.decode_forward`` -- attention over a paged key/value cache:
+  gathers each sequence's pages back into contiguous keys and values and
+  applies ``attention.forward`` (grouped-query heads share a key/value head).
 * ``philox`` -- Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random
   Numbers: As Easy as 1, 2, 3", SC'11) and the dropout keep-mask built on it.
 
@@ -31,6 +34,6 @@ against an independent library implementation (ATen's header-only
 function here is "parity unpinned".
 """
 
-from . import philox, attention, online  # noqa: F401
+from . import philox, attention, online, paged  # noqa: F401
 
-__all__ = ["philox", "attention", "online"]
+__all__ = ["philox", "attention", "online", "paged"]

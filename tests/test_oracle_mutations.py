@@ -137,3 +137,20 @@ def test_top_left_alignment_for_rectangular_is_caught():
     assert np.abs(mutant - want).max() > 1e-3
     got, _ = attention.forward(q, k, v, causal=True, scale=0.2)
     assert np.abs(got - want).max() < 1e-12
+
+
+def test_interleaved_gqa_head_mapping_is_caught():
+    """Query head h reads key/value head h // (H / H_kv); a mutant that reads
+    h % H_kv gives the wrong mean of V for the Q = 0 closed form."""
+    rng = np.random.default_rng(12)
+    H, H_kv, L, d = 6, 2, 9, 3
+    v = rng.standard_normal((L, H_kv, d))
+    want = [v[:, h // 3].mean(0) for h in range(H)]
+    mutant = [v[:, h % H_kv].mean(0) for h in range(H)]
+    assert max(np.abs(a - b).max() for a, b in zip(mutant, want)) > 1e-3
+    from oracle import paged
+    cache = v[None]  # one page holding all L positions
+    o, _ = paged.decode_forward(np.zeros((1, H, 1, d)), cache, cache, np.zeros((1, 1), dtype=np.int32),
+                                np.array([L]), causal=False, scale=1.0)
+    for h in range(H):
+        assert np.abs(o[0, h, 0] - want[h]).max() < 1e-12
