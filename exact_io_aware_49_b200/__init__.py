@@ -6,7 +6,8 @@ the package does not load the library; the first use of an entry point does,
 and fails loudly if the library is missing -- there is no fallback path.
 """
 
-_BINDING_NAMES = ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_stages", "fa_bwd_workspace_size",
+_BINDING_NAMES = ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_paged", "fa_bwd_stages",
+                  "fa_bwd_workspace_size",
                   "fa_dropout_mask", "fa_last_device_error", "fa_selftest_wait_timeout", "FAError", "load_library")
 
 

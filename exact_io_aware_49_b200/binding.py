@@ -65,6 +65,12 @@ def load_library(path=None):
     lib.fa_bwd_tiles.restype = i
     lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd_finish.restype = i
+    lib.fa_decode_num_splits.argtypes = [i, i, i, i, i]
+    lib.fa_decode_num_splits.restype = i
+    lib.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_decode_workspace_size.restype = sz
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, f, i, i, vp, sz, vp]
+    lib.fa_decode_paged.restype = i
     lib.fa_dropout_mask.argtypes = [vp, i, i, i, f, u64, vp]
     lib.fa_dropout_mask.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
@@ -282,6 +288,38 @@ def fa_bwd_stages(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, w
     if between:
         between(3)
     return dq, dk, dv
+
+
+def fa_decode_paged(q, k_cache, v_cache, block_table, seqlens_k, max_seqlen_k, causal, scale=None, num_splits=0,
+                    out=None, lse=None, workspace=None):
+    """(O [B, H, Nq, d], LSE [B, H, Nq]) of q over a paged key/value cache:
+    k_cache, v_cache [num_pages, page_size, H_kv, d]; block_table int32 [B, max_pages];
+    seqlens_k int32 [B] (all on the device); num_splits = 0 chooses the split count."""
+    lib = load_library()
+    _check_bhnd("q", q)
+    B, H, Nq, d = q.shape
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if not t.is_cuda or t.dtype != q.dtype or t.dim() != 4 or not t.is_contiguous() or t.shape[3] != d:
+            raise ValueError(f"{name} must be a contiguous [num_pages, page_size, H_kv, d] tensor of q's type")
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("v_cache must have k_cache's shape")
+    num_pages, page, H_kv, _ = k_cache.shape
+    for name, t, shape in (("block_table", block_table, (B, block_table.shape[-1])), ("seqlens_k", seqlens_k, (B,))):
+        if not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of shape {shape}")
+    scale = d ** -0.5 if scale is None else scale
+    splits = int(num_splits) or int(lib.fa_decode_num_splits(B, H_kv, H, Nq, int(max_seqlen_k)))
+    ws_bytes = int(lib.fa_decode_workspace_size(B, H, Nq, d, splits)) if splits > 0 else 0
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    _raise(lib.fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                               seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, H_kv, Nq, d, num_pages,
+                               page, block_table.shape[1], int(max_seqlen_k), int(bool(causal)), float(scale), splits,
+                               FA_DTYPE[q.dtype], workspace.data_ptr() if workspace is not None else None,
+                               workspace.numel() if workspace is not None else 0, _stream(q)), "fa_decode_paged")
+    return out, lse
 
 
 def fa_dropout_mask(B, H, N, p_drop, seed, device="cuda"):

@@ -460,6 +460,115 @@ fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void*
   return bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
 
+// ------------------------------------------------------------ decoding over a paged cache
+
+int fa_decode_num_splits(int B, int H_kv, int H, int Nq, int max_seqlen_k) {
+  if (B <= 0 || H_kv <= 0 || H <= 0 || Nq <= 0 || max_seqlen_k <= 0 || H % H_kv != 0) return 0;
+  const long long rows = static_cast<long long>(H / H_kv) * Nq;
+  const long long chunks = (rows + fa::decode_rows_per_cta() - 1) / fa::decode_rows_per_cta();
+  const long long ctas = static_cast<long long>(B) * H_kv * chunks;
+  const int tiles = (max_seqlen_k + fa::decode_keys_per_tile() - 1) / fa::decode_keys_per_tile();
+  // about two waves of CTAs on 148 SMs, at least one tile per split
+  long long splits = (2 * 148 + ctas - 1) / ctas;
+  if (splits > tiles) splits = tiles;
+  if (splits > 128) splits = 128;
+  if (splits < 1) splits = 1;
+  // no split without a tile: recompute from the tiles per split
+  const int per = static_cast<int>((tiles + splits - 1) / splits);
+  return (tiles + per - 1) / per;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || d <= 0 || num_splits <= 0) return 0;
+  if (num_splits == 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * Nq * num_splits;
+  return round_up(rows * d * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+fa_status fa_decode_paged(const void* Q, const void* K_cache, const void* V_cache, const int32_t* block_table,
+                          const int32_t* seqlens_k, void* O, float* LSE, int B, int H, int H_kv, int Nq, int d,
+                          int num_pages, int page_size, int max_pages_per_seq, int max_seqlen_k, int causal,
+                          float scale, int num_splits, fa_dtype dtype, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  if (!Q || !K_cache || !V_cache || !block_table || !seqlens_k || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (misaligned(Q, 16) || misaligned(K_cache, 16) || misaligned(V_cache, 16) || misaligned(O, 16) ||
+      misaligned(LSE, 4) || misaligned(block_table, 4) || misaligned(seqlens_k, 4))
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || H_kv <= 0 || Nq <= 0 || d <= 0 || num_pages <= 0 || page_size <= 0 ||
+      max_pages_per_seq <= 0 || max_seqlen_k <= 0 || num_splits < 0)
+    return FA_ERR_INVALID_ARG;
+  if (H % H_kv != 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_seqlen_k) > static_cast<long long>(max_pages_per_seq) * page_size)
+    return FA_ERR_INVALID_ARG;
+  fa_status st = check_scalars(d, scale, 0.0f);
+  if (st != FA_OK) return st;
+  if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_pages) * page_size >= (1ll << 31) ||
+      static_cast<long long>(B) * max_pages_per_seq >= (1ll << 31) ||
+      static_cast<long long>(B) * H * Nq >= (1ll << 31) || B > 65535)
+    return FA_ERR_UNSUPPORTED;
+  const int splits = num_splits ? num_splits : fa_decode_num_splits(B, H_kv, H, Nq, max_seqlen_k);
+  if (splits < 1 || splits > 1024) return FA_ERR_INVALID_ARG;
+  if (splits > 1) {
+    if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fa_decode_workspace_size(B, H, Nq, d, splits)) return FA_ERR_INVALID_ARG;
+  }
+  const int group = H / H_kv;
+  const int rows = group * Nq;
+  const int chunks = (rows + fa::decode_rows_per_cta() - 1) / fa::decode_rows_per_cta();
+  if (static_cast<long long>(H_kv) * chunks > 65535) return FA_ERR_UNSUPPORTED;
+
+  fa::DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  const CUtensorMapDataType dt = elem_type(dtype == FA_DTYPE_F16);
+  // (d, H_kv, num_pages * page_size) over [num_pages, page_size, H_kv, d]; one box = one page of one head
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_kv),
+                        static_cast<cuuint64_t>(num_pages) * page_size};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H_kv) * d * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(page_size)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (enc(&a.tmK, dt, 3, const_cast<void*>(K_cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+          CUDA_SUCCESS ||
+      enc(&a.tmV, dt, 3, const_cast<void*>(V_cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+          CUDA_SUCCESS)
+    return FA_ERR_CUDA;
+  fa::DecodeParams& p = a.p;
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.O = static_cast<uint16_t*>(O);
+  p.LSE = LSE;
+  if (splits > 1) {
+    const size_t prow = static_cast<size_t>(B) * H * Nq * splits;
+    p.O_part = static_cast<float*>(workspace);
+    p.LSE_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(prow * d * sizeof(float), 256));
+  }
+  p.block_table = block_table;
+  p.seqlens = seqlens_k;
+  p.err = error_word_ptr();
+  if (!p.err) return FA_ERR_CUDA;
+  p.H = H;
+  p.Nq = Nq;
+  p.group = group;
+  p.rows = rows;
+  p.row_chunks = chunks;
+  p.max_pages = max_pages_per_seq;
+  p.page = page_size;
+  const int tiles = (max_seqlen_k + fa::decode_keys_per_tile() - 1) / fa::decode_keys_per_tile();
+  p.splits = splits;
+  p.tiles_per_split = (tiles + splits - 1) / splits;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  a.B = B;
+  a.H_kv = H_kv;
+  a.d = d;
+  a.f16 = dtype == FA_DTYPE_F16 ? 1 : 0;
+  return fa::launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ utilities
 
 fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed, void* stream) {

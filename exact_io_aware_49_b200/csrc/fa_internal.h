@@ -110,6 +110,35 @@ struct BwdArgs {
   uint32_t philox_rk[20];  // Philox round keys of the seed (rounds 0..9, k0 / k1 interleaved)
 };
 
+// Decoding over a paged key/value cache (fa_decode.cu).
+struct DecodeParams {
+  const uint16_t* Q;   // [B, H, Nq, d]
+  uint16_t* O;         // [B, H, Nq, d]
+  float* LSE;          // [B, H, Nq]
+  float* O_part;       // fp32 [B, H, Nq, splits, d] workspace (splits > 1)
+  float* LSE_part;     // fp32 [B, H, Nq, splits] workspace (splits > 1)
+  const int* block_table;  // [B, max_pages]
+  const int* seqlens;      // [B]
+  unsigned* err;
+  int H, Nq, group;    // group = H / H_kv query heads per key/value head
+  int rows;            // group * Nq query rows per key/value head
+  int row_chunks;      // blocks of up to 16 rows
+  int max_pages, page;
+  int splits, tiles_per_split;
+  int causal;
+  float scale_log2;
+};
+
+struct DecodeArgs {
+  CUtensorMap tmK, tmV;  // (d, H_kv, num_pages * page) maps, 64 x 1 x page boxes, 128B swizzle
+  DecodeParams p;
+  int B, H_kv, d, f16;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int decode_rows_per_cta();
+int decode_keys_per_tile();
+
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
 // The three backward stages; fa_bwd runs them in this order.  Only the fields
 // each stage reads need to be set.

@@ -294,6 +294,43 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
                          float p_drop, uint64_t seed, void* stream);
 
 /*
+ * Decoding over a paged key/value cache: exact attention of the newest Nq
+ * queries of each sequence over all of its cached positions, with the cache
+ * kept in fixed-size pages that need not be contiguous (the serving setting
+ * of the "FlashAttention" glossary's vLLM / PagedAttention entries).
+ *   Q, O        : [B, H, Nq, d] of ``dtype``; O = softmax(scale Q K^T + mask) V
+ *   LSE         : out, fp32 [B, H, Nq]
+ *   K_cache, V_cache : [num_pages, page_size, H_kv, d] of ``dtype``
+ *   block_table : DEVICE int32 [B, max_pages_per_seq]; entry (b, n) is the
+ *                 page holding positions n*page_size .. of sequence b (only
+ *                 the entries covering seqlens_k[b] are read)
+ *   seqlens_k   : DEVICE int32 [B], cached positions of each sequence
+ *                 (clamped to [0, max_pages_per_seq * page_size])
+ *   H_kv        : key/value heads; H must be a multiple of it and query head
+ *                 h reads key/value head h / (H / H_kv)
+ *   causal      : nonzero -> query i of sequence b is position
+ *                 seqlens_k[b] - Nq + i and sees positions up to it
+ *   max_seqlen_k: the largest seqlens_k entry (sizes the launch)
+ *   page_size   : 16, 32, 64 or 128; d in {64, 128}; no dropout
+ *   num_splits  : how many parts each sequence's positions are cut into
+ *                 (each a thread block, merged by log-sum-exp); 0 chooses
+ *                 fa_decode_num_splits(); with more than one split the call
+ *                 needs ``workspace`` of fa_decode_workspace_size() bytes,
+ *                 256-byte aligned (with one split it may be NULL).
+ * A row that sees no position gets O = 0 and LSE = -inf.  Page ids outside
+ * [0, num_pages) read as zeros; the tables live on the device, so the library
+ * cannot check them otherwise.
+ */
+int fa_decode_num_splits(int B, int H_kv, int H, int Nq, int max_seqlen_k);
+size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int num_splits);
+fa_status fa_decode_paged(const void* Q, const void* K_cache, const void* V_cache,
+                          const int32_t* block_table, const int32_t* seqlens_k,
+                          void* O, float* LSE, int B, int H, int H_kv, int Nq, int d,
+                          int num_pages, int page_size, int max_pages_per_seq, int max_seqlen_k,
+                          int causal, float scale, int num_splits, fa_dtype dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Test/inspection export: writes the dropout keep mask Z (1 = kept, 0 =
  * dropped) as uint8 [B, H, N, N] into device memory ``mask`` with the same
  * device Philox code the kernels use.  N here only needs to be positive.

@@ -185,3 +185,29 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(ImportError):
         binding.load_library(str(tmp_path / "missing.so"))
+
+
+def _decode(lib, Q=A, BT=A, SL=A, B=2, H=8, H_kv=2, Nq=1, d=128, pages=64, page=16, maxp=8, maxk=100, scale=0.1,
+            splits=1, dtype=0, ws=0, ws_bytes=0):
+    return lib.fa_decode_paged(Q, A, A, BT, SL, A, A, B, H, H_kv, Nq, d, pages, page, maxp, maxk, 1, scale, splits,
+                               dtype, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(Q=0), 1), (dict(BT=0), 1), (dict(SL=A + 2), 1), (dict(H=6, H_kv=4), 1), (dict(maxk=129), 1),
+    (dict(scale=0.0), 1), (dict(dtype=5), 1), (dict(splits=-1), 1), (dict(splits=3), 1),  # no workspace
+    (dict(page=8, maxp=16), 2), (dict(page=48), 2), (dict(d=96), 2), (dict(Nq=0), 1),
+])
+def test_decode_rejects_bad_arguments(lib, kw, want):
+    assert _decode(lib, **kw) == want
+
+
+def test_decode_split_choice_and_workspace(lib):
+    # one split when there are already enough (sequence, head) blocks; more for few long sequences
+    assert lib.fa_decode_num_splits(64, 8, 32, 1, 4096) == 1
+    s = lib.fa_decode_num_splits(1, 8, 32, 1, 32768)
+    assert 2 <= s <= 128
+    assert lib.fa_decode_num_splits(1, 1, 1, 1, 100) == 1  # a single 128-key tile cannot be split
+    assert lib.fa_decode_num_splits(1, 3, 4, 1, 100) == 0  # H not a multiple of H_kv
+    assert lib.fa_decode_workspace_size(2, 8, 1, 128, 1) == 0
+    assert lib.fa_decode_workspace_size(2, 8, 1, 128, 4) == 2 * 8 * 4 * 128 * 4 + 256
