@@ -13,23 +13,32 @@
 //   * a row that sees no key gets O = 0, LSE = -inf.
 //
 // Design (B200).  Decoding reads every cached key and value once and does
-// ~2 * rows FLOPs per element, so for the few query rows per key/value head
-// that decoding has, the kernel is HBM-bound: it streams 128-key tiles (1 to
-// 8 pages each, located through the block table) with TMA into 128-byte-
-// swizzled shared memory through a 3- or 4-stage mbarrier ring and does the
-// arithmetic on the CUDA cores in fp32.
-//   * grid = (split, key/value head x block of up to 16 query rows, sequence):
-//     the rows of all query heads sharing a key/value head are done together,
-//     so each cached byte is read once per row block; long sequences are cut
-//     into splits that run on different SMs;
-//   * per tile (512 threads): four lanes per key compute the scores of all
-//     rows, one warp per row updates the running max / sum and turns scores
-//     into probabilities, and each thread accumulates P V for a column pair
-//     over a group of the tile's keys (packed f32x2 FMAs); the key groups are
-//     added once at the end;
-//   * splits write fp32 partial outputs with their LSE; a merge kernel
-//     combines them with the log-sum-exp weights (one split writes the final
-//     output directly).
+// ~2 * rows FLOPs per element; the arithmetic is a pair of small products per
+// 128-key tile, so it runs on the tensor cores in the transposed form where
+// the 128 keys are the M = 128 side and the (up to 16) query rows the N = 16
+// side, leaving the CUDA cores only the softmax:
+//   * S^T = K_tile Q^T   (tcgen05, A = K tile, B = Q rows, fp32 in TMEM:
+//     lane = key, column = query row);
+//   * softmax over keys, i.e. across TMEM lanes: each of 128 threads holds
+//     one key's 16 scores, a 16-shuffle reduce-scatter per warp and one
+//     exchange through shared memory give every row's tile max and sum; the
+//     O rescale is lazy (stale max kept until a row's max grows by more than
+//     8 in log2 units, as in the forward kernel); P goes to shared memory as
+//     16-bit [16 rows x 128 keys];
+//   * O^T += V_tile^T P^T (tcgen05, A = V tile read MN-major, B = P; lane =
+//     dimension, column = query row);
+//   * warp 4 streams the tiles (1 to 8 pages each, located through the block
+//     table) with TMA through a 3-stage (d = 128) / 4-stage (d = 64) mbarrier
+//     ring and issues the MMAs; warps 0-3 do the softmax, the rescale and the
+//     epilogue.
+// For d = 64 the V tile carries a second, all-zero 64-column box so the P V
+// product keeps M = 128 (dimensions 64..127 come out as zeros).
+// grid = (split, key/value head x block of up to 16 query rows, sequence): all
+// query heads sharing a key/value head are done together, so each cached byte
+// is read once per row block; long sequences are cut into splits that run on
+// different SMs, written as fp32 partials with their LSE and combined by a
+// merge kernel with the log-sum-exp weights (one split writes the final
+// output directly).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -41,33 +50,73 @@
 namespace fa {
 namespace {
 
-constexpr int kDecThreads = 512;
-constexpr int kTileKeys = 128;  // keys per tile
-constexpr int kMaxRows = 8;     // query rows per CTA (one softmax warp each)
-constexpr int kKeyLanes = kDecThreads / kTileKeys;  // lanes per key in the score phase (4)
+constexpr int kDecThreads = 160;  // 4 softmax warps + 1 producer warp
+constexpr int kProducerWarp = 4;
+constexpr int kTileKeys = 128;    // keys per tile = TMEM lanes of S^T
+constexpr int kMaxRows = 16;      // query rows per CTA = N of both products
+constexpr float kDecRescaleTau = 8.0f;
 
 template <int D>
 struct DecSmem {
   static constexpr int kStages = (D == 128) ? 3 : 4;
-  static constexpr int kHalf = kTileKeys * D * 2;  // K or V tile: 128 keys x D 16-bit
-  static constexpr int kBox = kTileKeys * 128;     // one 64-column, 128-byte-row box of a tile
-  static constexpr int kStage = 2 * kHalf;         // K then V
-  // query rows, fp32, pre-scaled to log2 units; each of the kKeyLanes dimension
-  // parts of a row is padded by 4 floats so the lanes of a key read different banks
-  static constexpr int kQPart = D / kKeyLanes + 4;
-  static constexpr int kQ = kStages * kStage;
-  static constexpr int kS = kQ + kMaxRows * kKeyLanes * kQPart * 4;  // fp32 [kMaxRows][kTileKeys]
-  static constexpr int kStat = kS + kMaxRows * kTileKeys * 4;         // m, l, alpha: fp32 [kMaxRows] each
-  static constexpr int kBar = kStat + 3 * kMaxRows * 4;
-  static constexpr int kMisc = kBar + kStages * 8;  // abort flag
+  static constexpr int kBox = kTileKeys * 128;  // one 64-column, 128-byte-row box of a tile (16 KB)
+  static constexpr int kKBytes = kTileKeys * D * 2;
+  static constexpr int kVBytes = 2 * kBox;       // two boxes; for d = 64 the second stays zero
+  static constexpr int kStage = kKBytes + kVBytes;
+  static constexpr int kQ = kStages * kStage;    // Q rows: [16][D] 16-bit, 128B-swizzled K-major
+  static constexpr int kP = kQ + kMaxRows * D * 2;  // P: 2 x [16][128] 16-bit, 128B-swizzled K-major
+  static constexpr int kPBytes = kMaxRows * kTileKeys * 2;
+  static constexpr int kRed = kP + 2 * kPBytes;  // fp32 [2 parities][max, sum][16 rows][4 warps]
+  static constexpr int kBar = kRed + 2 * 2 * kMaxRows * 4 * 4;
+  // full[kStages], s_ready[2], p_ready[2], pv_done[2], drain (the pairs by tile parity: a
+  // role may run one tile ahead of the role that waits, never two)
+  static constexpr int kNumBars = kStages + 7;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kUsed = kMisc + 16;
-  // P V: each thread owns a column pair and a group of the tile's keys; the
-  // groups' partial sums are added once at the end (through the stage buffers)
-  static constexpr int kColPairs = D / 2;
-  static constexpr int kKeyGroups = kDecThreads / kColPairs;  // 8 (D = 128) or 16 (D = 64)
-  static constexpr int kKeysPerGroup = kTileKeys / kKeyGroups;
-  static_assert(kKeyGroups * kMaxRows * D * 4 <= kStages * kStage, "partial sums fit the stage buffers");
 };
+
+// Reduce-scatter of 16 per-lane values over a warp: afterwards the lanes with
+// bit 0 clear hold the warp-wide max (kMax) or sum of column
+// col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter16(float (&v)[16], int lane) {
+  float a[8], b4[4], c2[2];
+  const bool up16 = lane & 16, up8 = lane & 8, up4 = lane & 4, up2 = lane & 2;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float send = up16 ? v[k] : v[k + 8];
+    const float keep = up16 ? v[k + 8] : v[k];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+    a[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float send = up8 ? a[k] : a[k + 4];
+    const float keep = up8 ? a[k + 4] : a[k];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+    b4[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float send = up4 ? b4[k] : b4[k + 2];
+    const float keep = up4 ? b4[k + 2] : b4[k];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+    c2[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+  float d;
+  {
+    const float send = up2 ? c2[0] : c2[1];
+    const float keep = up2 ? c2[1] : c2[0];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+    d = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+  const float recv = __shfl_xor_sync(0xffffffffu, d, 1);
+  return kMax ? fmaxf(d, recv) : d + recv;
+}
+
+__device__ __forceinline__ int scatter_col(int lane) {
+  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+}
 
 template <int D, bool F16>
 __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -78,15 +127,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (!smem_layout_fits(smem_raw, smem, L::kUsed, p.err)) return;
-  float* qs = reinterpret_cast<float*>(smem + L::kQ);
-  float* ss = reinterpret_cast<float*>(smem + L::kS);
-  float* m_s = reinterpret_cast<float*>(smem + L::kStat);
-  float* l_s = m_s + kMaxRows;
-  float* a_s = l_s + kMaxRows;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
+  uint64_t* s_ready = full + S;  // [2], by tile parity
+  uint64_t* p_ready = s_ready + 2;  // [2], by tile parity
+  uint64_t* pv_done = p_ready + 2;  // [2], by tile parity
+  uint64_t* drain = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  float* red = reinterpret_cast<float*>(smem + L::kRed);
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x;
   const int g = blockIdx.y / p.row_chunks;  // key/value head
   const int r0 = (blockIdx.y - g * p.row_chunks) * kMaxRows;
@@ -96,245 +147,298 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   const int Lk = min(max(p.seqlens[b], 0), p.max_pages * p.page);
   const int n_tiles = (Lk + kTileKeys - 1) / kTileKeys;
   const int t_begin = split * p.tiles_per_split;
-  const int t_end = min(n_tiles, t_begin + p.tiles_per_split);
+  const int n = max(0, min(n_tiles, t_begin + p.tiles_per_split) - t_begin);  // tiles of this split
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    mbar_init(&s_ready[0], 1);
+    mbar_init(&s_ready[1], 1);
+    mbar_init(&p_ready[0], 4);
+    mbar_init(&p_ready[1], 4);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  // query rows in fp32, multiplied by scale * log2(e) so scores come out in log2 units
-  for (int idx = tid; idx < R * (D / 8); idx += kDecThreads) {
+  // Q rows -> the B operand of S^T: [16][D], 128-byte rows in 64-column boxes
+  // (2 KB each), 16-byte chunks swizzled by row; rows past R are zero
+  uint8_t* qsm = smem + L::kQ;
+  for (int idx = tid; idx < kMaxRows * (D / 8); idx += kDecThreads) {
     const int r = idx / (D / 8), c8 = idx - r * (D / 8);
-    const int rr = r0 + r;
-    const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
-    const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((static_cast<size_t>(b) * p.H + h) * p.Nq + i) * D + c8 * 8);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    const int dim0 = c8 * 8, part = dim0 / (D / kKeyLanes), within = dim0 - part * (D / kKeyLanes);
-    float* dst = qs + (r * kKeyLanes + part) * L::kQPart + within;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack2<F16>(w[e]);
-      dst[2 * e] = f.x * p.scale_log2;
-      dst[2 * e + 1] = f.y * p.scale_log2;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R) {
+      const int rr = r0 + r;
+      const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
+      v = *reinterpret_cast<const uint4*>(p.Q + ((static_cast<size_t>(b) * p.H + h) * p.Nq + i) * D + c8 * 8);
+    }
+    *reinterpret_cast<uint4*>(qsm + (c8 / 8) * (kMaxRows * 128) + r * 128 + (((c8 % 8) ^ (r & 7)) << 4)) = v;
+  }
+  if (D == 64) {
+    // the second V box of every stage stays zero
+    for (int idx = tid; idx < S * (L::kBox / 16); idx += kDecThreads) {
+      const int s = idx / (L::kBox / 16), o = idx - s * (L::kBox / 16);
+      *reinterpret_cast<uint4*>(smem + s * L::kStage + L::kKBytes + L::kBox + o * 16) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  if (tid < kMaxRows) {
-    m_s[tid] = -CUDART_INF_F;
-    l_s[tid] = 0.f;
+  fence_proxy_async_smem();
+  if (warp == kProducerWarp) {
+    tmem_alloc(tmem_slot, 64);  // S^T double buffer: columns [0, 16) and [16, 32); O^T [32, 48)
+    tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_o = tmem + 32;  // S^T of tile it: tmem + (it & 1) * 16
 
-  // thread 0 streams the tiles: the pages of tile t that hold valid positions
-  auto issue = [&](int t, int st) {
-    const int pages_per_tile = kTileKeys / p.page;
-    const int first = t * kTileKeys;
-    const int pages_here = min(pages_per_tile, (Lk - first + p.page - 1) / p.page);
-    mbar_expect_tx(&full[st], static_cast<uint32_t>(pages_here * 2 * (D / 64) * p.page * 128));
-    for (int n = 0; n < pages_here; ++n) {
-      const int pid = p.block_table[static_cast<size_t>(b) * p.max_pages + first / p.page + n];
-      for (int c = 0; c < D / 64; ++c) {
-        uint8_t* kd = smem + st * L::kStage + c * L::kBox + n * p.page * 128;
-        // an out-of-range page id reads zeros (outside the tensor map)
-        tma_load_3d(kd, &tmK, c * 64, g, pid * p.page, &full[st]);
-        tma_load_3d(kd + L::kHalf, &tmV, c * 64, g, pid * p.page, &full[st]);
-      }
-    }
-  };
-  int issued = 0;
-  if (tid == 0) {
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-    for (int k = 0; k < S - 1 && t_begin + k < t_end; ++k) issue(t_begin + k, k);
-    issued = max(0, min(S - 1, t_end - t_begin));
-  }
-
-  // score phase mapping: key j, dimension part (kKeyLanes adjacent lanes per key)
-  const int sj = tid / kKeyLanes, spart = tid % kKeyLanes;
-  constexpr int kChunksPer = D / kKeyLanes / 8;  // 16-byte chunks per lane
-  // P V mapping: column pair cp, key group kg
-  const int cp = tid % L::kColPairs, kg = tid / L::kColPairs;
-  const int vcol = 2 * cp;
-  const int vbox = vcol / 64, vchunk = (vcol % 64) / 8, vbyte = (vcol % 8) * 2;
-  float acc[kMaxRows][2];
-#pragma unroll
-  for (int r = 0; r < kMaxRows; ++r) acc[r][0] = acc[r][1] = 0.f;
-
-  bool ok = true;
-  int stop_it = 0;  // first tile not consumed when the loop stops early
-  for (int t = t_begin, it = 0; t < t_end; ++t, ++it) {
-    const int st = it % S;
-    // the stage of tile t + S - 1 was last read in the previous iteration,
-    // which every thread has left (barrier at the end of the loop)
-    if (tid == 0 && t + S - 1 < t_end) {
-      issue(t + S - 1, (it + S - 1) % S);
-      ++issued;
-    }
-    if (!mbar_wait(&full[st], (it / S) & 1, abort_flag, p.err)) {
-      ok = false;
-      stop_it = it;
-      break;
-    }
-    const int first = t * kTileKeys;
-    const int nvalid = min(kTileKeys, Lk - first);
-    const uint8_t* kt = smem + st * L::kStage;
-    const uint8_t* vt = kt + L::kHalf;
-
-    // ---- scores: kKeyLanes lanes per key, each a part of the dimensions
-    {
-      float s[kMaxRows];
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) s[r] = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < kChunksPer; ++cc) {
-        const int c = spart * kChunksPer + cc;  // 16-byte chunk of the row
-        const uint4 kv = *reinterpret_cast<const uint4*>(kt + (c / 8) * L::kBox + sj * 128 +
-                                                         (((c % 8) ^ (sj & 7)) << 4));
-        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
-        float kf[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack2<F16>(w[e]);
-          kf[2 * e] = f.x;
-          kf[2 * e + 1] = f.y;
-        }
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
-          if (r < R) {
-            const float* qr = qs + (r * kKeyLanes + spart) * L::kQPart + cc * 8;
-            const float4 q0 = *reinterpret_cast<const float4*>(qr);
-            const float4 q1 = *reinterpret_cast<const float4*>(qr + 4);
-            uint64_t a2 = fma_f2(f2_pack(q0.x, q0.y), f2_pack(kf[0], kf[1]), f2_pack(s[r], 0.f));
-            a2 = fma_f2(f2_pack(q0.z, q0.w), f2_pack(kf[2], kf[3]), a2);
-            a2 = fma_f2(f2_pack(q1.x, q1.y), f2_pack(kf[4], kf[5]), a2);
-            a2 = fma_f2(f2_pack(q1.z, q1.w), f2_pack(kf[6], kf[7]), a2);
-            float lo, hi;
-            f2_unpack(a2, lo, hi);
-            s[r] = lo + hi;
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA + MMA
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      auto issue = [&](int it) {
+        const int st = it % S;
+        const int first = (t_begin + it) * kTileKeys;
+        const int pages_here = min(kTileKeys / p.page, (Lk - first + p.page - 1) / p.page);
+        mbar_expect_tx(&full[st], static_cast<uint32_t>(pages_here * 2 * (D / 64) * p.page * 128));
+        for (int pg = 0; pg < pages_here; ++pg) {
+          const int pid = p.block_table[static_cast<size_t>(b) * p.max_pages + first / p.page + pg];
+          for (int c = 0; c < D / 64; ++c) {
+            // an out-of-range page id reads zeros (outside the tensor map)
+            uint8_t* kd = smem + st * L::kStage + c * L::kBox + pg * p.page * 128;
+            tma_load_3d(kd, &tmK, c * 64, g, pid * p.page, &full[st]);
+            tma_load_3d(kd + L::kKBytes, &tmV, c * 64, g, pid * p.page, &full[st]);
           }
         }
-      }
-      const int pos = first + sj;
+      };
+      const uint32_t q_addr = smem_u32(qsm);
+      constexpr uint32_t idesc_s = idesc_f32acc(128, kMaxRows, false, false, F16);
+      constexpr uint32_t idesc_o = idesc_f32acc(128, kMaxRows, true, false, F16);
+      int issued = 0;
+      for (; issued < min(S - 1, n); ++issued) issue(issued);
+      bool ok = true;
+      int consumed = 0;  // tiles whose copies have landed
+      // S^T = K Q^T of tile it into its TMEM buffer: M = 128 keys, N = 16 rows, K = D (both K-major)
+      auto issue_s = [&](int it) -> bool {
+        const int st = it % S;
+        if (!mbar_wait(&full[st], (it / S) & 1, abort_flag, p.err)) return false;
+        consumed = it + 1;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + st * L::kStage);
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) {
-        if (r < R) {
-          float v = s[r];
-#pragma unroll
-          for (int o = 1; o < kKeyLanes; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (spart == 0) {
-            const int i = (r0 + r) % p.Nq;
-            const bool visible = sj < nvalid && (!p.causal || pos <= Lk - p.Nq + i);
-            ss[r * kTileKeys + sj] = visible ? v : -CUDART_INF_F;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_k = (kk / 4) * L::kBox + (kk % 4) * 32;
+          const uint32_t off_q = (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
+          mma_ss(tmem + (it & 1) * 16, sdesc_sw128(k_addr + off_k, 16, 1024), sdesc_sw128(q_addr + off_q, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_ready[it & 1]);
+        return true;
+      };
+      ok = issue_s(0);
+      for (int it = 0; ok && it < n; ++it) {
+        // the next tile's S^T runs while the softmax warps work on this one; its
+        // buffer was last read by the softmax of tile it - 1 (p_ready seen below)
+        if (it + 1 < n && !issue_s(it + 1)) { ok = false; break; }
+        // refill the stage of tile it - 1 once its P V product has read it
+        if (issued < n) {
+          if (it >= 1 && !mbar_wait(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
+          issue(issued);
+          ++issued;
+        }
+        if (!mbar_wait(&p_ready[it & 1], (it >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        // O^T += V^T P^T: M = 128 dimensions (V read MN-major), N = 16 rows, K = 128 keys
+        const uint32_t v_addr = smem_u32(smem + (it % S) * L::kStage) + L::kKBytes;
+        const uint32_t p_addr = smem_u32(smem + L::kP + (it & 1) * L::kPBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+          const uint32_t off_p = (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
+          mma_ss(tm_o, sdesc_sw128(v_addr + kk * 2048, L::kBox, 1024), sdesc_sw128(p_addr + off_p, 16, 1024),
+                 idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&pv_done[it & 1]);
+      }
+      if (!ok) {
+        // copies and products in flight finish before shared and tensor memory go away
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+        for (int it2 = consumed; it2 < issued; ++it2) mbar_wait_drain(&full[it2 % S], (it2 / S) & 1);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_st[kMaxRows], l_r[kMaxRows];  // per row: stale max (log2 units) and sum, same in every thread
+#pragma unroll
+    for (int c = 0; c < kMaxRows; ++c) {
+      m_st[c] = -CUDART_INF_F;
+      l_r[c] = 0.f;
+    }
+    const int col = scatter_col(lane);
+    // Every wait below is bounded and may end differently in different
+    // threads; the named barriers AND the outcomes, so the 128 threads leave
+    // the loop together and tensor-memory instructions only run when all
+    // agree.
+    bool ok = true;
+    for (int it = 0; it < n; ++it) {
+      const int first = (t_begin + it) * kTileKeys;
+      const int j = warp * 32 + lane;  // this thread's key in the tile
+      const int pos = first + j;
+      ok = named_bar_and(1, 128, mbar_wait(&s_ready[it & 1], (it >> 1) & 1, abort_flag, p.err));
+      if (!ok) break;
+      tc_fence_after();
+      // S^T is done, so the tile's copies have landed.  V rows of positions
+      // past the sequence (or of pages not loaded) may hold anything, NaN
+      // included, and 0 * NaN would reach O through the tensor core: zero them.
+      if (pos >= Lk) {
+        uint8_t* vrow = smem + (it % S) * L::kStage + L::kKBytes + j * 128;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(vrow + c * L::kBox + q * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      uint32_t sr[16];
+      tmem_ld16(tmem + (it & 1) * 16 + lane_base, sr);
+      tmem_ld_wait();
+      reg_fence16(sr);
+      float s[16];
+#pragma unroll
+      for (int c = 0; c < kMaxRows; ++c) {
+        const int i = (r0 + c) % p.Nq;
+        const bool visible = c < R && pos < Lk && (!p.causal || pos <= Lk - p.Nq + i);
+        s[c] = visible ? __uint_as_float(sr[c]) * p.scale_log2 : -CUDART_INF_F;
+      }
+      // tile max per row: reduce over this warp's keys, then over the 4 warps
+      float* rmax = red + ((it & 1) * 2 + 0) * kMaxRows * 4;
+      float* rsum = red + ((it & 1) * 2 + 1) * kMaxRows * 4;
+      {
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = s[c];
+        const float wm = warp_reduce_scatter16<true>(v, lane);
+        if (!(lane & 1)) rmax[col * 4 + warp] = wm;
+      }
+      // (this barrier also covers the P buffer: the product of tile it - 2 has read it)
+      const bool p_free = (it < 2) || mbar_wait(&pv_done[it & 1], ((it - 2) >> 1) & 1, abort_flag, p.err);
+      ok = named_bar_and(1, 128, p_free);
+      if (!ok) break;
+      float alpha[kMaxRows];
+      bool rescale = false;  // the same in every thread: computed from the same shared values
+#pragma unroll
+      for (int c = 0; c < kMaxRows; ++c) {
+        const float4 w4 = *reinterpret_cast<const float4*>(rmax + c * 4);
+        const float m_tile = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+        const float m_new = fmaxf(m_st[c], m_tile);
+        alpha[c] = 1.f;
+        if (m_new > m_st[c] + kDecRescaleTau) {  // also the first visible key of the row (m_st = -inf)
+          alpha[c] = ex2_approx(m_st[c] - m_new);  // 0 when m_st = -inf
+          m_st[c] = m_new;
+          rescale = true;
+        }
+      }
+      float pv[16];
+#pragma unroll
+      for (int c = 0; c < kMaxRows; ++c) {
+        const float mu = (m_st[c] == -CUDART_INF_F) ? 0.f : m_st[c];
+        pv[c] = ex2_approx(s[c] - mu);  // 0 for masked keys
+      }
+      uint8_t* psm = smem + L::kP + (it & 1) * L::kPBytes;
+      {
+        const int box = j / 64, kin = j % 64;
+#pragma unroll
+        for (int c = 0; c < kMaxRows; ++c) {
+          const uint32_t bits = pack2<F16>(pv[c], 0.f);
+          *reinterpret_cast<uint16_t*>(psm + box * (kMaxRows * 128) + c * 128 + (((kin >> 3) ^ (c & 7)) << 4) +
+                                       (kin & 7) * 2) = static_cast<uint16_t>(bits & 0xFFFFu);
+        }
+      }
+      {
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = pv[c];
+        const float ws = warp_reduce_scatter16<false>(v, lane);
+        if (!(lane & 1)) rsum[col * 4 + warp] = ws;
+      }
+      // rescale O^T (lane = dimension) when a row's max moved: the previous
+      // P V product must have finished
+      const bool prev_done =
+          !(rescale && it > 0) || mbar_wait(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.err);
+      ok = named_bar_and(1, 128, prev_done);  // also: every row sum partial is written
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < kMaxRows; ++c) {
+        const float4 w4 = *reinterpret_cast<const float4*>(rsum + c * 4);
+        l_r[c] = l_r[c] * alpha[c] + ((w4.x + w4.y) + (w4.z + w4.w));
+      }
+      if (rescale && it > 0) {
+        tc_fence_after();
+        uint32_t orow[16];
+        tmem_ld16(tm_o + lane_base, orow);
+        tmem_ld_wait();
+        reg_fence16(orow);
+#pragma unroll
+        for (int c = 0; c < kMaxRows; ++c) orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha[c]);
+        tmem_st16(tm_o + lane_base, orow);
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[it & 1]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && n > 0)
+      ok = named_bar_and(1, 128, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.err));
+    if (ok) {
+      float o[16];
+      if (n > 0) {
+        tc_fence_after();
+        uint32_t orow[16];
+        tmem_ld16(tm_o + lane_base, orow);
+        tmem_ld_wait();
+        reg_fence16(orow);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) o[c] = __uint_as_float(orow[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) o[c] = 0.f;
+      }
+      const int dim = warp * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < kMaxRows; ++c) {
+        if (c >= R) continue;
+        const int rr = r0 + c;
+        const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
+        const size_t row = (static_cast<size_t>(b) * p.H + h) * p.Nq + i;
+        const float l = l_r[c];
+        const float val = (l > 0.f) ? o[c] / l : 0.f;
+        const float lse = (l > 0.f) ? (m_st[c] + lg2_approx(l)) * 0.69314718055994531f : -CUDART_INF_F;
+        if (dim < D) {
+          if (p.splits == 1)
+            p.O[row * D + dim] = static_cast<uint16_t>(pack2<F16>(val, 0.f) & 0xFFFFu);
+          else
+            p.O_part[(row * p.splits + split) * D + dim] = val;
+        }
+        if (dim == 0) {
+          if (p.splits == 1)
+            p.LSE[row] = lse;
+          else
+            p.LSE_part[row * p.splits + split] = lse;
         }
       }
     }
-    __syncthreads();
-
-    // ---- online softmax: warp r takes row r
-    {
-      const int r = tid >> 5, lane = tid & 31;
-      if (r < R) {
-        float4 x = *reinterpret_cast<const float4*>(ss + r * kTileKeys + lane * 4);
-        float mx = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_old = m_s[r];
-        const float m_new = fmaxf(m_old, mx);
-        const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;  // nothing visible yet: P = 0
-        x.x = ex2_approx(x.x - m_use);
-        x.y = ex2_approx(x.y - m_use);
-        x.z = ex2_approx(x.z - m_use);
-        x.w = ex2_approx(x.w - m_use);
-        float sum = (x.x + x.y) + (x.z + x.w);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        *reinterpret_cast<float4*>(ss + r * kTileKeys + lane * 4) = x;
-        if (lane == 0) {
-          const float alpha = (m_old == -CUDART_INF_F) ? 0.f : ex2_approx(m_old - m_use);
-          a_s[r] = alpha;
-          m_s[r] = m_new;
-          l_s[r] = l_s[r] * alpha + sum;
-        }
-      }
-    }
-    __syncthreads();
-
-    // ---- O += P V for this thread's column pair and key group
-    {
-#pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) {
-        if (r < R) {
-          const float a = a_s[r];
-          acc[r][0] *= a;
-          acc[r][1] *= a;
-        }
-      }
-      const int j_lo = kg * L::kKeysPerGroup;
-      const int j_hi = min(j_lo + L::kKeysPerGroup, nvalid);
-      const uint8_t* vb = vt + vbox * L::kBox + vbyte;
-      for (int j0 = j_lo; j0 < j_hi; j0 += 4) {
-        float2 v[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = j0 + e;
-          // rows past the sequence may hold anything: read them as 0
-          const uint32_t bits = *reinterpret_cast<const uint32_t*>(vb + j * 128 + ((vchunk ^ (j & 7)) << 4));
-          v[e] = (j < j_hi) ? unpack2<F16>(bits) : make_float2(0.f, 0.f);
-        }
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
-          if (r < R) {
-            const float4 pr = *reinterpret_cast<const float4*>(ss + r * kTileKeys + j0);
-            uint64_t a2 = f2_pack(acc[r][0], acc[r][1]);
-            a2 = fma_f2(f2_pack(pr.x, pr.x), f2_pack(v[0].x, v[0].y), a2);
-            a2 = fma_f2(f2_pack(pr.y, pr.y), f2_pack(v[1].x, v[1].y), a2);
-            a2 = fma_f2(f2_pack(pr.z, pr.z), f2_pack(v[2].x, v[2].y), a2);
-            a2 = fma_f2(f2_pack(pr.w, pr.w), f2_pack(v[3].x, v[3].y), a2);
-            f2_unpack(a2, acc[r][0], acc[r][1]);
-          }
-        }
-      }
-    }
-    __syncthreads();  // the stage and the probabilities may be overwritten now
   }
-
-  if (!ok) {
-    // let the copies already in flight land before the CTA's shared memory goes away
-    if (tid == 0)
-      for (int it = stop_it; it < issued; ++it) mbar_wait_drain(&full[it % S], (it / S) & 1);
-    __syncthreads();
-    return;
-  }
-
-  // ---- add the key groups' partial sums (the stage buffers are idle now)
-  float* part = reinterpret_cast<float*>(smem);  // [kKeyGroups][kMaxRows][D]
-#pragma unroll
-  for (int r = 0; r < kMaxRows; ++r)
-    if (r < R)
-      *reinterpret_cast<float2*>(part + (kg * kMaxRows + r) * D + vcol) = make_float2(acc[r][0], acc[r][1]);
+  // teardown: every role is done with tensor memory
+  tc_fence_before();
   __syncthreads();
-
-  // ---- outputs: the final row (one split) or an fp32 partial with its LSE
-  for (int idx = tid; idx < R * D; idx += kDecThreads) {
-    const int r = idx / D, col = idx - r * D;
-    float o = 0.f;
-#pragma unroll
-    for (int q = 0; q < L::kKeyGroups; ++q) o += part[(q * kMaxRows + r) * D + col];
-    const int rr = r0 + r;
-    const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
-    const size_t row = (static_cast<size_t>(b) * p.H + h) * p.Nq + i;
-    const float l = l_s[r];
-    o = (l > 0.f) ? o / l : 0.f;
-    const float lse = (l > 0.f) ? (m_s[r] + lg2_approx(l)) * 0.69314718055994531f : -CUDART_INF_F;
-    if (p.splits == 1) {
-      p.O[row * D + col] = static_cast<uint16_t>(pack2<F16>(o, 0.f) & 0xFFFFu);
-      if (col == 0) p.LSE[row] = lse;
-    } else {
-      p.O_part[(row * p.splits + split) * D + col] = o;
-      if (col == 0) p.LSE_part[row * p.splits + split] = lse;
-    }
-  }
+  tc_fence_after();
+  if (warp == kProducerWarp) tmem_dealloc(tmem, 64);
 }
 
 // One warp per output row: O = sum_s w_s O_s / sum_s w_s with w_s = exp(LSE_s - max),

@@ -79,12 +79,16 @@ def test_decode_matches_oracle(lens, H, H_kv, Nq, d, page, causal, splits):
 
 
 def test_split_counts_agree():
+    """Every split count is the same exact result up to rounding: P is rounded
+    to 16 bits against each split's own running maximum, so the outputs may
+    differ by the O bound (rel-Frobenius 5e-3); the fp32 LSE much less."""
     outs = []
     for splits in (1, 2, 5, 0):
         q, kc, vc, table, lens, o, lse = _run([3000, 1500], 8, 2, 1, 128, 16, True, splits, seed=3)
+        _check(q, kc, vc, table, lens, o, lse, True)
         outs.append((o, lse))
     for o, lse in outs[1:]:
-        assert pu.rel_fro(pu.f64(o), pu.f64(outs[0][0])) < 2e-3
+        assert pu.rel_fro(pu.f64(o), pu.f64(outs[0][0])) < pu.O_REL_FRO
         assert np.abs(pu.f64(lse) - pu.f64(outs[0][1])).max() < 1e-4
 
 
