@@ -78,7 +78,9 @@ long long pad128(long long n) { return (n + 127) / 128 * 128; }
 fa_status check_scalars(int d, float scale, float p_drop) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // 32 and 96 run on the 64- and 128-column kernels: the tensor maps read the
+  // columns past d as zeros and only d columns are stored
+  if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -557,6 +559,7 @@ fa_status fa_decode_paged(const void* Q, const void* K_cache, const void* V_cach
   p.row_chunks = chunks;
   p.max_pages = max_pages_per_seq;
   p.page = page_size;
+  p.dh = d;
   const int tiles = (max_seqlen_k + fa::decode_keys_per_tile() - 1) / fa::decode_keys_per_tile();
   p.splits = splits;
   p.tiles_per_split = (tiles + splits - 1) / splits;

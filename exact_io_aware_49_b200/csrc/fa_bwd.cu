@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
                                                                 float* __restrict__ Dvec,
                                                                 float* __restrict__ lse2,
                                                                 float* __restrict__ dQacc, const SeqLayout seq,
-                                                                int Npad, long long acc_vec4,
+                                                                int dh, int Npad, long long acc_vec4,
                                                                 unsigned* __restrict__ dq_order, int n_order) {
   const int lane = threadIdx.x & 31;
   const int rows_pad = seq.B * seq.H * Npad;  // < 2^31, checked on the host
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
     const size_t row = static_cast<size_t>(su.q0 + i) * seq.tok_stride + static_cast<size_t>(su.g) * seq.q_head_stride;
     // lane covers elements [8*lane, 8*lane+8) when 8*lane < D
     float acc = 0.f;
-    if (lane * 8 < D) {
+    if (lane * 8 < dh) {
       const uint4 a = *reinterpret_cast<const uint4*>(O + row + lane * 8);
       const uint4 b = *reinterpret_cast<const uint4*>(dO + row + lane * 8);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
@@ -122,15 +122,17 @@ template <bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ dQacc,
                                                                 uint16_t* __restrict__ dQ, float scale,
                                                                 const SeqLayout seq, int d, long long n8) {
-  const int shift = (d == 128) ? 4 : 3;  // log2(d / 8)
+  const int per_row = d / 8;
+  const int shift = (per_row == 16) ? 4 : (per_row == 8) ? 3 : (per_row == 4) ? 2 : -1;  // log2(d / 8), if any
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < n8;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     // fixed length: dQ has the accumulator's layout; packed: row g * total_q + t
     // of the accumulator is token t of head g in [total_q, H, d]
     long long dst = idx * 8;
     if (seq.cu_q) {
-      const int row = static_cast<int>(idx >> shift);  // < 2^31 rows
-      const int part = static_cast<int>(idx & ((1 << shift) - 1));
+      const long long rowl = (shift >= 0) ? (idx >> shift) : idx / per_row;
+      const int row = static_cast<int>(rowl);  // < 2^31 rows
+      const int part = static_cast<int>(idx - rowl * per_row);
       const int g = row / seq.total_q;
       const int t = row - g * seq.total_q;
       dst = t * seq.tok_stride + g * seq.q_head_stride + part * 8;
@@ -201,6 +203,7 @@ struct BwdParams {
   unsigned* dq_order;  // deterministic mode: per (unit, query tile) count of dQ adds done; else nullptr
   unsigned* err;
   SeqLayout seq;
+  int dh;  // head dimension of the tensors (D, or 32 / 96 padded to D = 64 / 128)
   float scale;
   float scale_log2;
   uint32_t drop_t;
@@ -366,7 +369,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       static_cast<size_t>(su.k0 + kj * 128 + (threadIdx.x & 127)) * p.seq.tok_stride +
                       static_cast<size_t>(su.g) * p.seq.k_head_stride;
       uint4* d4 = reinterpret_cast<uint4*>(dst);
-      for (int e = 0; e < D / 8; ++e) d4[e] = make_uint4(0u, 0u, 0u, 0u);
+      for (int e = 0; e < D / 8; ++e)
+        if (e * 8 < p.dh) d4[e] = make_uint4(0u, 0u, 0u, 0u);
     }
     return;
   }
@@ -549,8 +553,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
             // rows past the tensor are skipped; rows of the next packed
-            // sequence receive exact zeros (their P is 0 here)
-            tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, su.q0 + qrow, su.g);
+            // sequence receive exact zeros (their P is 0 here); boxes of
+            // padded columns (head dimension 32 / 96) are not issued
+            if (r * kCols + 32 * bx < p.dh)
+              tma_reduce_add_3d(&tmDQ, stage + bx * L::kBox, r * kCols + 32 * bx, su.q0 + qrow, su.g);
           bulk_commit_group();
           if (det && r == 1) {
             // both halves are in the accumulator before the next key tile may add
@@ -700,7 +706,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           o[e] = pack2<F16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-        if (key_valid) {
+        if (key_valid && 32 * c < p.dh) {  // padded columns are not stored
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
           for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
@@ -739,6 +745,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.Dvec = a.Dvec;
   p.err = a.err;
   p.seq = a.seq;
+  p.dh = a.d;
   p.scale = a.scale;
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
@@ -764,18 +771,18 @@ void launch_preprocess_typed(const BwdArgs& a, long long blocks, int Npad, long 
   const int n_order = a.dq_order ? a.seq.B * a.seq.H * (Npad / 128) : 0;
   const uint16_t* O = static_cast<const uint16_t*>(a.O);
   const uint16_t* dO = static_cast<const uint16_t*>(a.dO);
-  if (a.d == 64)
+  if (a.d <= 64)
     fa_bwd_preprocess_kernel<64, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, Npad, acc_vec4, a.dq_order, n_order);
+        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, a.d, Npad, acc_vec4, a.dq_order, n_order);
   else
     fa_bwd_preprocess_kernel<128, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, Npad, acc_vec4, a.dq_order, n_order);
+        O, dO, a.LSE, a.Dvec, a.lse2, a.dQacc, a.seq, a.d, Npad, acc_vec4, a.dq_order, n_order);
 }
 
 template <bool F16, bool DET>
 cudaError_t launch_bwd_tiles_typed(const BwdArgs& a, cudaStream_t stream) {
   const bool drop = a.drop_t != 0;
-  if (a.d == 64) {
+  if (a.d <= 64) {
     if (a.causal)
       return drop ? launch_bwd_main<64, true, true, F16, DET>(a, stream)
                   : launch_bwd_main<64, true, false, F16, DET>(a, stream);

@@ -166,11 +166,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   uint8_t* qsm = smem + L::kQ;
   for (int idx = tid; idx < kMaxRows * (D / 8); idx += kDecThreads) {
     const int r = idx / (D / 8), c8 = idx - r * (D / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);  // rows past R and padded columns stay zero
+    if (r < R && c8 * 8 < p.dh) {
       const int rr = r0 + r;
       const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
-      v = *reinterpret_cast<const uint4*>(p.Q + ((static_cast<size_t>(b) * p.H + h) * p.Nq + i) * D + c8 * 8);
+      v = *reinterpret_cast<const uint4*>(p.Q + ((static_cast<size_t>(b) * p.H + h) * p.Nq + i) * p.dh + c8 * 8);
     }
     *reinterpret_cast<uint4*>(qsm + (c8 / 8) * (kMaxRows * 128) + r * 128 + (((c8 % 8) ^ (r & 7)) << 4)) = v;
   }
@@ -419,11 +419,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         const float l = l_r[c];
         const float val = (l > 0.f) ? o[c] / l : 0.f;
         const float lse = (l > 0.f) ? (m_st[c] + lg2_approx(l)) * 0.69314718055994531f : -CUDART_INF_F;
-        if (dim < D) {
+        if (dim < p.dh) {
           if (p.splits == 1)
-            p.O[row * D + dim] = static_cast<uint16_t>(pack2<F16>(val, 0.f) & 0xFFFFu);
+            p.O[row * p.dh + dim] = static_cast<uint16_t>(pack2<F16>(val, 0.f) & 0xFFFFu);
           else
-            p.O_part[(row * p.splits + split) * D + dim] = val;
+            p.O_part[(row * p.splits + split) * p.dh + dim] = val;
         }
         if (dim == 0) {
           if (p.splits == 1)
@@ -447,7 +447,7 @@ template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_decode_merge_kernel(const float* __restrict__ O_part,
                                                               const float* __restrict__ LSE_part,
                                                               uint16_t* __restrict__ O, float* __restrict__ LSE,
-                                                              long long rows, int splits) {
+                                                              long long rows, int splits, int dh) {
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   for (long long row = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
@@ -466,16 +466,20 @@ __global__ void __launch_bounds__(256) fa_decode_merge_kernel(const float* __res
       for (int s = 0; s < splits; ++s) {
         const float w = __expf(ls[s] - mx);  // 0 for a split that saw nothing
         wsum += w;
-        const float* op = O_part + (row * splits + s) * D + lane * kPer;
+        const float* op = O_part + (row * splits + s) * dh + lane * kPer;
+        if (lane * kPer < dh) {
 #pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, op[e], acc[e]);
+          for (int e = 0; e < kPer; ++e) acc[e] = fmaf(w, op[e], acc[e]);
+        }
       }
     }
     const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+    if (lane * kPer < dh) {  // dh is a multiple of 32: a lane's columns are all in or all out
 #pragma unroll
-    for (int e = 0; e < kPer; e += 2) {
-      const uint32_t packed = pack2<F16>(acc[e] * inv, acc[e + 1] * inv);
-      *reinterpret_cast<uint32_t*>(O + row * D + lane * kPer + e) = packed;
+      for (int e = 0; e < kPer; e += 2) {
+        const uint32_t packed = pack2<F16>(acc[e] * inv, acc[e + 1] * inv);
+        *reinterpret_cast<uint32_t*>(O + row * dh + lane * kPer + e) = packed;
+      }
     }
     if (lane == 0) LSE[row] = (wsum > 0.f) ? mx + __logf(wsum) : -CUDART_INF_F;
   }
@@ -496,14 +500,14 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   long long blocks = (rows + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
   fa_decode_merge_kernel<D, F16><<<static_cast<int>(blocks), 256, 0, stream>>>(p.O_part, p.LSE_part, p.O, p.LSE,
-                                                                                rows, p.splits);
+                                                                                rows, p.splits, p.dh);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.d == 64) return a.f16 ? launch_decode_t<64, true>(a, stream) : launch_decode_t<64, false>(a, stream);
+  if (a.d <= 64) return a.f16 ? launch_decode_t<64, true>(a, stream) : launch_decode_t<64, false>(a, stream);
   return a.f16 ? launch_decode_t<128, true>(a, stream) : launch_decode_t<128, false>(a, stream);
 }
 

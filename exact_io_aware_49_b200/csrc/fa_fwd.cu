@@ -111,6 +111,7 @@ struct FwdParams {
   float* LSE;
   unsigned* err;
   SeqLayout seq;
+  int dh;  // head dimension of the tensors (D, or 32 / 96 padded to D = 64 / 128)
   float scale_log2;
   uint32_t drop_t;
   float drop_scale;
@@ -453,7 +454,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow_g);
 #pragma unroll
-          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+          for (int e = 0; e < D / 8; ++e)
+            if (e * 8 < p.dh) dst[e] = make_uint4(0u, 0u, 0u, 0u);
           *lse_g = -CUDART_INF_F;
         }
       } else if (ok && mbar_wait(&bar.o_ready[q], 0, abort_flag, p.err)) {
@@ -471,7 +473,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             packed[e] = pack2<F16>(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-          if (row_ok) {
+          if (row_ok && c * 32 < p.dh) {  // padded columns are not stored
             uint4* dst = reinterpret_cast<uint4*>(orow_g + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -501,6 +503,7 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   p.LSE = a.LSE;
   p.err = a.err;
   p.seq = a.seq;
+  p.dh = a.d;
   p.scale_log2 = a.scale_log2;
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
@@ -523,7 +526,7 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
 template <bool F16>
 cudaError_t launch_fwd_typed(const FwdArgs& a, cudaStream_t stream) {
   const bool drop = a.drop_t != 0;
-  if (a.d == 64) {
+  if (a.d <= 64) {
     if (a.causal)
       return drop ? launch_fwd_t<64, true, true, F16>(a, stream) : launch_fwd_t<64, true, false, F16>(a, stream);
     return drop ? launch_fwd_t<64, false, true, F16>(a, stream) : launch_fwd_t<64, false, false, F16>(a, stream);

@@ -124,6 +124,7 @@ struct DecodeParams {
   int rows;            // group * Nq query rows per key/value head
   int row_chunks;      // blocks of up to 16 rows
   int max_pages, page;
+  int dh;  // head dimension of the tensors (D, or 32 / 96 padded to D = 64 / 128)
   int splits, tiles_per_split;
   int causal;
   float scale_log2;

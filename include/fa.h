@@ -29,8 +29,10 @@
  *    statistics (LSE) are fp32 [B, H, N]; every sum inside the kernels is fp32.
  *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
  *    aligned.  The library allocates nothing and keeps no per-call state.
- *  - Supported: d in {64, 128}; any N >= 1 (a partial last 128-row tile is
- *    handled inside the kernels); B*H*N < 2^31.  Queries and keys may differ
+ *  - Supported: d in {32, 64, 96, 128} (32 and 96 run on the 64- and
+ *    128-column kernels: the columns past d are read as zeros and never
+ *    stored); any N >= 1 (a partial last 128-row tile is handled inside the
+ *    kernels); B*H*N < 2^31.  Queries and keys may differ
  *    in number (``_qk`` and ``_varlen`` entry points).
  *  - Causal mask with Nq queries and Nk keys: query i sits at key position
  *    i + Nk - Nq (bottom-right alignment; top-left when Nq = Nk) and sees the
@@ -69,7 +71,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, p_drop outside [0,1), ... */
-  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d not in {64,128}, B*H*N too large */
+  FA_ERR_UNSUPPORTED = 2,  /* valid but not implemented: d not in {32,64,96,128}, B*H*N too large */
   FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (launch, tensor-map encoding, ...) */
   FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by fa_last_device_error) */
 } fa_status;
@@ -311,7 +313,7 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
  *   causal      : nonzero -> query i of sequence b is position
  *                 seqlens_k[b] - Nq + i and sees positions up to it
  *   max_seqlen_k: the largest seqlens_k entry (sizes the launch)
- *   page_size   : 16, 32, 64 or 128; d in {64, 128}; no dropout
+ *   page_size   : 16, 32, 64 or 128; d in {32, 64, 96, 128}; no dropout
  *   num_splits  : how many parts each sequence's positions are cut into
  *                 (each a thread block, merged by log-sum-exp); 0 chooses
  *                 fa_decode_num_splits(); with more than one split the call

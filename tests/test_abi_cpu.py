@@ -63,7 +63,7 @@ def _fwd(lib, Q=A, K=A, V=A, O=A, L=A, B=1, H=1, N=128, d=64, causal=0, scale=0.
     (dict(B=0), 1), (dict(H=-1), 1), (dict(N=0), 1), (dict(d=0), 1),
     (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
     (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("inf")), 1),
-    (dict(d=32), 2), (dict(d=96), 2),
+    (dict(d=48), 2), (dict(d=80), 2), (dict(d=256), 2),
     (dict(B=1 << 16, H=1 << 8, N=1 << 7), 2),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, want):
@@ -109,12 +109,12 @@ def test_ex_entry_points_reject_unknown_dtype(lib, dtype):
 def test_ex_entry_points_validate_like_the_plain_ones(lib, dtype):
     ws_ok = lib.fa_bwd_workspace_size(1, 1, 128, 64)
     assert lib.fa_fwd_ex(0, A, A, A, A, 1, 1, 128, 64, 0, 0.125, 0.0, 0, dtype, None) == 1
-    assert lib.fa_fwd_ex(A, A, A, A, A, 1, 1, 128, 96, 0, 0.125, 0.0, 0, dtype, None) == 2
+    assert lib.fa_fwd_ex(A, A, A, A, A, 1, 1, 128, 80, 0, 0.125, 0.0, 0, dtype, None) == 2
     assert lib.fa_fwd_ex(A, A, A, A + 8, A, 1, 1, 128, 64, 0, 0.125, 0.0, 0, dtype, None) == 1
     assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 1.0, 0, dtype, A, ws_ok, None) == 1
     assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 0.0, 0, dtype, A, ws_ok - 4,
                          None) == 1
-    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 32, 1, 0.125, 0.0, 0, dtype, A, ws_ok, None) == 2
+    assert lib.fa_bwd_ex(A, A, A, A, A, A, A, A, A, 1, 1, 128, 48, 1, 0.125, 0.0, 0, dtype, A, ws_ok, None) == 2
 
 
 def _varlen_fwd(lib, cu_q=A, cu_k=A, B=1, H=1, tq=64, tk=64, mq=64, mk=64, d=64, scale=0.125, p=0.0, dtype=0):
@@ -123,7 +123,7 @@ def _varlen_fwd(lib, cu_q=A, cu_k=A, B=1, H=1, tq=64, tk=64, mq=64, mk=64, d=64,
 
 @pytest.mark.parametrize("kw,want", [
     (dict(cu_q=0), 1), (dict(cu_k=0), 1), (dict(cu_q=A + 2), 1), (dict(B=0), 1), (dict(tq=0), 1),
-    (dict(mq=65), 1), (dict(mk=0), 1), (dict(p=1.0), 1), (dict(dtype=3), 1), (dict(d=96), 2),
+    (dict(mq=65), 1), (dict(mk=0), 1), (dict(p=1.0), 1), (dict(dtype=3), 1), (dict(d=80), 2),
     (dict(H=1 << 12, tq=1 << 19, tk=1 << 19, mq=1 << 10, mk=1 << 10), 2),
 ])
 def test_varlen_rejects_bad_arguments(lib, kw, want):
@@ -147,7 +147,7 @@ def test_varlen_workspace_size(lib):
 
 def test_qk_entry_points_validate(lib):
     assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 0, 64, 1, 0.125, 0.0, 0, 0, None) == 1
-    assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 256, 96, 1, 0.125, 0.0, 0, 0, None) == 2
+    assert lib.fa_fwd_qk(A, A, A, A, A, 1, 1, 128, 256, 80, 1, 0.125, 0.0, 0, 0, None) == 2
     ws = lib.fa_bwd_qk_workspace_size(1, 1, 128, 64, 0)
     assert ws == lib.fa_bwd_workspace_size(1, 1, 128, 64)
     assert lib.fa_bwd_qk_workspace_size(2, 3, 1000, 64, 1) == lib.fa_bwd_workspace_size(2, 3, 1000, 64) + 256
@@ -163,7 +163,7 @@ def test_stage_entry_points_reject_bad_arguments(lib):
     assert lib.fa_bwd_prepare(A, A, A, 1, 1, 128, 48, A, ws_ok, None) == 2
     assert lib.fa_bwd_tiles(A, A, A, A, A, 0, 1, 1, 128, 64, 1, 0.125, 0.0, 0, A, ws_ok, None) == 1
     assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, 64, 1, 0.125, 1.0, 0, A, ws_ok, None) == 1
-    assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, 96, 1, 0.125, 0.0, 0, A, ws_ok, None) == 2
+    assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, 80, 1, 0.125, 0.0, 0, A, ws_ok, None) == 2
     assert lib.fa_bwd_finish(A + 8, 1, 1, 128, 64, 0.125, A, ws_ok, None) == 1
     assert lib.fa_bwd_finish(A, 1, 1, 128, 64, 0.125, A + 64, ws_ok, None) == 1
     assert lib.fa_bwd_finish(A, 1, 1, 128, 64, -1.0, A, ws_ok, None) == 1
@@ -196,7 +196,7 @@ def _decode(lib, Q=A, BT=A, SL=A, B=2, H=8, H_kv=2, Nq=1, d=128, pages=64, page=
 @pytest.mark.parametrize("kw,want", [
     (dict(Q=0), 1), (dict(BT=0), 1), (dict(SL=A + 2), 1), (dict(H=6, H_kv=4), 1), (dict(maxk=129), 1),
     (dict(scale=0.0), 1), (dict(dtype=5), 1), (dict(splits=-1), 1), (dict(splits=3), 1),  # no workspace
-    (dict(page=8, maxp=16), 2), (dict(page=48), 2), (dict(d=96), 2), (dict(Nq=0), 1),
+    (dict(page=8, maxp=16), 2), (dict(page=48), 2), (dict(d=80), 2), (dict(Nq=0), 1),
 ])
 def test_decode_rejects_bad_arguments(lib, kw, want):
     assert _decode(lib, **kw) == want
