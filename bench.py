@@ -22,6 +22,12 @@ FLOPs per step: forward 4*B*H*N^2*d/2 (causal), backward 2.5x the forward.
             attention problem)
 
 ``--impl reference`` times that oracle instead (rank 0 only).
+
+``--decode`` prints a different line instead: the paged-cache decode kernel
+(fa_decode_paged) on 16 sequences x 32768 cached positions, 32 query / 8
+key-value heads, d=128, one query per sequence, pages of 64 positions in
+shuffled order; value = bytes of K and V read per call / call time (GB/s),
+roofline against the measured HBM copy bandwidth.
 Multi-GPU (torchrun): every rank runs the full workload on its own GPU -- the
 (b, h) units are independent, so there is no collective on the data path;
 ``scaling`` is "weak" and value sums the ranks' work over the slowest rank.
@@ -55,6 +61,8 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TILES_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_bwd.cu")
 FWD_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_fwd.cu")
+DECODE_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_decode.cu")
+DECODE_WORKLOAD = "decode_paged_B16_L32768_H32_Hkv8_d128"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
 
@@ -73,13 +81,13 @@ def _sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def _traffic(kernel, source):
+def _traffic(kernel, source, workload=WORKLOAD):
     """DRAM bytes per launch from the committed ncu summary, if taken on this exact source."""
     try:
         with open(TRAFFIC_FILE) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) >= 4 and parts[0] == kernel and parts[1] == WORKLOAD and parts[2] == _sha(source):
+                if len(parts) >= 4 and parts[0] == kernel and parts[1] == workload and parts[2] == _sha(source):
                     return float(parts[3])
     except OSError:
         pass
@@ -330,6 +338,111 @@ def run_ours(args, w, world, device):
     return out, (qh, kh, vh, doh)
 
 
+# --------------------------------------------------------------------- decode line
+
+DECODE = dict(B=16, H=32, H_kv=8, Nq=1, d=128, L=32768, page=64, seed=7)
+
+
+def run_decode(args, device):
+    """Paged-cache decode: HBM GB/s of the cached K and V per call (one GPU)."""
+    from exact_io_aware_49_b200 import binding
+    c = DECODE
+    B, H, H_kv, Nq, d, L, page = c["B"], c["H"], c["H_kv"], c["Nq"], c["d"], c["L"], c["page"]
+    gen = torch.Generator(device="cpu").manual_seed(c["seed"])
+    n_pages = B * ((L + page - 1) // page)
+    kc = torch.randn(n_pages, page, H_kv, d, generator=gen, dtype=torch.float32).to(torch.bfloat16).to(device)
+    vc = torch.randn(n_pages, page, H_kv, d, generator=gen, dtype=torch.float32).to(torch.bfloat16).to(device)
+    table = torch.randperm(n_pages, generator=gen).to(torch.int32).view(B, -1).to(device)
+    lens = torch.full((B,), L, dtype=torch.int32, device=device)
+    qh = torch.randn(B, H, Nq, d, generator=gen, dtype=torch.float32).to(torch.bfloat16).pin_memory()
+    q = qh.to(device)
+    lib = binding.load_library()
+    splits = int(lib.fa_decode_num_splits(B, H_kv, H, Nq, L))
+    ws = torch.empty(max(1, int(lib.fa_decode_workspace_size(B, H, Nq, d, splits))), dtype=torch.uint8,
+                     device=device)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, Nq, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def call(qq):
+        return binding.fa_decode_paged(qq, kc, vc, table, lens, L, True, d ** -0.5, num_splits=splits, out=o,
+                                       lse=lse, workspace=ws)
+
+    for _ in range(args.warmup):
+        call(q)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(device)
+    time.sleep(0.6)
+    sampler.start()
+    evs = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call(q)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    kv_bytes = 2 * B * L * H_kv * d * 2
+    io_bytes = kv_bytes + 2 * q.numel() * 2 + lse.numel() * 4
+    # end to end through the public API: the step's query in, output and LSE out
+    oh = torch.empty_like(qh).pin_memory()
+    lseh = torch.empty(B, H, Nq, dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        q.copy_(qh, non_blocking=True)
+        call(q)
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        q.copy_(qh, non_blocking=True)
+        call(q)
+        oh.copy_(o, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = a.elapsed_time(b) / args.steps
+    if binding.fa_last_device_error() != 0:
+        raise RuntimeError("a bounded device wait timed out during the decode benchmark")
+    peaks, peak_src = _peaks()
+    achieved = io_bytes / (ms * 1e-3) / 1e9
+    # oracle on a bounded sample: one sequence, the 4 query heads of one key/value head
+    from oracle import paged
+    qs = qh[:1, :4].to(torch.float64).numpy()
+    pages0 = table[0].long()
+    kcs = kc[pages0][:, :, :1].to(torch.float64).cpu().numpy()  # sequence 0's pages, key/value head 0
+    vcs = vc[pages0][:, :, :1].to(torch.float64).cpu().numpy()
+    tab = np.arange(kcs.shape[0], dtype=np.int32)[None]
+    t0 = time.time()
+    n_rep = 0
+    while time.time() - t0 < 10.0:
+        paged.decode_forward(qs, kcs, vcs, tab, np.array([L]), causal=True, scale=d ** -0.5)
+        n_rep += 1
+    cpu_s = (time.time() - t0) / n_rep
+    cpu_bytes = 2 * L * 1 * d * 2
+    return {
+        "metric": "paged-cache decode attention: K/V bytes read per second (bf16)", "value": kv_bytes / (ms * 1e-3) / 1e9,
+        "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded randn, bf16; pages in shuffled order)",
+        "config": {"workload": DECODE_WORKLOAD, **{k: v for k, v in c.items() if k != "seed"},
+                   "causal": True, "num_splits": splits,
+                   "l2": "no flush: the K/V cache is 2.1 GB, larger than the 126 MB L2"},
+        "roofline": {"bound": "hbm", "kernel": "fa_decode_kernel (+ split merge)", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "peak_kind": f"hbm_gbs ({peak_src})", "algorithmic_bytes": io_bytes,
+                     "traffic": _traffic("fa_decode", DECODE_SOURCE, DECODE_WORKLOAD)},
+        "e2e": {"value": kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": qh.numel() * 2, "d2h_bytes_per_step": oh.numel() * 2 + lseh.numel() * 4},
+        "gpu_launches": args.steps * (2 if splits > 1 else 1),
+        "clocks": clocks,
+        "cpu_baseline": {"value": cpu_bytes / cpu_s / 1e9, "unit": "GB/s", "cores": _CORES, "kind": "oracle",
+                         "sample": f"fp64 NumPy paged oracle, 1 sequence x 4 query heads of one key/value head, "
+                                   f"{L} positions, {n_rep} runs in {time.time() - t0:.1f} s"},
+    }
+
+
 # --------------------------------------------------------------------- plumbing
 
 def _world():
@@ -360,9 +473,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true", help="the paged-cache decode line instead (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.decode:
+        print(json.dumps(run_decode(args, torch.device("cuda", 0))), flush=True)
+        return
     w = wl.BY_NAME[args.workload]
     world = _world()
     if world["size"] > 1:
