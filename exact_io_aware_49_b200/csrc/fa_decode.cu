@@ -201,9 +201,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         const int st = it % S;
         const int first = (t_begin + it) * kTileKeys;
         const int pages_here = min(kTileKeys / p.page, (Lk - first + p.page - 1) / p.page);
+        // read the tile's page ids first: the copies below are ordered after
+        // every earlier memory access, so interleaving would serialise the reads
+        constexpr int kMaxPagesPerTile = kTileKeys / 16;
+        int pids[kMaxPagesPerTile];
+        const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages + first / p.page;
+#pragma unroll
+        for (int pg = 0; pg < kMaxPagesPerTile; ++pg) pids[pg] = (pg < pages_here) ? bt[pg] : 0;
         mbar_expect_tx(&full[st], static_cast<uint32_t>(pages_here * 2 * (D / 64) * p.page * 128));
-        for (int pg = 0; pg < pages_here; ++pg) {
-          const int pid = p.block_table[static_cast<size_t>(b) * p.max_pages + first / p.page + pg];
+#pragma unroll
+        for (int pg = 0; pg < kMaxPagesPerTile; ++pg) {
+          if (pg >= pages_here) break;
+          const int pid = pids[pg];
           for (int c = 0; c < D / 64; ++c) {
             // an out-of-range page id reads zeros (outside the tensor map)
             uint8_t* kd = smem + st * L::kStage + c * L::kBox + pg * p.page * 128;
@@ -281,6 +290,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       l_r[c] = 0.f;
     }
     const int col = scatter_col(lane);
+    // last visible position of each row: the cached length, and under the
+    // causal mask the row's own position Lk - Nq + i; rows past R see nothing
+    int lim[kMaxRows];
+#pragma unroll
+    for (int c = 0; c < kMaxRows; ++c) {
+      const int i = (r0 + c) % p.Nq;
+      lim[c] = (c >= R) ? -1 : (p.causal ? min(Lk - 1, Lk - p.Nq + i) : Lk - 1);
+    }
     // Every wait below is bounded and may end differently in different
     // threads; the named barriers AND the outcomes, so the 128 threads leave
     // the loop together and tensor-memory instructions only run when all
@@ -309,11 +326,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       reg_fence16(sr);
       float s[16];
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) {
-        const int i = (r0 + c) % p.Nq;
-        const bool visible = c < R && pos < Lk && (!p.causal || pos <= Lk - p.Nq + i);
-        s[c] = visible ? __uint_as_float(sr[c]) * p.scale_log2 : -CUDART_INF_F;
-      }
+      for (int c = 0; c < kMaxRows; ++c) s[c] = (pos <= lim[c]) ? __uint_as_float(sr[c]) * p.scale_log2 : -CUDART_INF_F;
       // tile max per row: reduce over this warp's keys, then over the 4 warps
       float* rmax = red + ((it & 1) * 2 + 0) * kMaxRows * 4;
       float* rsum = red + ((it & 1) * 2 + 1) * kMaxRows * 4;
