@@ -68,9 +68,9 @@ struct DecSmem {
   static constexpr int kPBytes = kMaxRows * kTileKeys * 2;
   static constexpr int kRed = kP + 2 * kPBytes;  // fp32 [2 parities][max, sum][16 rows][4 warps]
   static constexpr int kBar = kRed + 2 * 2 * kMaxRows * 4 * 4;
-  // full[kStages], s_ready[2], p_ready[2], pv_done[2], drain (the pairs by tile parity: a
-  // role may run one tile ahead of the role that waits, never two)
-  static constexpr int kNumBars = kStages + 7;
+  // kfull[kStages], vfull[kStages], s_ready[2], p_ready[2], pv_done[2], drain (the pairs by
+  // tile parity: a role may run one tile ahead of the role that waits, never two)
+  static constexpr int kNumBars = 2 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kUsed = kMisc + 16;
 };
@@ -127,8 +127,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (!smem_layout_fits(smem_raw, smem, L::kUsed, p.err)) return;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* s_ready = full + S;  // [2], by tile parity
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + L::kBar);  // K of a stage landed
+  uint64_t* vfull = kfull + S;                                      // V of a stage landed
+  uint64_t* s_ready = vfull + S;  // [2], by tile parity
   uint64_t* p_ready = s_ready + 2;  // [2], by tile parity
   uint64_t* pv_done = p_ready + 2;  // [2], by tile parity
   uint64_t* drain = pv_done + 2;
@@ -150,7 +151,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   const int n = max(0, min(n_tiles, t_begin + p.tiles_per_split) - t_begin);  // tiles of this split
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&vfull[s], 1);
+    }
     mbar_init(&s_ready[0], 1);
     mbar_init(&s_ready[1], 1);
     mbar_init(&p_ready[0], 4);
@@ -208,7 +212,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages + first / p.page;
 #pragma unroll
         for (int pg = 0; pg < kMaxPagesPerTile; ++pg) pids[pg] = (pg < pages_here) ? bt[pg] : 0;
-        mbar_expect_tx(&full[st], static_cast<uint32_t>(pages_here * 2 * (D / 64) * p.page * 128));
+        // K and V complete separately: S^T needs only K, so it starts while V is still arriving
+        mbar_expect_tx(&kfull[st], static_cast<uint32_t>(pages_here * (D / 64) * p.page * 128));
+        mbar_expect_tx(&vfull[st], static_cast<uint32_t>(pages_here * (D / 64) * p.page * 128));
 #pragma unroll
         for (int pg = 0; pg < kMaxPagesPerTile; ++pg) {
           if (pg >= pages_here) break;
@@ -216,8 +222,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
           for (int c = 0; c < D / 64; ++c) {
             // an out-of-range page id reads zeros (outside the tensor map)
             uint8_t* kd = smem + st * L::kStage + c * L::kBox + pg * p.page * 128;
-            tma_load_3d(kd, &tmK, c * 64, g, pid * p.page, &full[st]);
-            tma_load_3d(kd + L::kKBytes, &tmV, c * 64, g, pid * p.page, &full[st]);
+            tma_load_3d(kd, &tmK, c * 64, g, pid * p.page, &kfull[st]);
+            tma_load_3d(kd + L::kKBytes, &tmV, c * 64, g, pid * p.page, &vfull[st]);
           }
         }
       };
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       // S^T = K Q^T of tile it into its TMEM buffer: M = 128 keys, N = 16 rows, K = D (both K-major)
       auto issue_s = [&](int it) -> bool {
         const int st = it % S;
-        if (!mbar_wait(&full[st], (it / S) & 1, abort_flag, p.err)) return false;
+        if (!mbar_wait(&kfull[st], (it / S) & 1, abort_flag, p.err)) return false;
         consumed = it + 1;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + st * L::kStage);
@@ -259,7 +265,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
           issue(issued);
           ++issued;
         }
-        if (!mbar_wait(&p_ready[it & 1], (it >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!mbar_wait(&p_ready[it & 1], (it >> 1) & 1, abort_flag, p.err) ||
+            !mbar_wait(&vfull[it % S], (it / S) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         // O^T += V^T P^T: M = 128 dimensions (V read MN-major), N = 16 rows, K = 128 keys
         const uint32_t v_addr = smem_u32(smem + (it % S) * L::kStage) + L::kKBytes;
@@ -276,7 +286,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         // copies and products in flight finish before shared and tensor memory go away
         mma_commit(drain);
         mbar_wait_drain(drain, 0);
-        for (int it2 = consumed; it2 < issued; ++it2) mbar_wait_drain(&full[it2 % S], (it2 / S) & 1);
+        for (int it2 = consumed; it2 < issued; ++it2) mbar_wait_drain(&kfull[it2 % S], (it2 / S) & 1);
+        for (int it2 = max(0, consumed - 1); it2 < issued; ++it2) mbar_wait_drain(&vfull[it2 % S], (it2 / S) & 1);
       }
     }
     __syncwarp();
@@ -310,16 +321,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       ok = named_bar_and(1, 128, mbar_wait(&s_ready[it & 1], (it >> 1) & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
-      // S^T is done, so the tile's copies have landed.  V rows of positions
-      // past the sequence (or of pages not loaded) may hold anything, NaN
-      // included, and 0 * NaN would reach O through the tensor core: zero them.
-      if (pos >= Lk) {
-        uint8_t* vrow = smem + (it % S) * L::kStage + L::kKBytes + j * 128;
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-          for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4*>(vrow + c * L::kBox + q * 16) = make_uint4(0u, 0u, 0u, 0u);
-      }
       uint32_t sr[16];
       tmem_ld16(tmem + (it & 1) * 16 + lane_base, sr);
       tmem_ld_wait();
@@ -337,9 +338,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         const float wm = warp_reduce_scatter16<true>(v, lane);
         if (!(lane & 1)) rmax[col * 4 + warp] = wm;
       }
+      // V rows of positions past the sequence (or of pages not loaded) may
+      // hold anything, NaN included, and 0 * NaN would reach O through the
+      // tensor core: once the tile's V has landed, zero them
+      bool v_ok = true;
+      if (first + kTileKeys > Lk) {
+        v_ok = mbar_wait(&vfull[it % S], (it / S) & 1, abort_flag, p.err);
+        if (v_ok && pos >= Lk) {
+          uint8_t* vrow = smem + (it % S) * L::kStage + L::kKBytes + j * 128;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(vrow + c * L::kBox + q * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       // (this barrier also covers the P buffer: the product of tile it - 2 has read it)
       const bool p_free = (it < 2) || mbar_wait(&pv_done[it & 1], ((it - 2) >> 1) & 1, abort_flag, p.err);
-      ok = named_bar_and(1, 128, p_free);
+      ok = named_bar_and(1, 128, p_free && v_ok);
       if (!ok) break;
       float alpha[kMaxRows];
       bool rescale = false;  // the same in every thread: computed from the same shared values
