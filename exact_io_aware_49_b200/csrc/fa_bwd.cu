@@ -14,9 +14,10 @@
 // Three kernels:
 //   1. preprocess: D_i = rowsum(dO * O) (fp32, from the stored 16-bit O),
 //      LSE2_i = LSE_i * log2(e), and zeroing of the fp32 dQ accumulator;
-//   2. main: one CTA per (b, h, 128-key tile j) keeps K_j, V_j in shared
-//      memory and dK_j, dV_j in tensor memory while it streams the query
-//      tiles i (i >= j when causal) through a two-stage TMA ring.  Per tile:
+//   2. main: one CTA per (sequence-or-batch entry, head, 128-key tile j)
+//      keeps K_j, V_j in shared memory and dK_j, dV_j in tensor memory while
+//      it streams the query tiles i that see a key of tile j (causal: query
+//      position i + Nk - Nq >= j) through a two-stage TMA ring.  Per tile:
 //        S^T = K_j Q_i^T and dP^T = V_j dO_i^T  (tcgen05, M = 128 keys)
 //        P^T = exp2(S^T scale log2e - LSE2_i), masked, dropout-masked
 //              -> written in the input type into TMEM over S^T
@@ -38,7 +39,9 @@
 //      MMAs; warp 9 issues TMA; warpgroup 3 drains dQ.
 //   3. convert: dQ = scale * dQacc, rounded to the input type.
 // Inputs and outputs are all bf16 or all fp16 (the F16 template flag); every
-// accumulation is fp32.
+// accumulation is fp32.  Each unit's rows come from a SeqLayout (fixed
+// [B, H, N, d] or packed variable-length [total, H, d], Nq and Nk may differ);
+// head dimensions 32 / 96 run on D = 64 / 128 with zero-filled columns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>

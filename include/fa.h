@@ -22,11 +22,14 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Tensors are dense, row-major [B, H, N, d] (strides H*N*d, N*d, d, 1) with
- *    16-bit elements passed as void*: bfloat16 for the plain entry points;
+ *  - Tensors are dense, row-major [B, H, N, d] (strides H*N*d, N*d, d, 1) --
+ *    except for the packed ``_varlen`` calls ([total, H, d]) and the paged
+ *    decode cache ([num_pages, page_size, H_kv, d]) -- with 16-bit elements
+ *    passed as void*: bfloat16 for fa_fwd / fa_bwd and their stages;
  *    bfloat16 or IEEE fp16 (binary16), as the ``dtype`` argument says, for
- *    the ``_ex`` ones.  All tensors of one call share the type.  Per-row
- *    statistics (LSE) are fp32 [B, H, N]; every sum inside the kernels is fp32.
+ *    every call that takes one.  All tensors of one call share the type.
+ *    Per-row statistics (LSE) are fp32 [B, H, N]; every sum inside the
+ *    kernels is fp32.
  *  - Every pointer argument is DEVICE memory owned by the caller, 16-byte
  *    aligned.  The library allocates nothing and keeps no per-call state.
  *  - Supported: d in {32, 64, 96, 128} (32 and 96 run on the 64- and
