@@ -167,24 +167,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
 
-// 2-D tiled load of one box into shared memory; completion is signalled on
-// ``bar`` as transaction bytes.  x = innermost coordinate (elements), y = row.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// 2-D tiled reduce-add of one shared-memory box into global memory (fp32 add,
-// element-wise atomic in L2).  x = innermost coordinate (elements), y = row.
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, const void* src, int x, int y) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(tm)),
-               "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until the shared-memory sources of all committed bulk groups have been read.
 __device__ __forceinline__ void bulk_wait_group_read0() {
@@ -198,12 +180,6 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
-// Four fp32 reductions into consecutive global words (16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
 
@@ -291,9 +267,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
 __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, bool a_mn_major, bool b_mn_major, bool f16) {
   return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
-  return idesc_f32acc(M, N, a_mn_major, b_mn_major, false);
 }
 
 // TMEM loads/stores, 32 lanes x 32 bits, 32 consecutive columns per thread.
@@ -392,13 +365,6 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
-// bf16x2 from two floats, round-to-nearest-even; ``lo`` lands in the low half.
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
 // 16-bit pairs of the kernels' element type (fp16 when F16, else bf16),
 // round-to-nearest-even; ``lo`` lands in the low half.
 template <bool F16>
@@ -431,13 +397,6 @@ __device__ __forceinline__ float2 unpack2(uint32_t v) {
     r.x = __uint_as_float(v << 16);
     r.y = __uint_as_float(v & 0xFFFF0000u);
   }
-  return r;
-}
-
-// bf16x2 of (max(lo, 0), max(hi, 0)), round-to-nearest-even.
-__device__ __forceinline__ uint32_t pack_bf16x2_relu(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.relu.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 
