@@ -470,14 +470,33 @@ int fa_decode_num_splits(int B, int H_kv, int H, int Nq, int max_seqlen_k) {
   const long long chunks = (rows + fa::decode_rows_per_cta() - 1) / fa::decode_rows_per_cta();
   const long long ctas = static_cast<long long>(B) * H_kv * chunks;
   const int tiles = (max_seqlen_k + fa::decode_keys_per_tile() - 1) / fa::decode_keys_per_tile();
-  // about two waves of CTAs on 148 SMs, at least one tile per split
-  long long splits = (2 * 148 + ctas - 1) / ctas;
-  if (splits > tiles) splits = tiles;
-  if (splits > 128) splits = 128;
-  if (splits < 1) splits = 1;
-  // no split without a tile: recompute from the tiles per split
-  const int per = static_cast<int>((tiles + splits - 1) / splits);
-  return (tiles + per - 1) / per;
+  // SMs of the current device (148 on B200; also the answer without a device)
+  static int sms = 0;
+  if (sms <= 0) {
+    int dev = 0, n = 0;
+    sms = (cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+              ? n
+              : 148;
+  }
+  // One CTA per SM, each streaming its tiles at about the same rate, plus a
+  // fixed cost per CTA (start-up, pipeline fill) worth about 4 tiles, and as
+  // much again for the merge launch when split: estimated time = waves x
+  // (tiles per CTA + 4) (+ 4).  Take the cheapest count, the fewest splits
+  // among equals.
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= 128 && s <= tiles; ++s) {
+    const int per = (tiles + s - 1) / s;
+    if ((tiles + per - 1) / per != s) continue;  // no split without a tile
+    const long long waves = (ctas * s + sms - 1) / sms;
+    const long long cost = waves * (per + 4) + (s > 1 ? 4 : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Nq, int d, int num_splits) {

@@ -210,4 +210,12 @@ def test_decode_split_choice_and_workspace(lib):
     assert lib.fa_decode_num_splits(1, 1, 1, 1, 100) == 1  # a single 128-key tile cannot be split
     assert lib.fa_decode_num_splits(1, 3, 4, 1, 100) == 0  # H not a multiple of H_kv
     assert lib.fa_decode_workspace_size(2, 8, 1, 128, 1) == 0
+    # every split holds at least one 128-position tile, whatever the shape
+    for B, H_kv, H, Nq, L in [(16, 8, 32, 1, 32768), (1, 8, 32, 1, 131072), (4, 8, 32, 4, 32768),
+                              (3, 2, 8, 1, 1000), (1, 1, 1, 1, 129), (2, 1, 64, 16, 70000), (500, 8, 8, 1, 300)]:
+        tiles = (L + 127) // 128
+        s = lib.fa_decode_num_splits(B, H_kv, H, Nq, L)
+        assert 1 <= s <= min(tiles, 128)
+        per = (tiles + s - 1) // s
+        assert (tiles + per - 1) // per == s, (B, H_kv, H, Nq, L, s)
     assert lib.fa_decode_workspace_size(2, 8, 1, 128, 4) == 2 * 8 * 4 * 128 * 4 + 256
