@@ -470,15 +470,15 @@ int fa_decode_num_splits(int B, int H_kv, int H, int Nq, int max_seqlen_k) {
   const long long chunks = (rows + fa::decode_rows_per_cta() - 1) / fa::decode_rows_per_cta();
   const long long ctas = static_cast<long long>(B) * H_kv * chunks;
   const int tiles = (max_seqlen_k + fa::decode_keys_per_tile() - 1) / fa::decode_keys_per_tile();
-  // SMs of the current device (148 on B200; also the answer without a device)
-  static int sms = 0;
-  if (sms <= 0) {
+  // SMs of the device current at the first call (148 on B200; also the answer
+  // without a device); a function-local static is initialised once, thread-safely
+  static const int sms = [] {
     int dev = 0, n = 0;
-    sms = (cudaGetDevice(&dev) == cudaSuccess &&
-           cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-              ? n
-              : 148;
-  }
+    return (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+               ? n
+               : 148;
+  }();
   // One CTA per SM, each streaming its tiles at about the same rate, plus a
   // fixed cost per CTA (start-up, pipeline fill) worth about 4 tiles, and as
   // much again for the merge launch when split: estimated time = waves x

@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int k = 0; k < kCols / 32; ++k) reg_fence32(v + 32 * k);
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        if (r > 0) asm volatile("bar.sync 2, 128;" ::: "memory");  // round 0's reduce has read the buffer
+        if (r > 0) asm volatile("bar.sync 2, 128;" ::: "memory");  // the first pass's reduce has read the buffer
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx)
 #pragma unroll
