@@ -29,8 +29,9 @@ Pins (tests/test_oracle_*.py, tests/test_philox_oracle.py): rows of P sum to
 one; Q = 0 closed forms; a hand-derived two-token example under
 tests/golden/; online recurrence == two-pass; gradients against central
 finite differences; shift / permutation / N = 1 / p = 0 invariants; Philox
-against an independent library implementation (ATen's header-only
-``philox_engine``) plus keep-rate and lag-1 correlation statistics.  No
+against its authors' published known-answer vectors (tests/golden/) and an
+independent library implementation (ATen's header-only ``philox_engine``),
+plus keep-rate and lag-1 correlation statistics.  No
 function here is "parity unpinned".
 """
 

@@ -110,6 +110,36 @@ def test_missing_philox_key_bump_is_caught_by_library_cross_check():
     assert mutant(1, 2, 3, 4, 5, 6) != ref
 
 
+@pytest.mark.parametrize("slip", ["none", "no_key_bump", "swapped_multipliers", "nine_rounds"])
+def test_philox_slips_fail_the_known_answer_vectors(slip):
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "philox4x32_10_kat.txt")
+    rows = []
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            lhs, rhs = line.split("->")
+            rows.append(([int(x, 16) for x in lhs.split()], [int(x, 16) for x in rhs.split()]))
+    m0, m1 = philox.PHILOX_M0, philox.PHILOX_M1
+    if slip == "swapped_multipliers":
+        m0, m1 = m1, m0
+    rounds = 9 if slip == "nine_rounds" else 10
+    bump = slip != "no_key_bump"
+
+    def mutant(c0, c1, c2, c3, k0, k1):
+        m32 = 0xFFFFFFFF
+        for r in range(rounds):
+            if r and bump:
+                k0, k1 = (k0 + 0x9E3779B9) & m32, (k1 + 0xBB67AE85) & m32
+            p0, p1 = c0 * m0, c2 * m1
+            c0, c1, c2, c3 = ((p1 >> 32) ^ c1 ^ k0) & m32, p1 & m32, ((p0 >> 32) ^ c3 ^ k1) & m32, p0 & m32
+        return [c0, c1, c2, c3]
+
+    if slip == "none":  # the restatement itself reproduces the vectors, so each mutant differs only by its slip
+        assert all(mutant(*ins) == want for ins, want in rows)
+    else:
+        assert any(mutant(*ins) != want for ins, want in rows)
+
+
 def test_keep_tie_break_at_threshold():
     """u16 == t is kept (keep <=> u16 >= t): find such draws and check them."""
     t = philox.keep_threshold(0.1)

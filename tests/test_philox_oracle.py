@@ -1,5 +1,7 @@
 """Pins for the oracle's Philox4x32-10 and dropout keep mask (CPU only).
 
+* the published known-answer vectors of Philox4x32-10
+  (``tests/golden/philox4x32_10_kat.txt``, cited there);
 * bit-exact agreement with an independent implementation: ATen's header-only
   ``philox_engine`` compiled with g++ from the installed torch headers;
 * the (i, j) -> output word / half mapping restated here against that engine;
@@ -39,6 +41,25 @@ def aten_philox():
 def _counters(rng, n):
     return [(int(rng.integers(0, 2**64, dtype=np.uint64)),) + tuple(int(x) for x in rng.integers(0, 2**32, size=4))
             for _ in range(n)]
+
+
+def _kat():
+    rows = []
+    with open(os.path.join(HERE, "golden", "philox4x32_10_kat.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            lhs, rhs = line.split("->")
+            rows.append(([int(x, 16) for x in lhs.split()], [int(x, 16) for x in rhs.split()]))
+    return rows
+
+
+def test_philox_known_answer_vectors():
+    rows = _kat()
+    assert len(rows) == 3
+    for (c0, c1, c2, c3, k0, k1), want in rows:
+        out = philox.philox4x32(*(np.array([x], dtype=np.uint64) for x in (c0, c1, c2, c3, k0, k1)))
+        assert [int(np.asarray(r).ravel()[0]) for r in out] == want
 
 
 def test_philox_matches_aten_engine(aten_philox):
