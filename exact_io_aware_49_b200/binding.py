@@ -87,13 +87,25 @@ def _stream(t):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
+def _guard(t):
+    """Makes ``t``'s device the current one for the call: the library sets kernel
+    attributes and launches on the current device."""
+    return torch.cuda.device(t.device)
+
+
 # element types of the ``_ex`` entry points (fa_dtype)
 FA_DTYPE = {torch.bfloat16: 0, torch.float16: 1}
 
 
-def _check_bhnd(name, t, shape=None, dtype=None):
+def _check_device(name, t, device):
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} like q")
+
+
+def _check_bhnd(name, t, shape=None, dtype=None, device=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    _check_device(name, t, device)
     if t.dtype not in FA_DTYPE:
         raise ValueError(f"{name} must be bf16 or fp16")
     if dtype is not None and t.dtype != dtype:
@@ -102,6 +114,22 @@ def _check_bhnd(name, t, shape=None, dtype=None):
         raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _check_f32(name, t, shape, device):
+    if not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor of shape {tuple(shape)}")
+    _check_device(name, t, device)
+
+
+def _ws_args(workspace, device):
+    """(pointer, bytes) of a caller's workspace (None -> (None, 0))."""
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check_device("workspace", workspace, device)
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
 
 
 def _raise(st, what):
@@ -116,23 +144,26 @@ def fa_fwd(q, k, v, causal, scale=None, p_drop=0.0, seed=0, out=None, lse=None):
     lib = load_library()
     _check_bhnd("q", q)
     B, H, Nq, d = q.shape
-    _check_bhnd("k", k, None, q.dtype)
+    dev = q.device
+    _check_bhnd("k", k, None, q.dtype, dev)
     Nk = k.shape[2]
     if (k.shape[0], k.shape[1], k.shape[3]) != (B, H, d):
         raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, Nk, {d}]")
-    _check_bhnd("v", v, k.shape, q.dtype)
+    _check_bhnd("v", v, k.shape, q.dtype, dev)
     scale = d ** -0.5 if scale is None else scale
     out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
-    _check_bhnd("out", out, q.shape, q.dtype)
+    lse = torch.empty((B, H, Nq), device=dev, dtype=torch.float32) if lse is None else lse
+    _check_bhnd("out", out, q.shape, q.dtype, dev)
+    _check_f32("lse", lse, (B, H, Nq), dev)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
     tail = (d, int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1))
-    if Nq != Nk:
-        _raise(lib.fa_fwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_qk")
-    elif q.dtype == torch.bfloat16:
-        _raise(lib.fa_fwd(*ptrs, B, H, Nq, *tail, _stream(q)), "fa_fwd")
-    else:
-        _raise(lib.fa_fwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_ex")
+    with _guard(q):
+        if Nq != Nk:
+            _raise(lib.fa_fwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_qk")
+        elif q.dtype == torch.bfloat16:
+            _raise(lib.fa_fwd(*ptrs, B, H, Nq, *tail, _stream(q)), "fa_fwd")
+        else:
+            _raise(lib.fa_fwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_ex")
     return out, lse
 
 
@@ -146,43 +177,46 @@ def fa_bwd(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, workspac
     (square bf16 tensors go to fa_bwd, square fp16 ones to fa_bwd_ex, Nq != Nk or
     ``deterministic`` -- a fixed order of the dQ additions -- to fa_bwd_qk)."""
     lib = load_library()
-    for name, t in (("q", q), ("o", o), ("do", do)):
-        _check_bhnd(name, t, q.shape, q.dtype)
+    _check_bhnd("q", q)
     B, H, Nq, d = q.shape
-    _check_bhnd("k", k, None, q.dtype)
+    dev = q.device
+    for name, t in (("o", o), ("do", do)):
+        _check_bhnd(name, t, q.shape, q.dtype, dev)
+    _check_bhnd("k", k, None, q.dtype, dev)
     Nk = k.shape[2]
     if (k.shape[0], k.shape[1], k.shape[3]) != (B, H, d):
         raise ValueError(f"k has shape {tuple(k.shape)}, expected [{B}, {H}, Nk, {d}]")
-    _check_bhnd("v", v, k.shape, q.dtype)
+    _check_bhnd("v", v, k.shape, q.dtype, dev)
     scale = d ** -0.5 if scale is None else scale
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Nq) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, Nq] tensor")
+    _check_f32("lse", lse, (B, H, Nq), dev)
     det = int(bool(deterministic))
     ws_bytes = int(lib.fa_bwd_qk_workspace_size(B, H, Nq, d, det))
     if workspace is None:
-        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(k) if dv is None else dv
-    _check_bhnd("dq", dq, q.shape, q.dtype)
-    _check_bhnd("dk", dk, k.shape, q.dtype)
-    _check_bhnd("dv", dv, k.shape, q.dtype)
+    _check_bhnd("dq", dq, q.shape, q.dtype, dev)
+    _check_bhnd("dk", dk, k.shape, q.dtype, dev)
+    _check_bhnd("dv", dv, k.shape, q.dtype, dev)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
             dk.data_ptr(), dv.data_ptr())
     tail = (d, int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1))
-    ws = (workspace.data_ptr(), workspace.numel(), _stream(q))
-    if Nq != Nk or det:
-        _raise(lib.fa_bwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], det, *ws), "fa_bwd_qk")
-    elif q.dtype == torch.bfloat16:
-        _raise(lib.fa_bwd(*ptrs, B, H, Nq, *tail, *ws), "fa_bwd")
-    else:
-        _raise(lib.fa_bwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], *ws), "fa_bwd_ex")
+    with _guard(q):
+        ws = (*_ws_args(workspace, dev), _stream(q))
+        if Nq != Nk or det:
+            _raise(lib.fa_bwd_qk(*ptrs, B, H, Nq, Nk, *tail, FA_DTYPE[q.dtype], det, *ws), "fa_bwd_qk")
+        elif q.dtype == torch.bfloat16:
+            _raise(lib.fa_bwd(*ptrs, B, H, Nq, *tail, *ws), "fa_bwd")
+        else:
+            _raise(lib.fa_bwd_ex(*ptrs, B, H, Nq, *tail, FA_DTYPE[q.dtype], *ws), "fa_bwd_ex")
     return dq, dk, dv
 
 
-def _check_packed(name, t, dtype=None, rows=None, H=None, d=None):
+def _check_packed(name, t, dtype=None, rows=None, H=None, d=None, device=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    _check_device(name, t, device)
     if t.dtype not in FA_DTYPE or (dtype is not None and t.dtype != dtype):
         raise ValueError(f"{name} must be bf16 or fp16, the type of q")
     if t.dim() != 3 or not t.is_contiguous():
@@ -192,9 +226,10 @@ def _check_packed(name, t, dtype=None, rows=None, H=None, d=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}")
 
 
-def _check_cu(name, cu, B):
+def _check_cu(name, cu, B, device=None):
     if not cu.is_cuda or cu.dtype != torch.int32 or cu.dim() != 1 or cu.numel() != B + 1 or not cu.is_contiguous():
         raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of B + 1 offsets")
+    _check_device(name, cu, device)
 
 
 def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, scale=None, p_drop=0.0,
@@ -204,20 +239,24 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_
     lib = load_library()
     _check_packed("q", q)
     total_q, H, d = q.shape
-    _check_packed("k", k, q.dtype, None, H, d)
+    dev = q.device
+    _check_packed("k", k, q.dtype, None, H, d, dev)
     total_k = k.shape[0]
-    _check_packed("v", v, q.dtype, total_k, H, d)
+    _check_packed("v", v, q.dtype, total_k, H, d, dev)
     B = cu_seqlens_q.numel() - 1
-    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
-    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B, dev)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B, dev)
     scale = d ** -0.5 if scale is None else scale
     out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((H, total_q), device=q.device, dtype=torch.float32) if lse is None else lse
-    _check_packed("out", out, q.dtype, total_q, H, d)
-    _raise(lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q, total_k,
-                             int(max_seqlen_q), int(max_seqlen_k), d, int(bool(causal)), float(scale), float(p_drop),
-                             int(seed) & (2**64 - 1), FA_DTYPE[q.dtype], _stream(q)), "fa_fwd_varlen")
+    lse = torch.empty((H, total_q), device=dev, dtype=torch.float32) if lse is None else lse
+    _check_packed("out", out, q.dtype, total_q, H, d, dev)
+    _check_f32("lse", lse, (H, total_q), dev)
+    with _guard(q):
+        _raise(lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                 cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q, total_k,
+                                 int(max_seqlen_q), int(max_seqlen_k), d, int(bool(causal)), float(scale),
+                                 float(p_drop), int(seed) & (2**64 - 1), FA_DTYPE[q.dtype], _stream(q)),
+               "fa_fwd_varlen")
     return out, lse
 
 
@@ -228,30 +267,34 @@ def fa_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
     lib = load_library()
     _check_packed("q", q)
     total_q, H, d = q.shape
-    _check_packed("k", k, q.dtype, None, H, d)
+    dev = q.device
+    _check_packed("k", k, q.dtype, None, H, d, dev)
     total_k = k.shape[0]
-    _check_packed("v", v, q.dtype, total_k, H, d)
-    _check_packed("o", o, q.dtype, total_q, H, d)
-    _check_packed("do", do, q.dtype, total_q, H, d)
+    _check_packed("v", v, q.dtype, total_k, H, d, dev)
+    _check_packed("o", o, q.dtype, total_q, H, d, dev)
+    _check_packed("do", do, q.dtype, total_q, H, d, dev)
     B = cu_seqlens_q.numel() - 1
-    _check_cu("cu_seqlens_q", cu_seqlens_q, B)
-    _check_cu("cu_seqlens_k", cu_seqlens_k, B)
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (H, total_q) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [H, total_q] tensor")
+    _check_cu("cu_seqlens_q", cu_seqlens_q, B, dev)
+    _check_cu("cu_seqlens_k", cu_seqlens_k, B, dev)
+    _check_f32("lse", lse, (H, total_q), dev)
     scale = d ** -0.5 if scale is None else scale
     det = int(bool(deterministic))
     ws_bytes = int(lib.fa_bwd_varlen_workspace_size(B, H, total_q, int(max_seqlen_q), d, det))
     if workspace is None:
-        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(k) if dv is None else dv
-    _raise(lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(),
-                             cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
-                             int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1),
-                             FA_DTYPE[q.dtype], det, workspace.data_ptr(), workspace.numel(), _stream(q)),
-           "fa_bwd_varlen")
+    _check_packed("dq", dq, q.dtype, total_q, H, d, dev)
+    _check_packed("dk", dk, q.dtype, total_k, H, d, dev)
+    _check_packed("dv", dv, q.dtype, total_k, H, d, dev)
+    with _guard(q):
+        _raise(lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                 lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(),
+                                 cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q),
+                                 int(max_seqlen_k), d, int(bool(causal)), float(scale), float(p_drop),
+                                 int(seed) & (2**64 - 1), FA_DTYPE[q.dtype], det, *_ws_args(workspace, dev),
+                                 _stream(q)), "fa_bwd_varlen")
     return dq, dk, dv
 
 
@@ -261,32 +304,38 @@ def fa_bwd_stages(q, k, v, o, do, lse, causal, scale=None, p_drop=0.0, seed=0, w
     given, is called before stage i and after the last (i = 0..3) -- e.g. to
     record CUDA events around the tiles kernel."""
     lib = load_library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do)):
-        _check_bhnd(name, t, q.shape, torch.bfloat16)
+    _check_bhnd("q", q, None, torch.bfloat16)
+    dev = q.device
+    for name, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bhnd(name, t, q.shape, torch.bfloat16, dev)
     B, H, N, d = q.shape
+    _check_f32("lse", lse, (B, H, N), dev)
     scale = d ** -0.5 if scale is None else scale
     if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), device=q.device, dtype=torch.uint8)
+        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
-    st = _stream(q)
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bhnd(name, t, q.shape, torch.bfloat16, dev)
     seed = int(seed) & (2**64 - 1)
-    ws, wsb = workspace.data_ptr(), workspace.numel()
-    if between:
-        between(0)
-    _raise(lib.fa_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, ws, wsb, st),
-           "fa_bwd_prepare")
-    if between:
-        between(1)
-    _raise(lib.fa_bwd_tiles(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                            B, H, N, d, int(bool(causal)), float(scale), float(p_drop), seed, ws, wsb, st),
-           "fa_bwd_tiles")
-    if between:
-        between(2)
-    _raise(lib.fa_bwd_finish(dq.data_ptr(), B, H, N, d, float(scale), ws, wsb, st), "fa_bwd_finish")
-    if between:
-        between(3)
+    ws, wsb = _ws_args(workspace, dev)
+    with _guard(q):
+        st = _stream(q)
+        if between:
+            between(0)
+        _raise(lib.fa_bwd_prepare(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, ws, wsb, st),
+               "fa_bwd_prepare")
+        if between:
+            between(1)
+        _raise(lib.fa_bwd_tiles(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                                dv.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), float(p_drop), seed, ws,
+                                wsb, st), "fa_bwd_tiles")
+        if between:
+            between(2)
+        _raise(lib.fa_bwd_finish(dq.data_ptr(), B, H, N, d, float(scale), ws, wsb, st), "fa_bwd_finish")
+        if between:
+            between(3)
     return dq, dk, dv
 
 
@@ -298,27 +347,33 @@ def fa_decode_paged(q, k_cache, v_cache, block_table, seqlens_k, max_seqlen_k, c
     lib = load_library()
     _check_bhnd("q", q)
     B, H, Nq, d = q.shape
+    dev = q.device
     for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
         if not t.is_cuda or t.dtype != q.dtype or t.dim() != 4 or not t.is_contiguous() or t.shape[3] != d:
             raise ValueError(f"{name} must be a contiguous [num_pages, page_size, H_kv, d] tensor of q's type")
+        _check_device(name, t, dev)
     if tuple(v_cache.shape) != tuple(k_cache.shape):
         raise ValueError("v_cache must have k_cache's shape")
     num_pages, page, H_kv, _ = k_cache.shape
     for name, t, shape in (("block_table", block_table, (B, block_table.shape[-1])), ("seqlens_k", seqlens_k, (B,))):
         if not t.is_cuda or t.dtype != torch.int32 or tuple(t.shape) != shape or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous int32 CUDA tensor of shape {shape}")
+        _check_device(name, t, dev)
     scale = d ** -0.5 if scale is None else scale
     splits = int(num_splits) or int(lib.fa_decode_num_splits(B, H_kv, H, Nq, int(max_seqlen_k)))
     ws_bytes = int(lib.fa_decode_workspace_size(B, H, Nq, d, splits)) if splits > 0 else 0
     if workspace is None and ws_bytes:
-        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        workspace = torch.empty(ws_bytes, device=dev, dtype=torch.uint8)
     out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
-    _raise(lib.fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
-                               seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, H_kv, Nq, d, num_pages,
-                               page, block_table.shape[1], int(max_seqlen_k), int(bool(causal)), float(scale), splits,
-                               FA_DTYPE[q.dtype], workspace.data_ptr() if workspace is not None else None,
-                               workspace.numel() if workspace is not None else 0, _stream(q)), "fa_decode_paged")
+    lse = torch.empty((B, H, Nq), device=dev, dtype=torch.float32) if lse is None else lse
+    _check_bhnd("out", out, q.shape, q.dtype, dev)
+    _check_f32("lse", lse, (B, H, Nq), dev)
+    with _guard(q):
+        _raise(lib.fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                                   seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, H_kv, Nq, d, num_pages,
+                                   page, block_table.shape[1], int(max_seqlen_k), int(bool(causal)), float(scale),
+                                   splits, FA_DTYPE[q.dtype], *_ws_args(workspace, dev), _stream(q)),
+               "fa_decode_paged")
     return out, lse
 
 
@@ -326,7 +381,8 @@ def fa_dropout_mask(B, H, N, p_drop, seed, device="cuda"):
     """uint8 [B, H, N, N] keep mask generated by the device Philox (test/inspection export)."""
     lib = load_library()
     mask = torch.empty((B, H, N, N), device=device, dtype=torch.uint8)
-    st = lib.fa_dropout_mask(mask.data_ptr(), B, H, N, float(p_drop), int(seed) & (2**64 - 1), _stream(mask))
+    with _guard(mask):
+        st = lib.fa_dropout_mask(mask.data_ptr(), B, H, N, float(p_drop), int(seed) & (2**64 - 1), _stream(mask))
     _raise(st, "fa_dropout_mask")
     return mask
 
@@ -334,8 +390,11 @@ def fa_dropout_mask(B, H, N, p_drop, seed, device="cuda"):
 def fa_selftest_wait_timeout(limit_us=1000, device="cuda"):
     """Runs the bounded-wait self-test kernel (a wait that can only time out)."""
     lib = load_library()
-    st = torch.cuda.current_stream(torch.device(device))
-    _raise(lib.fa_selftest_wait_timeout(int(limit_us), ctypes.c_void_p(st.cuda_stream)), "fa_selftest_wait_timeout")
+    dev = torch.device(device)
+    with torch.cuda.device(dev):
+        st = torch.cuda.current_stream(dev)
+        _raise(lib.fa_selftest_wait_timeout(int(limit_us), ctypes.c_void_p(st.cuda_stream)),
+               "fa_selftest_wait_timeout")
 
 
 def fa_last_device_error():
