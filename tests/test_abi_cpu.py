@@ -23,7 +23,8 @@ def lib():
 def _declared_functions():
     names = set()
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
-        text = open(h).read()
+        with open(h) as f:
+            text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
         for m in re.finditer(r"\b(fa_[a-z0-9_]+)\s*\(", text):

@@ -115,10 +115,11 @@ def test_philox_slips_fail_the_known_answer_vectors(slip):
     import os
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "philox4x32_10_kat.txt")
     rows = []
-    for line in open(path):
-        if line.strip() and not line.startswith("#"):
-            lhs, rhs = line.split("->")
-            rows.append(([int(x, 16) for x in lhs.split()], [int(x, 16) for x in rhs.split()]))
+    with open(path) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                lhs, rhs = line.split("->")
+                rows.append(([int(x, 16) for x in lhs.split()], [int(x, 16) for x in rhs.split()]))
     m0, m1 = philox.PHILOX_M0, philox.PHILOX_M1
     if slip == "swapped_multipliers":
         m0, m1 = m1, m0
