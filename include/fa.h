@@ -315,7 +315,9 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
  *                 h reads key/value head h / (H / H_kv)
  *   causal      : nonzero -> query i of sequence b is position
  *                 seqlens_k[b] - Nq + i and sees positions up to it
- *   max_seqlen_k: the largest seqlens_k entry (sizes the launch)
+ *   max_seqlen_k: the largest seqlens_k entry (sizes the launch; a sequence
+ *                 longer than it is read only up to max_seqlen_k rounded up
+ *                 to a multiple of 128 positions)
  *   page_size   : 16, 32, 64 or 128; d in {32, 64, 96, 128}; no dropout
  *   num_splits  : how many parts each sequence's positions are cut into
  *                 (each a thread block, merged by log-sum-exp); 0 chooses
