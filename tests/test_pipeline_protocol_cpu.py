@@ -1,0 +1,412 @@
+"""Model checks of the kernels' mbarrier protocols (CPU; race detection in
+place of compute-sanitizer, which is not available).
+
+The forward kernel (fa_fwd.cu: two query tiles per CTA, a shared K/V ring,
+S_q(t+1) issued after PV_q(t), lazy O rescale without a wait) and the
+backward kernel (fa_bwd.cu: K/V once, Q and dO rings of two stages, the dQ
+drain staged through the tile's dO buffer) are restated as roles that step
+through their waits, arrivals and tensor-core operations: a TMA producer
+whose copies complete in any order, an MMA issuer whose operations and
+commits complete asynchronously but in issue order, and the softmax /
+elementwise / drain warps.  Random interleavings must finish with
+
+  * no deadlock,
+  * every parity wait seeing its barrier at the awaited phase or one before
+    it (never two phases on, where the parity would alias),
+  * every buffer holding the expected tile when read and never refilled or
+    overwritten while a reader is pending,
+  * no O rescale against a queued PV.
+
+Planted slips in the restated protocols are caught, which shows the checks
+bite.  A change to a kernel's barrier protocol is to be mirrored here."""
+
+import random
+
+import pytest
+
+
+class Bar:
+    """mbarrier: ``count`` arrivals complete a phase; ``done`` phases so far."""
+
+    def __init__(self, name, count=1):
+        self.name, self.count, self.pending, self.done = name, count, 0, 0
+
+    def arrive(self, n=1):
+        for _ in range(n):
+            self.pending += 1
+            if self.pending == self.count:
+                self.pending = 0
+                self.done += 1
+
+
+class Protocol:
+    """Common scheduler: roles are generators yielding ('wait', bar, phase) or None."""
+
+    def __init__(self, rng):
+        self.rng = rng
+        self.fifo, self.loads, self.errors = [], [], []
+
+    def ready(self, bar, k):
+        if bar.done >= k + 2:
+            self.errors.append(f"parity alias on {bar.name}: waiting for phase {k}, {bar.done} done")
+        return bar.done >= k + 1
+
+    def run(self, roles):
+        pending = [None] * len(roles)
+        alive = list(range(len(roles)))
+        for _ in range(500000):
+            if not (alive or self.fifo or self.loads):
+                return
+            choices = [("role", r) for r in alive if pending[r] is None or self.ready(pending[r][1], pending[r][2])]
+            if self.fifo:
+                choices.append(("mma", None))
+            if self.loads:
+                choices.append(("load", None))
+            if not choices:
+                self.errors.append("deadlock: " + str({r: (pending[r][1].name, pending[r][2]) for r in alive}))
+                return
+            kind, r = self.rng.choice(choices)
+            if kind == "mma":
+                self.fire_mma()
+            elif kind == "load":
+                self.fire_load()
+            else:
+                pending[r] = None
+                try:
+                    pending[r] = next(roles[r])
+                except StopIteration:
+                    alive.remove(r)
+            if self.errors:
+                return
+        self.errors.append("no termination")
+
+
+class Forward(Protocol):
+    def __init__(self, rng, nt0, nt1, nq, S, p_rescale, slip=None):
+        super().__init__(rng)
+        self.nt = [nt0, nt1 if nq == 2 else 0]
+        self.nq, self.S, self.p_rescale, self.slip = nq, S, p_rescale, slip
+        self.nt_all = nt1 if nq == 2 else nt0
+        self.q = Bar("q")
+        self.kfull = [Bar(f"kfull{s}") for s in range(S)]
+        self.vfull = [Bar(f"vfull{s}") for s in range(S)]
+        self.kvempty = [Bar(f"kvempty{s}") for s in range(S)]
+        self.s_ready = [Bar(f"s_ready{q}") for q in range(2)]
+        self.p_ready = [Bar(f"p_ready{q}", 4) for q in range(2)]
+        self.o_ready = [Bar(f"o_ready{q}") for q in range(2)]
+        self.kst, self.vst, self.readers = [None] * S, [None] * S, [0] * S
+        self.sbuf, self.sreading, self.pwritten = [None, None], [set(), set()], {}
+        self.o_pv, self.pv_queued = [-1, -1], [0, 0]
+
+    def producer(self):
+        if self.nt_all == 0:
+            return
+        self.loads.append(("q", None))
+        for t in range(self.nt_all):
+            s = t % self.S
+            # the slip: from the ring's third use of a stage on, refill without waiting for its release
+            if t >= self.S and not (self.slip == "early_stage_reuse" and t >= 2 * self.S):
+                yield ("wait", self.kvempty[s], t // self.S - 1)
+            if self.readers[s]:
+                self.errors.append(f"stage {s} refilled while read (tile {t})")
+            self.loads.append(("k", (s, t)))
+            self.loads.append(("v", (s, t)))
+            yield None
+
+    def mma(self):
+        if self.nt_all == 0:
+            return
+        yield ("wait", self.q, 0)
+        yield ("wait", self.kfull[0], 0)
+        for q in range(self.nq):
+            if self.nt[q]:
+                self.issue_s(q, 0, 0)
+        for t in range(self.nt_all):
+            s, s1 = t % self.S, (t + 1) % self.S
+            yield ("wait", self.vfull[s], t // self.S)
+            next_k = False
+            for q in range(self.nq):
+                if t >= self.nt[q]:
+                    continue
+                yield ("wait", self.p_ready[q], t)
+                self.readers[s] += 1
+                self.pv_queued[q] += 1
+                self.fifo.append(("pv", q, t, s))
+                if t == self.nt[q] - 1:
+                    self.fifo.append(("commit", self.o_ready[q]))
+                else:
+                    if not next_k:
+                        yield ("wait", self.kfull[s1], (t + 1) // self.S)
+                        next_k = True
+                    self.issue_s(q, t + 1, s1)
+            self.fifo.append(("commit", self.kvempty[s]))
+            yield None
+
+    def issue_s(self, q, t, s):
+        self.readers[s] += 1
+        self.fifo.append(("s", q, t, s))
+        self.fifo.append(("commit", self.s_ready[q]))
+
+    def softmax(self, q, w):
+        for t in range(self.nt[q]):
+            yield ("wait", self.s_ready[q], t)
+            if self.sbuf[q] != ("S", t):
+                self.errors.append(f"tile {q} warp {w} t {t}: buffer holds {self.sbuf[q]}")
+            self.sreading[q].add(w)
+            yield None
+            if t > 0 and self.rng.random() < self.p_rescale:
+                if self.o_pv[q] != t - 1 or self.pv_queued[q]:
+                    self.errors.append(f"tile {q} t {t}: O rescaled at PV {self.o_pv[q]}, {self.pv_queued[q]} queued")
+                yield None
+            self.sreading[q].discard(w)
+            self.pwritten.setdefault((q, t), set()).add(w)
+            if len(self.pwritten[(q, t)]) == 4:
+                self.sbuf[q] = ("P", t)
+            self.p_ready[q].arrive()
+            yield None
+        if self.nt[q]:
+            yield ("wait", self.o_ready[q], 0)
+            if self.o_pv[q] != self.nt[q] - 1:
+                self.errors.append(f"tile {q}: epilogue with O at PV {self.o_pv[q]}")
+
+    def fire_load(self):
+        kind, arg = self.loads.pop(self.rng.randrange(len(self.loads)))
+        if kind == "q":
+            self.q.arrive()
+        elif kind == "k":
+            self.kst[arg[0]] = arg[1]
+            self.kfull[arg[0]].arrive()
+        else:
+            self.vst[arg[0]] = arg[1]
+            self.vfull[arg[0]].arrive()
+
+    def fire_mma(self):
+        op = self.fifo.pop(0)
+        if op[0] == "commit":
+            op[1].arrive()
+            return
+        kind, q, t, s = op
+        if kind == "s":
+            if self.kst[s] != t:
+                self.errors.append(f"S{q}({t}) read a K stage holding {self.kst[s]}")
+            if self.sreading[q]:
+                self.errors.append(f"S{q}({t}) overwrote S while it was read")
+            if self.sbuf[q] is not None and self.sbuf[q][0] == "P" and self.sbuf[q][1] > self.o_pv[q]:
+                self.errors.append(f"S{q}({t}) overwrote P before its PV")
+            self.sbuf[q] = ("S", t)
+        else:
+            if self.vst[s] != t or len(self.pwritten.get((q, t), ())) != 4:
+                self.errors.append(f"PV{q}({t}): V stage holds {self.vst[s]}, P incomplete")
+            self.o_pv[q] = t
+            self.pv_queued[q] -= 1
+        self.readers[s] -= 1
+
+    def check(self):
+        self.run([self.producer(), self.mma()] + [self.softmax(q, w) for q in range(self.nq) for w in range(4)])
+        return self.errors
+
+
+class Backward(Protocol):
+    def __init__(self, rng, nq, slip=None):
+        super().__init__(rng)
+        self.nq, self.slip = nq, slip
+        self.kvfull = Bar("kvfull")
+        self.qfull = [Bar(f"qfull{s}") for s in range(2)]
+        self.dofull = [Bar(f"dofull{s}") for s in range(2)]
+        self.empty = [Bar(f"empty{s}") for s in range(2)]
+        self.dostage = [Bar(f"dostage{s}") for s in range(2)]
+        self.sready, self.dpready = Bar("sready"), Bar("dpready")
+        self.pready, self.dsready = Bar("pready", 8), Bar("dsready", 8)
+        self.dsfree, self.dqready, self.dqfree = Bar("dsfree"), Bar("dqready"), Bar("dqfree", 4)
+        self.dkdv = Bar("dkdvready")
+        self.qst, self.dost = [None, None], [None, None]
+        self.q_readers, self.do_readers = [0, 0], [0, 0]
+        self.tm_s = self.tm_dp = self.ds_smem = None
+        self.s_reading, self.dp_reading = set(), set()
+        self.p_written, self.ds_written = {}, {}
+        self.ds_readers, self.dq_reading, self.staging, self.dv_last = 0, False, None, -1
+
+    def producer(self):
+        self.loads.append(("kv", None))
+        for it in range(self.nq):
+            s = it & 1
+            if it >= 2:
+                yield ("wait", self.empty[s], (it >> 1) - 1)
+            if self.q_readers[s]:
+                self.errors.append(f"Q stage {s} refilled while read (tile {it})")
+            self.loads.append(("q", (s, it)))
+            yield None
+            if it >= 2 and self.slip != "no_dostage_wait":
+                yield ("wait", self.dostage[s], (it >> 1) - 1)
+            if self.do_readers[s] or self.staging == it - 2:
+                self.errors.append(f"dO stage {s} refilled while in use (tile {it})")
+            self.loads.append(("do", (s, it)))
+            yield None
+
+    def mma(self):
+        yield ("wait", self.kvfull, 0)
+        yield ("wait", self.qfull[0], 0)
+        self.op("S", 0, 0, self.sready)
+        yield ("wait", self.dofull[0], 0)
+        self.op("dP", 0, 0, self.dpready)
+        for it in range(self.nq):
+            s, s1, more = it & 1, (it + 1) & 1, it + 1 < self.nq
+            yield ("wait", self.pready, it)
+            self.op("dV", it, s)
+            if more:
+                yield ("wait", self.qfull[s1], (it + 1) >> 1)
+                self.op("S", it + 1, s1, self.sready)
+            yield ("wait", self.dsready, it)
+            self.op("dQ", it, None, self.dqready)
+            self.op("dK", it, s, self.empty[s])
+            self.fifo.append(("commit", self.dsfree))
+            if more:
+                if self.slip != "no_dqfree_wait":
+                    yield ("wait", self.dqfree, it)
+                yield ("wait", self.dofull[s1], (it + 1) >> 1)
+                self.op("dP", it + 1, s1, self.dpready)
+            yield None
+        self.fifo.append(("commit", self.dkdv))
+
+    def op(self, kind, it, s, commit=None):
+        if kind in ("S", "dK"):
+            self.q_readers[s] += 1
+        if kind in ("dV", "dP"):
+            self.do_readers[s] += 1
+        if kind in ("dQ", "dK"):
+            self.ds_readers += 1
+        self.fifo.append(("op", kind, it, s))
+        if commit is not None:
+            self.fifo.append(("commit", commit))
+
+    def drain(self):
+        for it in range(self.nq):
+            s = it & 1
+            yield ("wait", self.dqready, it)
+            if self.tm_dp != ("dQ", it) or self.do_readers[s] or self.dost[s] != ("dO", it):
+                self.errors.append(f"drain {it}: dQ cols {self.tm_dp}, dO stage {self.dost[s]}")
+            self.dq_reading, self.staging = True, it
+            self.dost[s] = ("staging", it)
+            yield None
+            self.dq_reading = False
+            self.dqfree.arrive(4)  # all of dQ is out of TMEM
+            yield None
+            self.staging = None  # the reduce-adds have read the staging buffer
+            self.dostage[s].arrive()
+            yield None
+
+    def elementwise(self, w):
+        for it in range(self.nq):
+            s = it & 1
+            yield ("wait", self.qfull[s], it >> 1)
+            yield ("wait", self.sready, it)
+            if self.tm_s != ("S", it) or self.qst[s] != it:
+                self.errors.append(f"warp {w} tile {it}: S cols {self.tm_s}, vectors of {self.qst[s]}")
+            self.s_reading.add(w)
+            yield None
+            self.s_reading.discard(w)
+            self.p_written.setdefault(it, set()).add(w)
+            if len(self.p_written[it]) == 8:
+                self.tm_s = ("P", it)
+            self.pready.arrive()
+            yield ("wait", self.dpready, it)
+            if self.tm_dp != ("dP", it) or self.qst[s] != it:
+                self.errors.append(f"warp {w} tile {it}: dP cols {self.tm_dp}, vectors of {self.qst[s]}")
+            self.dp_reading.add(w)
+            yield None
+            self.dp_reading.discard(w)
+            if it > 0:
+                yield ("wait", self.dsfree, it - 1)
+            if self.ds_readers:
+                self.errors.append(f"warp {w} tile {it}: dS written while read")
+            self.ds_written.setdefault(it, set()).add(w)
+            if len(self.ds_written[it]) == 8:
+                self.ds_smem = ("dS", it)
+            self.dsready.arrive()
+            yield None
+        yield ("wait", self.dkdv, 0)
+
+    def fire_load(self):
+        kind, arg = self.loads.pop(self.rng.randrange(len(self.loads)))
+        if kind == "kv":
+            self.kvfull.arrive()
+        elif kind == "q":
+            self.qst[arg[0]] = arg[1]
+            self.qfull[arg[0]].arrive()
+        else:
+            self.dost[arg[0]] = ("dO", arg[1])
+            self.dofull[arg[0]].arrive()
+
+    def fire_mma(self):
+        e = self.fifo.pop(0)
+        if e[0] == "commit":
+            e[1].arrive()
+            return
+        _, kind, it, s = e
+        if kind == "S":
+            busy = self.tm_s is not None and self.tm_s[0] == "P" and self.dv_last < self.tm_s[1]
+            if self.qst[s] != it or self.s_reading or busy:
+                self.errors.append(f"S{it}: Q stage {self.qst[s]}, S/P cols {self.tm_s} in use")
+            self.tm_s = ("S", it)
+            self.q_readers[s] -= 1
+        elif kind == "dP":
+            if self.dost[s] != ("dO", it) or self.dp_reading or self.dq_reading:
+                self.errors.append(f"dP{it}: dO stage {self.dost[s]}, dP/dQ cols {self.tm_dp} in use")
+            self.tm_dp = ("dP", it)
+            self.do_readers[s] -= 1
+        elif kind == "dV":
+            if self.tm_s != ("P", it) or self.dost[s] != ("dO", it):
+                self.errors.append(f"dV{it}: S cols {self.tm_s}, dO stage {self.dost[s]}")
+            self.dv_last = it
+            self.do_readers[s] -= 1
+        elif kind == "dQ":
+            if self.ds_smem != ("dS", it) or self.dp_reading or self.dq_reading:
+                self.errors.append(f"dQ{it}: dS {self.ds_smem}, dP cols in use")
+            self.tm_dp = ("dQ", it)
+            self.ds_readers -= 1
+        else:  # dK
+            if self.ds_smem != ("dS", it) or self.qst[s] != it:
+                self.errors.append(f"dK{it}: dS {self.ds_smem}, Q stage {self.qst[s]}")
+            self.ds_readers -= 1
+            self.q_readers[s] -= 1
+
+    def check(self):
+        self.run([self.producer(), self.mma(), self.drain()] + [self.elementwise(w) for w in range(8)])
+        return self.errors
+
+
+def _forward_cases():
+    for S in (2, 4):
+        for nq in (1, 2):
+            for nt0 in range(0, 6):
+                for nt1 in range(max(nt0, 1), 7):
+                    if nq == 1 and nt1 != nt0:
+                        continue
+                    yield S, nq, nt0, nt1
+
+
+def test_forward_protocol():
+    rng = random.Random(1)
+    for S, nq, nt0, nt1 in _forward_cases():
+        for _ in range(12):
+            errors = Forward(rng, nt0, nt1, nq, S, rng.choice([0.0, 0.5, 1.0])).check()
+            assert not errors, (S, nq, nt0, nt1, errors[:2])
+
+
+def test_backward_protocol():
+    rng = random.Random(2)
+    for nq in list(range(1, 8)) + [11]:
+        for _ in range(80):
+            errors = Backward(rng, nq).check()
+            assert not errors, (nq, errors[:2])
+
+
+def test_forward_slip_is_caught():
+    rng = random.Random(3)
+    assert any(Forward(rng, 6, 6, 1, 2, 0.0, slip="early_stage_reuse").check() for _ in range(40))
+
+
+@pytest.mark.parametrize("slip", ["no_dqfree_wait", "no_dostage_wait"])
+def test_backward_slips_are_caught(slip):
+    rng = random.Random(4)
+    assert any(Backward(rng, 4, slip=slip).check() for _ in range(40))
