@@ -2,9 +2,12 @@
 place of compute-sanitizer, which is not available).
 
 The forward kernel (fa_fwd.cu: two query tiles per CTA, a shared K/V ring,
-S_q(t+1) issued after PV_q(t), lazy O rescale without a wait) and the
-backward kernel (fa_bwd.cu: K/V once, Q and dO rings of two stages, the dQ
-drain staged through the tile's dO buffer) are restated as roles that step
+S_q(t+1) issued after PV_q(t), lazy O rescale without a wait), the backward
+kernel (fa_bwd.cu: K/V once, Q and dO rings of two stages, the dQ drain
+staged through the tile's dO buffer) and the paged decode kernel
+(fa_decode.cu: S^T double buffer issued a tile ahead, P and its products
+doubled by tile parity, stages refilled after their P V product, the tail
+tile's V rows zeroed by the softmax warps) are restated as roles that step
 through their waits, arrivals and tensor-core operations: a TMA producer
 whose copies complete in any order, an MMA issuer whose operations and
 commits complete asynchronously but in issue order, and the softmax /
@@ -375,6 +378,132 @@ class Backward(Protocol):
         return self.errors
 
 
+class Decode(Protocol):
+    """fa_decode.cu: one thread issues the page copies and both products; the
+    four softmax warps move together (named barriers), so they are one role
+    whose p_ready arrival counts four."""
+
+    def __init__(self, rng, n, S, tail, p_rescale, slip=None):
+        super().__init__(rng)
+        self.n, self.S, self.tail, self.p_rescale, self.slip = n, S, tail, p_rescale, slip
+        self.kfull = [Bar(f"kfull{s}") for s in range(S)]
+        self.vfull = [Bar(f"vfull{s}") for s in range(S)]
+        self.s_ready = [Bar(f"s_ready{b}") for b in range(2)]
+        self.p_ready = [Bar(f"p_ready{b}", 4) for b in range(2)]
+        self.pv_done = [Bar(f"pv_done{b}") for b in range(2)]
+        self.kst, self.vst, self.readers = [None] * S, [None] * S, [0] * S
+        self.sbuf, self.s_reading = [None, None], [False, False]
+        self.pbuf, self.p_readers = [None, None], [0, 0]
+        self.o_pv, self.pv_queued = -1, 0
+
+    def load(self, it):
+        st = it % self.S
+        if self.readers[st]:
+            self.errors.append(f"stage {st} refilled while read (tile {it})")
+        self.loads.append(("k", (st, it)))
+        self.loads.append(("v", (st, it)))
+
+    def issue_s(self, it):
+        st = it % self.S
+        yield ("wait", self.kfull[st], it // self.S)
+        self.readers[st] += 1
+        self.fifo.append(("s", it, st))
+        self.fifo.append(("commit", self.s_ready[it & 1]))
+
+    def producer(self):
+        n, S = self.n, self.S
+        if n == 0:  # a split without tiles issues nothing
+            return
+        issued = 0
+        while issued < min(S - 1, n):
+            self.load(issued)
+            issued += 1
+        yield from self.issue_s(0)
+        for it in range(n):
+            if it + 1 < n:
+                yield from self.issue_s(it + 1)
+            if issued < n:
+                if it >= 1 and self.slip != "no_refill_wait":
+                    yield ("wait", self.pv_done[(it - 1) & 1], (it - 1) >> 1)
+                self.load(issued)
+                issued += 1
+            if self.slip == "single_p_ready":
+                yield ("wait", self.p_ready[0], it)
+            else:
+                yield ("wait", self.p_ready[it & 1], it >> 1)
+            yield ("wait", self.vfull[it % S], it // S)
+            self.readers[it % S] += 1
+            self.p_readers[it & 1] += 1
+            self.pv_queued += 1
+            self.fifo.append(("pv", it, it % S))
+            self.fifo.append(("commit", self.pv_done[it & 1]))
+            yield None
+
+    def softmax(self):
+        n, S = self.n, self.S
+        for it in range(n):
+            b = it & 1
+            yield ("wait", self.s_ready[b], it >> 1)
+            if self.sbuf[b] != ("S", it):
+                self.errors.append(f"softmax {it}: S buffer {b} holds {self.sbuf[b]}")
+            self.s_reading[b] = True
+            yield None
+            if self.tail and it == n - 1:
+                # zero the V rows past the sequence once the tile's V has landed
+                yield ("wait", self.vfull[it % S], it // S)
+                if self.vst[it % S] != it or self.readers[it % S]:
+                    self.errors.append(f"softmax {it}: V stage holds {self.vst[it % S]} while zeroed")
+            if it >= 2:
+                yield ("wait", self.pv_done[b], (it - 2) >> 1)
+            if self.p_readers[b]:
+                self.errors.append(f"softmax {it}: P buffer {b} written while a product reads it")
+            self.pbuf[b] = it
+            rescale = it > 0 and self.rng.random() < self.p_rescale
+            if rescale:
+                yield ("wait", self.pv_done[(it - 1) & 1], (it - 1) >> 1)
+                if self.o_pv != it - 1 or self.pv_queued:
+                    self.errors.append(f"softmax {it}: O rescaled at PV {self.o_pv}, {self.pv_queued} queued")
+            self.s_reading[b] = False
+            self.p_ready[0 if self.slip == "single_p_ready" else b].arrive(4)
+            yield None
+        if n:
+            yield ("wait", self.pv_done[(n - 1) & 1], (n - 1) >> 1)
+            if self.o_pv != n - 1:
+                self.errors.append(f"epilogue with O at PV {self.o_pv}")
+
+    def fire_load(self):
+        kind, (st, it) = self.loads.pop(self.rng.randrange(len(self.loads)))
+        if kind == "k":
+            self.kst[st] = it
+            self.kfull[st].arrive()
+        else:
+            self.vst[st] = it
+            self.vfull[st].arrive()
+
+    def fire_mma(self):
+        e = self.fifo.pop(0)
+        if e[0] == "commit":
+            e[1].arrive()
+            return
+        kind, it, st = e
+        b = it & 1
+        if kind == "s":
+            if self.kst[st] != it or self.s_reading[b]:
+                self.errors.append(f"S{it}: K stage holds {self.kst[st]}, buffer {b} in use")
+            self.sbuf[b] = ("S", it)
+        else:
+            if self.vst[st] != it or self.pbuf[b] != it:
+                self.errors.append(f"PV{it}: V stage holds {self.vst[st]}, P buffer holds {self.pbuf[b]}")
+            self.o_pv = it
+            self.pv_queued -= 1
+            self.p_readers[b] -= 1
+        self.readers[st] -= 1
+
+    def check(self):
+        self.run([self.producer(), self.softmax()])
+        return self.errors
+
+
 def _forward_cases():
     for S in (2, 4):
         for nq in (1, 2):
@@ -410,3 +539,18 @@ def test_forward_slip_is_caught():
 def test_backward_slips_are_caught(slip):
     rng = random.Random(4)
     assert any(Backward(rng, 4, slip=slip).check() for _ in range(40))
+
+
+def test_decode_protocol():
+    rng = random.Random(5)
+    for S in (3, 4):
+        for n in list(range(0, 9)) + [13]:
+            for _ in range(40):
+                errors = Decode(rng, n, S, rng.random() < 0.5, rng.choice([0.0, 0.5, 1.0])).check()
+                assert not errors, (S, n, errors[:2])
+
+
+@pytest.mark.parametrize("slip", ["no_refill_wait", "single_p_ready"])
+def test_decode_slips_are_caught(slip):
+    rng = random.Random(6)
+    assert any(Decode(rng, 8, 3, False, 0.0, slip=slip).check() for _ in range(60))
