@@ -3,7 +3,6 @@ every entry point include/*.h declares, and rejects bad arguments before it
 makes any CUDA call.  Every call here carries at least one invalid argument,
 so nothing is ever launched."""
 
-import ctypes
 import glob
 import os
 import re

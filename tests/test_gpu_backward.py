@@ -7,7 +7,6 @@ of 256 query rows (dQ, which needs only those rows of S) and 256 key rows
 those for the checked heads block by block).  Tolerance: relative Frobenius
 error <= 2e-2 on each gradient."""
 
-import numpy as np
 import pytest
 import torch
 
