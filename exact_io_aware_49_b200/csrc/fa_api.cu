@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/fa.h"
 #include "fa_internal.h"
 #include "philox.cuh"
@@ -21,17 +23,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once.  The function-local static
+// is initialised exactly once even when several host threads make their first
+// call at the same time; a failed lookup is remembered as nullptr.
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
             cudaSuccess ||
         q != cudaDriverEntryPointSuccess)
       return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
   return fn;
 }
 
@@ -54,14 +58,20 @@ bool encode_map(CUtensorMap* tm, const void* base, int d, long long T, long long
   return r == CUDA_SUCCESS;
 }
 
+// Device address of g_fa_error_word on the current device, cached per device.
+// Concurrent first calls from several host threads may each look it up; they
+// store the same address, and the atomics make those stores race-free.
 unsigned* error_word_ptr() {
-  static unsigned* cache[128] = {nullptr};
+  static std::atomic<unsigned*> cache[128];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
-  if (dev < 128 && cache[dev]) return cache[dev];
+  if (dev < 128) {
+    unsigned* c = cache[dev].load(std::memory_order_acquire);
+    if (c) return c;
+  }
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return nullptr;
-  if (dev < 128) cache[dev] = static_cast<unsigned*>(p);
+  if (dev < 128) cache[dev].store(static_cast<unsigned*>(p), std::memory_order_release);
   return static_cast<unsigned*>(p);
 }
 

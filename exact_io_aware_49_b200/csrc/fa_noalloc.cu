@@ -15,6 +15,7 @@
 // device address is looked up with cudaGetSymbolAddress once per device, with
 // that device current, on the first call made on it.
 #include <cuda_runtime.h>
+#include <math.h>
 
 #include <atomic>
 
@@ -44,9 +45,14 @@ void* scratch_address() {
 extern "C" fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                                     const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                                     int causal, float scale, float p_drop, uint64_t seed, void* stream) {
-  // Validate the arguments first (same rules as fa_bwd, with a workspace that
-  // is known to be large enough) so a rejected call never touches the device.
+  // Validate the arguments first, with fa_bwd's rules and in its order (sizes,
+  // scalars, supported head dimension), so that the same bad arguments get the
+  // same status from both entry points; only then the scratch limit.  A
+  // rejected call never touches the device.
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
+  if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need == 0) return FA_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_UNSUPPORTED;

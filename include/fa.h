@@ -338,9 +338,19 @@ fa_status fa_decode_paged(const void* Q, const void* K_cache, const void* V_cach
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Test/inspection export: writes the dropout keep mask Z (1 = kept, 0 =
- * dropped) as uint8 [B, H, N, N] into device memory ``mask`` with the same
- * device Philox code the kernels use.  N here only needs to be positive.
+ * Test/inspection export of the attention-dropout pattern.  Dropout is
+ * Bernoulli per attention score, applied inside the softmax step, and its
+ * pattern is regenerated during the backward recomputation instead of being
+ * stored ("FlashAttention" glossary, Dropout bullet; "Flash Attention"
+ * glossary, Key Components).  This call writes that pattern, the keep mask
+ * Z (1 = kept, 0 = dropped), as uint8 [B, H, N, N] into caller-owned device
+ * memory ``mask`` (row i, column j = query i, key j), computed by the same
+ * device Philox4x32-10 and keep test the kernels use: counter
+ * (j >> 3, i, h, b), key (seed mod 2^32, seed >> 32), keep <=> u16 >= t with
+ * t = round-half-even(p_drop * 65536).  N only needs to be positive; the
+ * buffer must hold B*H*N*N bytes.  FA_ERR_INVALID_ARG for a null mask,
+ * non-positive sizes or p_drop outside [0, 1); FA_ERR_UNSUPPORTED when
+ * B*H*N >= 2^31.  Asynchronous on ``stream``.
  */
 fa_status fa_dropout_mask(uint8_t* mask, int B, int H, int N, float p_drop, uint64_t seed,
                           void* stream);
