@@ -3,6 +3,9 @@ inputs and compare with the tolerances the method fixes (bf16 I/O, fp32
 accumulation): O max-abs <= 1e-2 and relative Frobenius <= 5e-3; LSE
 absolute <= 1e-3; dQ/dK/dV relative Frobenius <= 2e-2; masks bit-exact."""
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -75,3 +78,13 @@ def oracle_fwd_head(q, k, v, b, h, causal, scale, p_drop, seed, rows=None):
     lse, o, _ = attention.row_stats(qh, kh, vh, np.zeros_like(vh), causal=causal, scale=scale, p_drop=p_drop,
                                     seed=seed, b=b, h=h, rows=rows)
     return o, lse
+
+
+def map_heads(fn, items):
+    """fn over ``items`` on a pool of host threads (NumPy releases the GIL in
+    its array kernels, so per-head oracle work runs in parallel); returns the
+    results in order and re-raises the first failure."""
+    items = list(items)
+    workers = max(1, min(len(items), len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(workers) as ex:
+        return list(ex.map(fn, items))

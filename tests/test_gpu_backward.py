@@ -7,6 +7,7 @@ of 256 query rows (dQ, which needs only those rows of S) and 256 key rows
 those for the checked heads block by block).  Tolerance: relative Frobenius
 error <= 2e-2 on each gradient."""
 
+import numpy as np
 import pytest
 import torch
 
@@ -28,7 +29,9 @@ def _run(q, k, v, do, causal, scale, p, seed):
 
 def _heads_full(q, k, v, do, res, heads, causal, scale, p, seed):
     o, lse, dq, dk, dv = res
-    for b, h in heads:
+
+    def one(bh):
+        b, h = bh
         args = [x[b, h].to(torch.float64).numpy() for x in (q, k, v, do)]
         kw = dict(causal=causal, scale=scale, p_drop=p, seed=seed, b=b, h=h)
         want_o, want_l = attention.forward(*args[:3], **kw)
@@ -38,6 +41,15 @@ def _heads_full(q, k, v, do, res, heads, causal, scale, p, seed):
         pu.check_grad(pu.f64(dq[b, h]), want_dq, f"dQ {(b, h)}")
         pu.check_grad(pu.f64(dk[b, h]), want_dk, f"dK {(b, h)}")
         pu.check_grad(pu.f64(dv[b, h]), want_dv, f"dV {(b, h)}")
+
+    pu.map_heads(one, heads)
+
+
+def _spread_heads(B, H, n):
+    """n (b, h) pairs spread over the batch and head indices."""
+    units = [(b, h) for b in range(B) for h in range(H)]
+    step = max(1, len(units) // n)
+    return [units[(i * step + i // 2) % len(units)] for i in range(n)]
 
 
 def test_causal_n1024_all_heads():
@@ -49,30 +61,53 @@ def test_causal_n1024_all_heads():
 
 
 def test_causal_dropout_n4096_full_size():
+    """B=4 H=16 N=4096 d=128, causal, p=0.1: whole heads (8 of the 64, spread
+    over b and h) of dQ, dK, dV, O and LSE."""
     w = wl.WORKLOADS[2]
     q, k, v, do = wl.draw_inputs(w)
     res = _run(q, k, v, do, w.causal, w.scale, w.p_drop, w.seed)
     for t in res:
         assert torch.isfinite(t.float()).all()
-    _heads_full(q, k, v, do, res, [(0, 0), (3, 15)], w.causal, w.scale, w.p_drop, w.seed)
+    heads = _spread_heads(w.B, w.H, 8)
+    assert len(set(heads)) == 8 and len({b for b, _ in heads}) == w.B
+    _heads_full(q, k, v, do, res, heads, w.causal, w.scale, w.p_drop, w.seed)
 
 
-@pytest.mark.parametrize("idx", [3, 4])
-def test_long_context_full_size_sampled(idx):
+@pytest.mark.parametrize("idx,kv_heads", [(3, 8), (4, 4)])
+def test_long_context_full_size_sampled(idx, kv_heads):
+    """Full-size launch.  dQ on the 256 seeded query rows of every head (each
+    needs only its own row of S); dK and dV on the same indices as key rows for
+    ``kv_heads`` heads spread over (b, h) -- those need LSE_i and D_i of every
+    query row, which the oracle evaluates for the checked heads in row blocks."""
     w = wl.WORKLOADS[idx]
     q, k, v, do = wl.draw_inputs(w)
     o, lse, dq, dk, dv = _run(q, k, v, do, w.causal, w.scale, w.p_drop, w.seed)
     for t in (o, lse, dq, dk, dv):
         assert torch.isfinite(t.float()).all()
     samples = wl.sample_rows(w, n_rows=256)
-    for b, h in [(0, 0), (w.B - 1, w.H - 1)]:
-        args = [x[b, h].to(torch.float64).numpy() for x in (q, k, v, do)]
-        kw = dict(causal=w.causal, scale=w.scale, p_drop=w.p_drop, seed=w.seed, b=b, h=h)
+
+    def kwargs(b, h):
+        return dict(causal=w.causal, scale=w.scale, p_drop=w.p_drop, seed=w.seed, b=b, h=h)
+
+    def head_args(b, h):
+        return [x[b, h].to(torch.float64).numpy() for x in (q, k, v, do)]
+
+    def dq_rows(bh):
+        b, h = bh
         rows = samples[b][h].numpy()
-        want_dq = attention.grad_rows(*args, rows=rows, **kw)
+        want_dq = attention.grad_rows(*head_args(b, h), rows=rows, **kwargs(b, h))
         pu.check_grad(pu.f64(dq[b, h])[rows], want_dq, f"dQ rows {(b, h)}")
-        lse_all, _, d_all = attention.row_stats(*args, **kw)
-        want_dk, want_dv = attention.grad_cols(*args, lse_all, d_all, cols=rows, **kw)
+
+    pu.map_heads(dq_rows, [(b, h) for b in range(w.B) for h in range(w.H)])
+
+    for b, h in _spread_heads(w.B, w.H, kv_heads):
+        args = head_args(b, h)
+        chunks = [np.arange(a, min(w.N, a + 2048)) for a in range(0, w.N, 2048)]
+        stats = pu.map_heads(lambda r: attention.row_stats(*args, rows=r, **kwargs(b, h)), chunks)
+        lse_all = np.concatenate([s[0] for s in stats])
+        d_all = np.concatenate([s[2] for s in stats])
+        rows = samples[b][h].numpy()
+        want_dk, want_dv = attention.grad_cols(*args, lse_all, d_all, cols=rows, **kwargs(b, h))
         pu.check_grad(pu.f64(dk[b, h])[rows], want_dk, f"dK rows {(b, h)}")
         pu.check_grad(pu.f64(dv[b, h])[rows], want_dv, f"dV rows {(b, h)}")
 

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import paged
+from oracle import attention, paged
 from tests import parity_util as pu
 
 pytestmark = pytest.mark.gpu
@@ -99,3 +99,38 @@ def test_decode_fp16():
 def test_no_device_wait_timed_out():
     from exact_io_aware_49_b200 import fa_last_device_error
     assert fa_last_device_error() == 0
+
+
+def test_bench_shape_sampled_sequences():
+    """The decode benchmark's launch: 16 sequences x 32768 cached positions,
+    32 query / 8 key-value heads, one query, d = 128, pages of 64 in shuffled
+    order, the split count fa_decode_num_splits picks (8 here).  The cache is
+    drawn on the device; every query head of three sequences (first, middle,
+    last) is checked against the oracle on those sequences' gathered pages."""
+    from exact_io_aware_49_b200 import binding, fa_decode_paged
+    B, H, H_kv, Nq, d, L, page = 16, 32, 8, 1, 128, 32768, 64
+    lib = binding.load_library()
+    splits = int(lib.fa_decode_num_splits(B, H_kv, H, Nq, L))
+    assert splits > 1
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    n_pages = B * (L // page)
+    kc = torch.randn(n_pages, page, H_kv, d, generator=gen, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(n_pages, page, H_kv, d, generator=gen, device="cuda").to(torch.bfloat16)
+    table = torch.randperm(n_pages, generator=gen, device="cuda").to(torch.int32).view(B, -1)
+    q = torch.randn(B, H, Nq, d, generator=gen, device="cuda").to(torch.bfloat16)
+    lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    o, lse = fa_decode_paged(q, kc, vc, table, lens, L, True, d ** -0.5, num_splits=splits)
+    torch.cuda.synchronize()
+    for b in (0, B // 2, B - 1):
+        pages = table[b].long()
+        k_b = kc[pages].reshape(L, H_kv, d).to(torch.float64).cpu().numpy()
+        v_b = vc[pages].reshape(L, H_kv, d).to(torch.float64).cpu().numpy()
+        q_b = q[b].to(torch.float64).cpu().numpy()
+
+        def one(h):
+            g = h // (H // H_kv)
+            want_o, want_l = attention.forward(q_b[h], k_b[:, g], v_b[:, g], causal=True, scale=d ** -0.5)
+            pu.check_o(pu.f64(o[b, h]), want_o, f"O seq {b} head {h}")
+            pu.check_lse(pu.f64(lse[b, h]), want_l, f"LSE seq {b} head {h}")
+
+        pu.map_heads(one, range(H))

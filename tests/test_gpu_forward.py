@@ -23,13 +23,16 @@ def _run(q, k, v, causal, scale, p, seed):
 
 
 def _compare_heads(q, k, v, o, lse, heads, causal, scale, p, seed, rows_by_head=None):
-    for b, h in heads:
+    def one(bh):
+        b, h = bh
         rows = None if rows_by_head is None else rows_by_head[(b, h)]
         want_o, want_l = pu.oracle_fwd_head(q, k, v, b, h, causal, scale, p, seed, rows)
         got_o = pu.f64(o[b, h]) if rows is None else pu.f64(o[b, h])[rows]
         got_l = pu.f64(lse[b, h]) if rows is None else pu.f64(lse[b, h])[rows]
         pu.check_o(got_o, want_o, f"head {(b, h)}")
         pu.check_lse(got_l, want_l, f"head {(b, h)}")
+
+    pu.map_heads(one, heads)
 
 
 def _all_heads(B, H):
@@ -51,21 +54,24 @@ def test_causal_n1024_all_heads():
 
 
 def test_causal_dropout_n4096_full_size():
+    """B=4 H=16 N=4096 d=128, causal, p=0.1: every element of every head."""
     w = wl.WORKLOADS[2]
     q, k, v, _ = wl.draw_inputs(w)
     o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
-    _compare_heads(q, k, v, o, lse, [(0, 0), (1, 7), (3, 15)], w.causal, w.scale, w.p_drop, w.seed)
+    _compare_heads(q, k, v, o, lse, _all_heads(w.B, w.H), w.causal, w.scale, w.p_drop, w.seed)
 
 
 @pytest.mark.parametrize("idx", [3, 4])
 def test_long_context_full_size_sampled_rows(idx):
+    """N = 16384 (logit spread ~16) and N = 32768 (p = 0.1) at full size: 256
+    seeded query rows of every head."""
     w = wl.WORKLOADS[idx]
     q, k, v, _ = wl.draw_inputs(w)
     o, lse = _run(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
     samples = wl.sample_rows(w, n_rows=256)
-    heads = [(0, 0), (w.B - 1, w.H - 1), (0, w.H // 2)]
+    heads = _all_heads(w.B, w.H)
     rows = {(b, h): samples[b][h].numpy() for b, h in heads}
     _compare_heads(q, k, v, o, lse, heads, w.causal, w.scale, w.p_drop, w.seed, rows)
 
