@@ -12,11 +12,15 @@ FLOPs per step: forward 4*B*H*N^2*d/2 (causal), backward 2.5x the forward.
 
   value     fwd+bwd TFLOP/s over all ranks, inputs resident in HBM, timed with
             CUDA events on the launching stream (max over ranks)
-  e2e       the same through the public Python API, each step also copying
-            Q, K, V, dO host->device from pinned memory and O, LSE, dQ, dK, dV
-            back to the host
+  e2e       the same through the C ABI's host-buffer call fa_fwd_bwd_host:
+            each step copies Q, K, V, dO host->device from pinned memory and
+            O, LSE, dQ, dK, dV back, in 8 groups of heads whose copies overlap
+            the kernels of the neighbouring groups on three streams
   roofline  the kernel with the largest share of the step, achieved TFLOP/s
-            from its own CUDA events against the measured bf16 peak
+            from its own CUDA events against the measured bf16 burst peak
+  other_workloads  fa_fwd and the backward on B=4 H=16 N=4096 d=128 causal
+            p=0.1 (the other dropout workload), each call timed with CUDA
+            events (median), TFLOP/s and % of the burst peak
   cpu_baseline  the fp64 oracle on this host's cores on a bounded sample
             (a causal prefix of one head, which is itself a complete causal
             attention problem)
@@ -65,6 +69,7 @@ FWD_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_fwd.cu")
 DECODE_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_decode.cu")
 DECODE_WORKLOAD = "decode_paged_B16_L32768_H32_Hkv8_d128"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+E2E_GROUPS = 8  # head groups of the host-buffer step (copies of one overlap the kernels of the next)
 
 
 def _peaks():
@@ -271,21 +276,20 @@ def run_ours(args, w, world, device):
     fwd_ms, bwd_ms, tiles_ms = per.mean(axis=0)
     ms_step_max = _max_over_ranks(world, ms_step, device)
 
-    # ---- end to end through the public API: H2D of the step's inputs, D2H of its results
-    from exact_io_aware_49_b200 import fa_bwd, fa_fwd
+    # ---- end to end through the C ABI on host buffers (fa_fwd_bwd_host): each
+    # step copies Q, K, V, dO in from pinned memory and O, LSE, dQ, dK, dV out,
+    # in groups of heads whose copies overlap the kernels on three streams
     oh = torch.empty_like(qh).pin_memory()
     dqh, dkh, dvh = (torch.empty_like(qh).pin_memory() for _ in range(3))
     lseh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    q2, k2, v2, do2 = (torch.empty_like(q) for _ in range(4))
+    groups = E2E_GROUPS
+    host_ws = torch.empty(binding.fa_fwd_bwd_host_workspace_size(w.B, w.H, w.N, w.d, groups), device=device,
+                          dtype=torch.uint8)
+    streams = [torch.cuda.Stream(device) for _ in range(3)]
 
     def e2e_step():
-        for dst, src in ((q2, qh), (k2, kh), (v2, vh), (do2, doh)):
-            dst.copy_(src, non_blocking=True)
-        o2, lse2 = fa_fwd(q2, k2, v2, w.causal, w.scale, w.p_drop, w.seed, out=o, lse=lse)
-        g = fa_bwd(q2, k2, v2, o2, do2, lse2, w.causal, w.scale, w.p_drop, w.seed, workspace=ws, dq=dq, dk=dk,
-                   dv=dv)
-        for dst, src in ((oh, o2), (lseh, lse2), (dqh, g[0]), (dkh, g[1]), (dvh, g[2])):
-            dst.copy_(src, non_blocking=True)
+        binding.fa_fwd_bwd_host(qh, kh, vh, doh, w.causal, w.scale, w.p_drop, w.seed, groups=groups, device=device,
+                                workspace=host_ws, streams=streams, out=oh, lse=lseh, dq=dqh, dk=dkh, dv=dvh)
 
     e2e_steps = max(1, min(args.steps, 10))
     for _ in range(min(args.warmup, 2)):
@@ -294,10 +298,10 @@ def run_ours(args, w, world, device):
     torch.cuda.synchronize(device)
     a = torch.cuda.Event(enable_timing=True)
     bev = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(streams[2])  # each call starts after the work on its copy-out stream
     for _ in range(e2e_steps):
         e2e_step()
-    bev.record(stream)
+    bev.record(streams[2])
     torch.cuda.synchronize(device)
     e2e_ms = _max_over_ranks(world, a.elapsed_time(bev) / e2e_steps, device)
     h2d = sum(x.numel() * x.element_size() for x in (qh, kh, vh, doh))
@@ -317,7 +321,9 @@ def run_ours(args, w, world, device):
     else:
         kname, k_ms, k_flops, src = "fa_fwd", fwd_ms, flops_fwd, FWD_SOURCE
     achieved = k_flops / (k_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # the dominant kernel runs ~30 ms at a time inside a sub-second timed
+    # region: the burst figure is its peak; the sustained fraction is kept beside it
+    peak = peaks["bf16_tflops"]
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak",
@@ -334,15 +340,55 @@ def run_ours(args, w, world, device):
         },
         "kernel_ms": {"fa_fwd": fwd_ms, "fa_bwd (3 stages)": bwd_ms, "fa_bwd_tiles": tiles_ms},
         "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
-                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "frac": achieved / peak, "peak_kind": f"bf16_tflops, burst ({peak_src})",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
                      "traffic": _traffic(kname, src)},
         "e2e": {"value": n * flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": f"fa_fwd_bwd_host (C ABI, pinned host buffers, {groups} head groups, 3 streams)"},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
+    if w.name == WORKLOAD and not args.no_other_workloads:
+        # the other d = 128 causal dropout workload the throughput target names
+        other = wl.BY_NAME["causal_dropout_N4096_d128"]
+        out["other_workloads"] = {other.name: time_other_workload(other, device, peaks)}
     return out, (qh, kh, vh, doh)
+
+
+def time_other_workload(w, device, peaks, reps=20, warmup=3):
+    """fa_fwd and the backward (three stages) on another workload's inputs,
+    each call timed alone with CUDA events on the launching stream (median of
+    ``reps``); reported beside the main line, not part of its value."""
+    from exact_io_aware_49_b200 import binding
+    stream = torch.cuda.current_stream(device)
+    q, k, v, do = (x.to(device) for x in wl.draw_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), device=device, dtype=torch.float32)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(binding.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), device=device, dtype=torch.uint8)
+    tf, tb = [], []
+    for it in range(warmup + reps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        binding.fa_fwd(q, k, v, w.causal, w.scale, w.p_drop, w.seed, out=o, lse=lse)
+        e[1].record(stream)
+        binding.fa_bwd_stages(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, workspace=ws, dq=dq,
+                              dk=dk, dv=dv)
+        e[2].record(stream)
+        torch.cuda.synchronize(device)
+        if it >= warmup:
+            tf.append(e[0].elapsed_time(e[1]))
+            tb.append(e[1].elapsed_time(e[2]))
+    fwd_ms, bwd_ms = float(np.median(tf)), float(np.median(tb))
+    fwd_tf = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
+    return {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "p_drop": w.p_drop,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_pct_of_burst": 100 * fwd_tf / peaks["bf16_tflops"],
+            "bwd_pct_of_burst": 100 * bwd_tf / peaks["bf16_tflops"],
+            "timing": f"CUDA events per call, median of {reps} after {warmup} warm-up calls; "
+                      "inputs (Q, K, V, dO 67 MB each) are resident, no L2 flush"}
 
 
 # --------------------------------------------------------------------- decode line
@@ -480,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the per-call timing of the N=4096 dropout workload beside the main line")
     ap.add_argument("--decode", action="store_true", help="the paged-cache decode line instead (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

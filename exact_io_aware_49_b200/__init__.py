@@ -7,7 +7,7 @@ and fails loudly if the library is missing -- there is no fallback path.
 """
 
 _BINDING_NAMES = ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_paged", "fa_bwd_stages",
-                  "fa_bwd_workspace_size",
+                  "fa_bwd_workspace_size", "fa_fwd_bwd_host", "fa_fwd_bwd_host_workspace_size",
                   "fa_dropout_mask", "fa_last_device_error", "fa_selftest_wait_timeout", "FAError", "load_library")
 
 

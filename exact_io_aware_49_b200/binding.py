@@ -65,6 +65,10 @@ def load_library(path=None):
     lib.fa_bwd_tiles.restype = i
     lib.fa_bwd_finish.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd_finish.restype = i
+    lib.fa_fwd_bwd_host_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_fwd_bwd_host_workspace_size.restype = sz
+    lib.fa_fwd_bwd_host.argtypes = [vp] * 9 + [i, i, i, i, i, f, f, u64, i, i, vp, sz, ctypes.POINTER(vp)]
+    lib.fa_fwd_bwd_host.restype = i
     lib.fa_decode_num_splits.argtypes = [i, i, i, i, i]
     lib.fa_decode_num_splits.restype = i
     lib.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
@@ -91,6 +95,11 @@ def _guard(t):
     """Makes ``t``'s device the current one for the call: the library sets kernel
     attributes and launches on the current device."""
     return torch.cuda.device(t.device)
+
+
+def _on_device(device):
+    """The same for an explicit device (calls whose tensors are on the host)."""
+    return torch.cuda.device(device)
 
 
 # element types of the ``_ex`` entry points (fa_dtype)
@@ -400,3 +409,57 @@ def fa_selftest_wait_timeout(limit_us=1000, device="cuda"):
 def fa_last_device_error():
     """Synchronises; returns the status of bounded device waits since the last call."""
     return int(load_library().fa_last_device_error())
+
+
+def _check_host(name, t, shape, dtype):
+    if t.is_cuda or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} CPU tensor of shape {tuple(shape)}")
+
+
+def fa_fwd_bwd_host_workspace_size(B, H, N, d, groups):
+    return int(load_library().fa_fwd_bwd_host_workspace_size(B, H, N, d, groups))
+
+
+def fa_fwd_bwd_host(q, k, v, do, causal, scale=None, p_drop=0.0, seed=0, groups=8, device=None, workspace=None,
+                    streams=None, out=None, lse=None, dq=None, dk=None, dv=None):
+    """Forward and backward of attention on HOST tensors (the C ABI's
+    fa_fwd_bwd_host): q, k, v, do are CPU [B, H, N, d] bf16 or fp16 tensors
+    (pin them for the copies to overlap the kernels); returns CPU
+    (O, LSE, dQ, dK, dV).  The work is cut into ``groups`` groups of (b, h)
+    units copied in, computed and copied out on three CUDA streams of
+    ``device`` (``streams``: three torch.cuda.Stream, created if omitted).
+    Returns once the work is enqueued; synchronise ``streams[2]`` (or the
+    device) before reading the outputs."""
+    lib = load_library()
+    if q.dtype not in FA_DTYPE or q.dim() != 4:
+        raise ValueError("q must be a [B, H, N, d] bf16 or fp16 tensor")
+    B, H, N, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+        _check_host(name, t, q.shape, q.dtype)
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    scale = d ** -0.5 if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32) if lse is None else lse
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_host(name, t, q.shape, q.dtype)
+    _check_host("lse", lse, (B, H, N), torch.float32)
+    ws_bytes = fa_fwd_bwd_host_workspace_size(B, H, N, d, groups)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, device=device, dtype=torch.uint8)
+    if streams is None:
+        streams = [torch.cuda.Stream(device) for _ in range(3)]
+    if len(streams) != 3:
+        raise ValueError("streams must hold three CUDA streams")
+    handles = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(st.cuda_stream) for st in streams])
+    ws, wsb = _ws_args(workspace, device)
+    if wsb < ws_bytes:
+        raise ValueError(f"workspace holds {wsb} bytes, fa_fwd_bwd_host needs {ws_bytes}")
+    with _on_device(device):
+        _raise(lib.fa_fwd_bwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                                   int(bool(causal)), float(scale), float(p_drop), int(seed) & (2**64 - 1),
+                                   FA_DTYPE[q.dtype], int(groups), ws, wsb, handles), "fa_fwd_bwd_host")
+    return out, lse, dq, dk, dv

@@ -45,13 +45,13 @@ EncodeTiledFn get_encode_fn() {
 // head with 128-byte swizzle.  Rows past T are outside the tensor: loads
 // zero-fill them, reductions skip them.
 bool encode_map(CUtensorMap* tm, const void* base, int d, long long T, long long G, long long tok, long long grp,
-                CUtensorMapDataType dt) {
+                CUtensorMapDataType dt, int box_rows = 128) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t esize = (dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32) ? 4 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(G)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(tok) * esize, static_cast<cuuint64_t>(grp) * esize};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(tm, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -89,10 +89,14 @@ fa_status check_scalars(int d, float scale, float p_drop) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
   // 32 and 96 run on the 64- and 128-column kernels: the tensor maps read the
-  // columns past d as zeros and only d columns are stored
-  if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
+  // columns past d as zeros and only d columns are stored; 192 and 256 run on
+  // the wide forward kernel (the backward and decode kernels stop at 128)
+  if (d != 32 && d != 64 && d != 96 && d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
+
+// Head dimensions the backward and decode kernels take.
+bool narrow_head(int d) { return d <= 128; }
 
 uint32_t drop_threshold(float p_drop) {
   // round-half-even(p * 65536) in double precision (default rounding mode)
@@ -109,7 +113,7 @@ struct Problem {
   uint64_t seed;
   bool f16;
   bool deterministic;  // backward: fixed order of the dQ additions
-  long long groups() const { return seq.cu_q ? seq.H : static_cast<long long>(seq.B) * seq.H; }
+  long long groups() const { return seq.cu_q ? seq.H : static_cast<long long>(seq.units); }
 };
 
 // Fixed lengths: [B, H, Nq, d] queries, [B, H, Nk, d] keys.
@@ -123,6 +127,8 @@ fa_status fixed_problem(Problem* pb, int B, int H, int Nq, int Nk, int d, int ca
   memset(pb, 0, sizeof(*pb));
   pb->seq.B = B;
   pb->seq.H = H;
+  pb->seq.units = B * H;  // < 2^31, checked above
+  pb->seq.unit0 = 0;
   pb->seq.Nq = Nq;
   pb->seq.Nk = Nk;
   pb->seq.total_q = Nq;
@@ -159,6 +165,8 @@ fa_status packed_problem(Problem* pb, const int* cu_q, const int* cu_k, int B, i
   pb->seq.cu_k = cu_k;
   pb->seq.B = B;
   pb->seq.H = H;
+  pb->seq.units = B * H;  // < 2^31, checked above
+  pb->seq.unit0 = 0;
   pb->seq.Nq = max_q;
   pb->seq.Nk = max_k;
   pb->seq.total_q = total_q;
@@ -178,11 +186,14 @@ fa_status packed_problem(Problem* pb, const int* cu_q, const int* cu_k, int B, i
 // Workspace: fp32 dQ accumulator [G, total_q, d], then the fp32 D and
 // LSE * log2(e) vectors [B * H, pad128(Nq)], then (deterministic mode only)
 // one uint32 counter per (unit, query tile), each part rounded to 256 bytes.
+size_t order_bytes(const Problem& pb) {
+  return pb.deterministic ? static_cast<size_t>(pb.seq.units) * (pad128(pb.seq.Nq) / 128) * 4 : 0;
+}
+
 size_t workspace_bytes(const Problem& pb) {
   const size_t acc = static_cast<size_t>(pb.groups()) * pb.seq.total_q * pb.d * sizeof(float);
-  const size_t vec = static_cast<size_t>(pb.seq.B) * pb.seq.H * pad128(pb.seq.Nq) * sizeof(float);
-  const size_t order = pb.deterministic ? static_cast<size_t>(pb.seq.B) * pb.seq.H * (pad128(pb.seq.Nq) / 128) * 4 : 0;
-  return round_up(acc, 256) + 2 * round_up(vec, 256) + round_up(order, 256);
+  const size_t vec = static_cast<size_t>(pb.seq.units) * pad128(pb.seq.Nq) * sizeof(float);
+  return round_up(acc, 256) + 2 * round_up(vec, 256) + round_up(order_bytes(pb), 256);
 }
 
 bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base) {
@@ -190,9 +201,9 @@ bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base) {
                     elem_type(pb.f16));
 }
 
-bool encode_k_like(const Problem& pb, CUtensorMap* tm, const void* base) {
+bool encode_k_like(const Problem& pb, CUtensorMap* tm, const void* base, int box_rows = 128) {
   return encode_map(tm, base, pb.d, pb.seq.total_k, pb.groups(), pb.seq.tok_stride, pb.seq.k_head_stride,
-                    elem_type(pb.f16));
+                    elem_type(pb.f16), box_rows);
 }
 
 void fill_common(const Problem& pb, fa::SeqLayout* seq, int* d, int* causal, float* scale_log2, uint32_t* drop_t,
@@ -215,7 +226,9 @@ fa_status fwd_run(const Problem& pb, const void* Q, const void* K, const void* V
     return FA_ERR_INVALID_ARG;
   fa::FwdArgs a;
   memset(&a, 0, sizeof(a));
-  if (!encode_q_like(pb, &a.tmQ, Q) || !encode_k_like(pb, &a.tmK, K) || !encode_k_like(pb, &a.tmV, V))
+  // the wide-head kernel streams 64-key tiles
+  const int kv_rows = narrow_head(pb.d) ? 128 : 64;
+  if (!encode_q_like(pb, &a.tmQ, Q) || !encode_k_like(pb, &a.tmK, K, kv_rows) || !encode_k_like(pb, &a.tmV, V, kv_rows))
     return FA_ERR_CUDA;
   a.f16 = pb.f16 ? 1 : 0;
   a.O = O;
@@ -228,6 +241,7 @@ fa_status fwd_run(const Problem& pb, const void* Q, const void* K, const void* V
 }
 
 fa_status check_workspace(const Problem& pb, const void* workspace, size_t bytes) {
+  if (!narrow_head(pb.d)) return FA_ERR_UNSUPPORTED;  // no backward kernel for d > 128
   if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
   if (bytes < workspace_bytes(pb)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -243,7 +257,7 @@ void bwd_args(const Problem& pb, fa::BwdArgs* a, void* workspace) {
   a->f16 = pb.f16 ? 1 : 0;
   char* ws = static_cast<char*>(workspace);
   const size_t acc = round_up(static_cast<size_t>(pb.groups()) * pb.seq.total_q * pb.d * sizeof(float), 256);
-  const size_t vec = round_up(static_cast<size_t>(pb.seq.B) * pb.seq.H * pad128(pb.seq.Nq) * sizeof(float), 256);
+  const size_t vec = round_up(static_cast<size_t>(pb.seq.units) * pad128(pb.seq.Nq) * sizeof(float), 256);
   a->dQacc = reinterpret_cast<float*>(ws);
   a->Dvec = reinterpret_cast<float*>(ws + acc);
   a->lse2 = reinterpret_cast<float*>(ws + acc + vec);
@@ -315,6 +329,47 @@ fa_status bwd_run(const Problem& pb, const void* Q, const void* K, const void* V
 
 bool dtype_ok(fa_dtype dtype) { return dtype == FA_DTYPE_BF16 || dtype == FA_DTYPE_F16; }
 
+// ------------------------------------------------------------ host-buffer step
+
+// Device layout of fa_fwd_bwd_host's workspace: kHostSlots staging slots of
+// the per-group tensors (Q, K, V, dO in; O, dQ, dK, dV out: [units, N, d]
+// 16-bit each; LSE [units, N] fp32), then the backward workspace of one group
+// (the groups run one after another on the compute stream and share it).
+constexpr int kHostSlots = 3;
+
+struct HostPlan {
+  int units_total;   // B * H
+  int per_group;     // units in each group but possibly the last
+  int groups;        // number of groups
+  size_t tensor;     // bytes of one staged [per_group, N, d] 16-bit tensor, rounded to 256
+  size_t lse;        // bytes of the staged [per_group, N] LSE, rounded to 256
+  size_t slot;       // bytes of one staging slot
+  size_t bwd;        // bytes of the shared backward workspace
+};
+
+bool host_plan(int B, int H, int N, int d, int groups, HostPlan* hp) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || groups <= 0) return false;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh >= (1ll << 31) || bh * N >= (1ll << 31)) return false;
+  hp->units_total = static_cast<int>(bh);
+  if (groups > hp->units_total) groups = hp->units_total;
+  hp->per_group = (hp->units_total + groups - 1) / groups;
+  hp->groups = (hp->units_total + hp->per_group - 1) / hp->per_group;
+  hp->tensor = round_up(static_cast<size_t>(hp->per_group) * N * d * 2, 256);
+  hp->lse = round_up(static_cast<size_t>(hp->per_group) * N * sizeof(float), 256);
+  hp->slot = 8 * hp->tensor + hp->lse;
+  Problem pb;
+  memset(&pb, 0, sizeof(pb));
+  pb.seq.B = B;
+  pb.seq.H = H;
+  pb.seq.units = hp->per_group;
+  pb.seq.Nq = N;
+  pb.seq.total_q = N;
+  pb.d = d;
+  hp->bwd = round_up(workspace_bytes(pb), 256);
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -370,10 +425,11 @@ fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, fl
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   Problem pb;
-  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || static_cast<long long>(B) * H >= (1ll << 31)) return 0;
   memset(&pb, 0, sizeof(pb));
   pb.seq.B = B;
   pb.seq.H = H;
+  pb.seq.units = B * H;
   pb.seq.Nq = N;
   pb.seq.total_q = N;
   pb.d = d;
@@ -382,10 +438,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 
 size_t fa_bwd_qk_workspace_size(int B, int H, int Nq, int d, int deterministic) {
   Problem pb;
-  if (B <= 0 || H <= 0 || Nq <= 0 || d <= 0) return 0;
+  if (B <= 0 || H <= 0 || Nq <= 0 || d <= 0 || static_cast<long long>(B) * H >= (1ll << 31)) return 0;
   memset(&pb, 0, sizeof(pb));
   pb.seq.B = B;
   pb.seq.H = H;
+  pb.seq.units = B * H;
   pb.seq.Nq = Nq;
   pb.seq.total_q = Nq;
   pb.d = d;
@@ -395,11 +452,13 @@ size_t fa_bwd_qk_workspace_size(int B, int H, int Nq, int d, int deterministic) 
 
 size_t fa_bwd_varlen_workspace_size(int B, int H, int total_q, int max_seqlen_q, int d, int deterministic) {
   Problem pb;
-  if (B <= 0 || H <= 0 || total_q <= 0 || max_seqlen_q <= 0 || d <= 0) return 0;
+  if (B <= 0 || H <= 0 || total_q <= 0 || max_seqlen_q <= 0 || d <= 0 || static_cast<long long>(B) * H >= (1ll << 31))
+    return 0;
   memset(&pb, 0, sizeof(pb));
   pb.seq.cu_q = reinterpret_cast<const int*>(1);  // packed layout: G = H
   pb.seq.B = B;
   pb.seq.H = H;
+  pb.seq.units = B * H;
   pb.seq.Nq = max_seqlen_q;
   pb.seq.total_q = total_q;
   pb.d = d;
@@ -472,6 +531,110 @@ fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void*
   return bwd_run(pb, Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, stream);
 }
 
+// ------------------------------------------------------------ host-buffer step
+
+size_t fa_fwd_bwd_host_workspace_size(int B, int H, int N, int d, int groups) {
+  HostPlan hp;
+  if (!host_plan(B, H, N, d, groups, &hp)) return 0;
+  return kHostSlots * hp.slot + hp.bwd;
+}
+
+fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const void* dO, void* O, float* LSE,
+                          void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+                          float p_drop, uint64_t seed, fa_dtype dtype, int groups, void* workspace,
+                          size_t workspace_bytes_, void* const* streams) {
+  if (!dtype_ok(dtype)) return FA_ERR_INVALID_ARG;
+  Problem whole;
+  fa_status st = fixed_problem(&whole, B, H, N, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
+  if (st != FA_OK) return st;
+  if (!narrow_head(d)) return FA_ERR_UNSUPPORTED;  // the backward stops at d = 128
+  HostPlan hp;
+  if (!host_plan(B, H, N, d, groups, &hp)) return FA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !dO || !O || !LSE || !dQ || !dK || !dV || !streams) return FA_ERR_INVALID_ARG;
+  if (!workspace || misaligned(workspace, 256) || workspace_bytes_ < kHostSlots * hp.slot + hp.bwd)
+    return FA_ERR_INVALID_ARG;
+  cudaStream_t s_in = static_cast<cudaStream_t>(streams[0]);
+  cudaStream_t s_cmp = static_cast<cudaStream_t>(streams[1]);
+  cudaStream_t s_out = static_cast<cudaStream_t>(streams[2]);
+  char* ws = static_cast<char*>(workspace);
+  char* bwd_ws = ws + kHostSlots * hp.slot;
+  const size_t row = static_cast<size_t>(N) * d * 2;  // bytes of one unit of a 16-bit tensor
+  // events: copy-in done, compute done, copy-out done, per group
+  const int ng = hp.groups;
+  cudaEvent_t* ev = new cudaEvent_t[3 * ng + 1];
+  int made = 0;
+  for (; made < 3 * ng + 1; ++made)
+    if (cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming) != cudaSuccess) break;
+  st = (made == 3 * ng + 1) ? FA_OK : FA_ERR_CUDA;
+  // the call starts after the work already on the copy-out stream (an earlier
+  // call's last copies still reading the staging slots this call refills)
+  if (st == FA_OK && (cudaEventRecord(ev[3 * ng], s_out) != cudaSuccess ||
+                      cudaStreamWaitEvent(s_in, ev[3 * ng], 0) != cudaSuccess ||
+                      cudaStreamWaitEvent(s_cmp, ev[3 * ng], 0) != cudaSuccess))
+    st = FA_ERR_CUDA;
+  const char* src_in[4] = {static_cast<const char*>(Q), static_cast<const char*>(K), static_cast<const char*>(V),
+                           static_cast<const char*>(dO)};
+  char* dst_out[4] = {static_cast<char*>(O), static_cast<char*>(dQ), static_cast<char*>(dK), static_cast<char*>(dV)};
+  for (int g = 0; st == FA_OK && g < ng; ++g) {
+    const int u0 = g * hp.per_group;
+    const int gu = (u0 + hp.per_group <= hp.units_total) ? hp.per_group : hp.units_total - u0;
+    char* slot = ws + (g % kHostSlots) * hp.slot;
+    char* in[4] = {slot, slot + hp.tensor, slot + 2 * hp.tensor, slot + 3 * hp.tensor};  // Q, K, V, dO
+    char* out[4] = {slot + 4 * hp.tensor, slot + 5 * hp.tensor, slot + 6 * hp.tensor,
+                    slot + 7 * hp.tensor};  // O, dQ, dK, dV
+    float* lse = reinterpret_cast<float*>(slot + 8 * hp.tensor);
+    cudaEvent_t ev_in = ev[3 * g], ev_cmp = ev[3 * g + 1], ev_out = ev[3 * g + 2];
+    // copy-in: the slot's inputs are free once the group that used it last has computed
+    if (g >= kHostSlots && cudaStreamWaitEvent(s_in, ev[3 * (g - kHostSlots) + 1], 0) != cudaSuccess) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    for (int k = 0; k < 4 && st == FA_OK; ++k)
+      if (cudaMemcpyAsync(in[k], src_in[k] + static_cast<size_t>(u0) * row, static_cast<size_t>(gu) * row,
+                          cudaMemcpyHostToDevice, s_in) != cudaSuccess)
+        st = FA_ERR_CUDA;
+    if (st != FA_OK || cudaEventRecord(ev_in, s_in) != cudaSuccess) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    // compute: after this group's inputs, and after the slot's outputs of the
+    // group before have been copied out
+    if (cudaStreamWaitEvent(s_cmp, ev_in, 0) != cudaSuccess ||
+        (g >= kHostSlots && cudaStreamWaitEvent(s_cmp, ev[3 * (g - kHostSlots) + 2], 0) != cudaSuccess)) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    Problem pg = whole;  // the group as a problem of gu units starting at unit u0
+    pg.seq.units = gu;
+    pg.seq.unit0 = u0;
+    if ((st = fwd_run(pg, in[0], in[1], in[2], out[0], lse, s_cmp)) != FA_OK) break;
+    if ((st = bwd_run(pg, in[0], in[1], in[2], out[0], in[3], lse, out[1], out[2], out[3], bwd_ws, hp.bwd,
+                      s_cmp)) != FA_OK)
+      break;
+    if (cudaEventRecord(ev_cmp, s_cmp) != cudaSuccess) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    // copy-out
+    if (cudaStreamWaitEvent(s_out, ev_cmp, 0) != cudaSuccess) {
+      st = FA_ERR_CUDA;
+      break;
+    }
+    for (int k = 0; k < 4 && st == FA_OK; ++k)
+      if (cudaMemcpyAsync(dst_out[k] + static_cast<size_t>(u0) * row, out[k], static_cast<size_t>(gu) * row,
+                          cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+        st = FA_ERR_CUDA;
+    if (st == FA_OK && cudaMemcpyAsync(LSE + static_cast<size_t>(u0) * N, lse, static_cast<size_t>(gu) * N * 4,
+                                       cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+      st = FA_ERR_CUDA;
+    if (st == FA_OK && cudaEventRecord(ev_out, s_out) != cudaSuccess) st = FA_ERR_CUDA;
+  }
+  // events may be destroyed while work that records them is still queued
+  for (int k = 0; k < made; ++k) cudaEventDestroy(ev[k]);
+  delete[] ev;
+  return st;
+}
+
 // ------------------------------------------------------------ decoding over a paged cache
 
 int fa_decode_num_splits(int B, int H_kv, int H, int Nq, int max_seqlen_k) {
@@ -533,6 +696,7 @@ fa_status fa_decode_paged(const void* Q, const void* K_cache, const void* V_cach
   if (static_cast<long long>(max_seqlen_k) > static_cast<long long>(max_pages_per_seq) * page_size)
     return FA_ERR_INVALID_ARG;
   fa_status st = check_scalars(d, scale, 0.0f);
+  if (st == FA_OK && !narrow_head(d)) st = FA_ERR_UNSUPPORTED;
   if (st != FA_OK) return st;
   if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(num_pages) * page_size >= (1ll << 31) ||

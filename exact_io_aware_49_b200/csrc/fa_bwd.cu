@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const uint16_t* 
                                                                 int dh, int Npad, long long acc_vec4,
                                                                 unsigned* __restrict__ dq_order, int n_order) {
   const int lane = threadIdx.x & 31;
-  const int rows_pad = seq.B * seq.H * Npad;  // < 2^31, checked on the host
+  const int rows_pad = seq.units * Npad;  // < 2^31, checked on the host
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int prow = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); prow < rows_pad; prow += warps) {
     const int unit = prow / Npad;
@@ -160,7 +160,7 @@ constexpr int kBwdLoadWarp = 9;
 // two elementwise warpgroups, the dQ-drain warpgroup, the control warpgroup.
 constexpr int kBwdLaunchRegs = 128;
 constexpr int kEwRegs = 168;
-constexpr int kDqRegs = 112;
+constexpr int kDqRegs = 120;
 constexpr int kCtlRegs = 56;
 static_assert(2 * 128 * kEwRegs + 128 * kDqRegs + 128 * kCtlRegs <= kBwdThreads * kBwdLaunchRegs, "register split");
 
@@ -282,7 +282,9 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
 }
 
 // Keep bits of the dropout mask for this lane's key row and 32 consecutive
-// queries q0 .. q0+31: bit l of the result is keep(key, q0 + l).
+// queries q0 .. q0+31: bit l of the result is keep(key, q0 + l).  ``phx``
+// holds the per-key-group part of the Philox rounds (counter words key >> 3,
+// h, b are fixed, the query varies).
 //
 // The Philox counter (key >> 3, query, h, b) yields 8 keys x 1 query per call,
 // so lane l8 of each group of 8 consecutive keys evaluates queries
@@ -294,20 +296,23 @@ __device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
 // butterfly of lane shuffles then transposes each 8 x 8 bit block so that lane
 // k' holds bit l = keep(its key, query q0 + 8 j + l).
 template <bool kHighT>
-__device__ __forceinline__ uint32_t keep_bits_32(uint32_t key_grp, uint32_t q0, uint32_t h, uint32_t b,
-                                                 const uint32_t* rk, uint32_t c2, int lane) {
+__device__ __forceinline__ uint32_t keep_bits_32(const PhiloxFixed023& phx, uint32_t q0, const uint32_t* rk,
+                                                 uint32_t c2, int lane) {
   const uint32_t l8 = static_cast<uint32_t>(lane & 7);
   uint32_t W = 0;
+  uint32_t cq[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) cq[j] = q0 + 8 * j + l8;
+  uint32_t w4[4][4];
+  philox4x32_10_c1_batch<4>(cq, phx, rk, w4);  // the 4 calls in lockstep
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint32_t w[4];
-    philox4x32_10_rk(key_grp, q0 + 8 * j + l8, h, b, rk, w);
     uint32_t acc = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const uint32_t y = (w[e] & 0x7FFF7FFFu) + c2;
-      const uint32_t zm = (kHighT ? (w[e] & y) : (w[e] | y)) & 0x80008000u;  // keep bits at 15 and 31
-      acc = mad_hi_u32(zm, 1u << (17 + 2 * e), acc);                          // -> bits 2e and 16 + 2e
+      const uint32_t y = (w4[j][e] & 0x7FFF7FFFu) + c2;
+      const uint32_t zm = (kHighT ? (w4[j][e] & y) : (w4[j][e] | y)) & 0x80008000u;  // keep bits at 15 and 31
+      acc = mad_hi_u32(zm, 1u << (17 + 2 * e), acc);                                  // -> bits 2e and 16 + 2e
     }
     W |= ((acc | (acc >> 15)) & 0xFFu) << (8 * j);
   }
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     constexpr int kCols = D / 2;       // columns per round
     constexpr int kBoxes = kCols / 32;  // 32-column fp32 boxes per round
     const int wq = warp & 3;
-    const int c = wq * 32 + lane;  // query row within the tile == TMEM lane
+    const int c = wq * 32 + lane;  // query row within the tile == TMEM lane (keep bits: key row)
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kColDP;
     const bool leader = threadIdx.x == 12 * 32;
     volatile int* go = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
@@ -583,22 +588,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = wq * 32 + lane;  // key row within the tile == TMEM lane
     const uint32_t t_row = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
+    const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
     const DropConst dk = make_drop_const(p.drop_t);
     const bool hi_t = p.drop_t > 0x8000u;
-    const uint32_t hh = static_cast<uint32_t>(su.h), bb = static_cast<uint32_t>(su.b);
-    const uint32_t key_grp = static_cast<uint32_t>((kj * 128 + r) >> 3);
-    const uint32_t ds_row = sm_ds + g * L::kBox + r * 128;
-    // keep bits of this thread's 64 query columns for the coming query tile;
-    // computed one tile ahead, while the warp would otherwise wait for S^T
-    uint32_t zb[2] = {0u, 0u};
-    auto keep_bits_tile = [&](int qi_next) {
-      const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g);
-#pragma unroll
-      for (int half = 0; half < 2; ++half)
-        zb[half] = hi_t ? keep_bits_32<true>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane)
-                        : keep_bits_32<false>(key_grp, q0 + 32 * half, hh, bb, p.philox_rk, dk.c2, lane);
+    const PhiloxFixed023 phx = philox_fix023(static_cast<uint32_t>((kj * 128 + r) >> 3), static_cast<uint32_t>(su.h),
+                                             static_cast<uint32_t>(su.b), p.philox_rk);
+    uint32_t zbn[2] = {0u, 0u};
+    auto keep_half = [&](int qi_next, int half) {
+      const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g + 32 * half);
+      zbn[half] = hi_t ? keep_bits_32<true>(phx, q0, p.philox_rk, dk.c2, lane)
+                       : keep_bits_32<false>(phx, q0, p.philox_rk, dk.c2, lane);
     };
-    if (DROPOUT) keep_bits_tile(qi_of(0));
+    // keep bits of this thread's 64 query columns, computed one tile ahead
+    // (at the end of the previous tile, while the warp would wait for S^T)
+    if (DROPOUT) {
+      keep_half(qi_of(0), 0);
+      keep_half(qi_of(0), 1);
+    }
     // masking: query i = qi * 128 + c sees this thread's key j = kj * 128 + r
     // iff i + Nk - Nq >= j, i.e. c >= lo0 - qi * 128; query tiles up to qi_mask
     // hold such pairs for some key of the tile; a tile past the unit's last
@@ -612,6 +618,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int qi = qi_of(it);
       if (!mbar_wait(&bars[kQFull0 + s], (it >> 1) & 1, abort_flag, p.err) ||
           !mbar_wait(&bars[kSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+      const uint32_t zb[2] = {zbn[0], zbn[1]};
       tc_fence_after();
       uint32_t sr[64];
       tmem_ld32(t_row + kColS + 64 * g, sr);
@@ -690,7 +697,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kDSReady]);
-      if (DROPOUT && it + 1 < nq) keep_bits_tile(qi_of(it + 1));
+      if (DROPOUT && it + 1 < nq) {
+        keep_half(qi_of(it + 1), 0);
+        keep_half(qi_of(it + 1), 1);
+      }
     }
     if (ok && mbar_wait(&bars[kDKDVReady], 0, abort_flag, p.err)) {
       // -------------------------------------------------------------- dK / dV epilogue
@@ -754,7 +764,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
   for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
-  p.BH = a.seq.B * a.seq.H;
+  p.BH = a.seq.units;
   const int n_kt = (a.seq.Nk + 127) / 128;
   {
     // units per group: about 512 key-tile work units per group; the CTAs
@@ -771,7 +781,7 @@ cudaError_t launch_bwd_main(const BwdArgs& a, cudaStream_t stream) {
 
 template <bool F16>
 void launch_preprocess_typed(const BwdArgs& a, long long blocks, int Npad, long long acc_vec4, cudaStream_t stream) {
-  const int n_order = a.dq_order ? a.seq.B * a.seq.H * (Npad / 128) : 0;
+  const int n_order = a.dq_order ? a.seq.units * (Npad / 128) : 0;
   const uint16_t* O = static_cast<const uint16_t*>(a.O);
   const uint16_t* dO = static_cast<const uint16_t*>(a.dO);
   if (a.d <= 64)
@@ -803,8 +813,8 @@ cudaError_t launch_bwd_tiles_typed(const BwdArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream) {
   const int Npad = (a.seq.Nq + 127) / 128 * 128;
-  const long long rows_pad = static_cast<long long>(a.seq.B) * a.seq.H * Npad;
-  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.B) * a.seq.H;
+  const long long rows_pad = static_cast<long long>(a.seq.units) * Npad;
+  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.units);
   const long long acc_vec4 = groups * a.seq.total_q * a.d / 4;
   long long blocks = (rows_pad + 7) / 8;  // one warp per row, 8 warps per block
   if (blocks > 148 * 16) blocks = 148 * 16;
@@ -825,7 +835,7 @@ cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream) {
-  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.B) * a.seq.H;
+  const long long groups = a.seq.cu_q ? a.seq.H : static_cast<long long>(a.seq.units);
   const long long n8 = groups * a.seq.total_q * a.d / 8;
   long long blocks = (n8 + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;

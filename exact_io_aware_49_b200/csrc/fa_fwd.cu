@@ -45,8 +45,41 @@
 #include "philox.cuh"
 #include "sm100.cuh"
 
+#ifndef FA_FWD_KEEP_FMT
+#define FA_FWD_KEEP_FMT 0  // 0: 4 packed words a row, 1: 32 words (byte signs)
+#endif
+#ifndef FA_FWD_DRAW_NB
+#define FA_FWD_DRAW_NB 8
+#endif
+
 namespace fa {
 namespace {
+
+// byte-sign format: kz[m] holds pair 2m's keep bits in the signs of bytes 0, 1
+// and pair 2m + 1's in bytes 2, 3
+template <bool kHighT, int kNB>
+__device__ __forceinline__ void draw_keep_bytes(uint32_t jb0, const PhiloxFixed123& f, const uint32_t* rk,
+                                                uint32_t c2, uint32_t (&kz)[32]) {
+#pragma unroll
+  for (int g0 = 0; g0 < 16; g0 += kNB) {
+    uint32_t w[kNB][4];
+    if (kNB == 1)
+      philox4x32_10_c0(jb0 + g0, f, rk, w[0]);
+    else
+      philox4x32_10_c0_batch<kNB>(jb0 + g0, f, rk, w);
+#pragma unroll
+    for (int n = 0; n < kNB; ++n) {
+      uint32_t z[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t y = (w[n][e] & 0x7FFF7FFFu) + c2;
+        z[e] = kHighT ? (w[n][e] & y) : (w[n][e] | y);
+      }
+      kz[2 * (g0 + n)] = prmt(z[0], z[1], 0x7531u);
+      kz[2 * (g0 + n) + 1] = prmt(z[2], z[3], 0x7531u);
+    }
+  }
+}
 
 constexpr int kBM = 128;             // query rows per tile
 constexpr int kBN = 128;             // keys per tile
@@ -326,11 +359,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t t_s = t_lane + q * 128;
       const uint32_t t_o = t_lane + 256 + q * D;
       const float sl2 = p.scale_log2;
-      // keep test on the FMA pipe: for a 16-bit draw u, the float 2^23 + u is
-      // exact, and sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0
-      const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
-      const int h = su.h;
-      const int b = su.b;
+      // dropout: the Philox counter of this row is (j >> 3, i, h, b); the
+      // parts of its first two rounds that do not depend on j are fixed here
+      const PhiloxFixed123 phx = philox_fix123(static_cast<uint32_t>(i), static_cast<uint32_t>(su.h),
+                                               static_cast<uint32_t>(su.b), p.philox_rk);
+      const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
+      const bool hi_t = p.drop_t > 0x8000u;
       // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
       // last key, and under the causal mask the row's position i + Nk - Nq);
       // tiles from t_mask on are the first that can hold a masked key for
@@ -340,9 +374,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (CAUSAL) t_mask = min(t_mask, max(0, floor_div((qt0 + q) * kBM + delta - (kBN - 1), kBN) + 1));
       float m = -CUDART_INF_F;  // running max of scale*log2(e)*S, possibly stale
       float l = 0.f;            // running sum of exp2(x - m)
+      // running sum of (p - p rounded to 16 bits) over the largest P of each
+      // tile: l - lc is the sum the rounded P actually carry into O (exact
+      // for the elements that dominate a row), while l itself gives LSE
+      float lc = 0.f;
       bool ok = true;
       const int ntq = q ? nt1 : nt0;
       for (int t = 0; t < ntq; ++t) {
+        // keep bits of the tile's 128 keys, drawn before S is ready: while the
+        // tensor core computes S the warp would only wait, and the 16 Philox
+        // calls run 8 at a time in lockstep (the S row's registers are free)
+#if FA_FWD_KEEP_FMT == 0
+        uint32_t W[4] = {0u, 0u, 0u, 0u};
+        if (DROPOUT) {
+          if (hi_t)
+            draw_keep_words<true, kBN / 8>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, W);
+          else
+            draw_keep_words<false, kBN / 8>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, W);
+          asm volatile("" : "+r"(W[0]), "+r"(W[1]), "+r"(W[2]), "+r"(W[3]));  // not sunk past the wait
+        }
+#else
+        uint32_t kz[32];
+        if (DROPOUT) {
+          if (hi_t)
+            draw_keep_bytes<true, FA_FWD_DRAW_NB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
+          else
+            draw_keep_bytes<false, FA_FWD_DRAW_NB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
+          reg_fence32(kz);
+        }
+#endif
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -373,68 +433,69 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mx3 = max3f(mx3, s[c + 6], s[c + 7]);
         }
         static_assert(kBN % 8 == 0, "row max covers the tile in steps of 8");
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const float s_max = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_tile = s_max * sl2;
         const float m_new = fmaxf(m, m_tile);
-        if (__any_sync(0xffffffffu, m_new > m + kRescaleTau)) {
-          const float alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
+        // lazy rescale: the warp moves to the new maximum only when some row's
+        // maximum grew by more than kRescaleTau (warp-uniform decision)
+        const bool rescale = __any_sync(0xffffffffu, m_new > m + kRescaleTau);
+        float alpha = 1.f;
+        if (rescale) {
+          alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
           l *= alpha;
-          if (t > 0) {
-            // O accumulator of this row: all earlier PV MMAs completed before S_t was committed
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t orow[32];
-              tmem_ld32(t_o + c * 32, orow);
-              tmem_ld_wait();
-              reg_fence32(orow);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-              tmem_st32(t_o + c * 32, orow);
-            }
-          }
+          lc *= alpha;
           m = m_new;
         }
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         // a row that has seen no key yet keeps m = -inf: its P is exp2(-inf) = 0
         const float m_use = (m == -CUDART_INF_F) ? 0.f : m;
+        {
+          // the tile's largest P, computed exactly as in the loop below, minus
+          // its 16-bit rounding (0 when the whole tile is masked for this row)
+          const float p_top = ex2_approx(fmaf(s_max, sl2, -m_use));
+          lc += p_top - unpack2<F16>(pack2<F16>(p_top, 0.f)).x;
+        }
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
 #pragma unroll
-        for (int g = 0; g < kBN / 8; ++g) {
-          uint32_t w[4];
-          if (DROPOUT)
-            philox4x32_10_rk(static_cast<uint32_t>(t * (kBN / 8) + g), static_cast<uint32_t>(i),
-                             static_cast<uint32_t>(h), static_cast<uint32_t>(b), p.philox_rk, w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * g + e;
-            float x0, x1;
-            f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
-            uint64_t pp = f2_pack(p0, p1);
-            if (e & 1)
-              rs1 = add_f2(rs1, pp);
-            else
-              rs0 = add_f2(rs0, pp);
-            if (DROPOUT) {
-              // keep = sat((2^23 + u16) - (2^23 + t - 1)): exactly 1.0 if u16 >= t, else 0.0
-              const float u0 = __uint_as_float(prmt(w[e], 0x4B000000u, 0x7610u));
-              const float u1 = __uint_as_float(prmt(w[e], 0x4B000000u, 0x7632u));
-              float k0, k1;
-              asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k0) : "f"(u0), "f"(drop_bias));
-              asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(u1), "f"(drop_bias));
-              pp = mul_f2(pp, f2_pack(k0, k1));
-            }
-            float q0, q1;
-            f2_unpack(pp, q0, q1);
-            pk[c] = pack2<F16>(q0, q1);
-          }
+        for (int c = 0; c < kBN / 2; ++c) {
+          float x0, x1;
+          f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          const uint64_t pp = f2_pack(p0, p1);
+          if (c & 1)
+            rs1 = add_f2(rs1, pp);
+          else
+            rs0 = add_f2(rs0, pp);
+          pk[c] = pack2<F16>(p0, p1);
+          // dropped keys: zero the 16-bit P (the row sum l keeps them)
+#if FA_FWD_KEEP_FMT == 0
+          if (DROPOUT) pk[c] &= keep_mask_pair(W, c);
+#else
+          if (DROPOUT) pk[c] &= prmt(kz[c >> 1], 0u, (c & 1) ? 0xBBAAu : 0x9988u);
+#endif
         }
         {
           float a0, a1;
           f2_unpack(add_f2(rs0, rs1), a0, a1);
           l += a0 + a1;
+        }
+        if (rescale && t > 0) {
+          // O accumulator of this row, after the S row is consumed (fewer live
+          // registers); every earlier PV MMA completed before S_t was committed
+          // and the next one waits for p_ready
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orow[32];
+            tmem_ld32(t_o + c * 32, orow);
+            tmem_ld_wait();
+            reg_fence32(orow);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+            tmem_st32(t_o + c * 32, orow);
+          }
         }
         tmem_st32(t_s, pk);
         tmem_st32(t_s + 32, pk + 32);
@@ -462,7 +523,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ---------------------------------------------------------- epilogue
         tc_fence_after();
         // l = 0: the row saw no key (O = 0, LSE = -inf)
-        const float inv = (l > 0.f) ? p.drop_scale / l : 0.f;
+        // O is normalised by the sum of the P it was built from (l - lc),
+        // the LSE by the exact sum l
+        const float inv = (l > 0.f) ? p.drop_scale / (l - lc) : 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -508,7 +571,7 @@ cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t stream) {
   p.drop_t = a.drop_t;
   p.drop_scale = a.drop_scale;
   for (int r = 0; r < 20; ++r) p.philox_rk[r] = a.philox_rk[r];
-  p.BH = a.seq.B * a.seq.H;
+  p.BH = a.seq.units;
   const int n_qb = ((a.seq.Nq + kBM - 1) / kBM + 1) / 2;
   {
     // units per group: about 256 work units (~2 waves on 148 SMs) per group,
@@ -539,6 +602,7 @@ cudaError_t launch_fwd_typed(const FwdArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream) {
+  if (a.d > 128) return launch_fwd_wide(a, stream);  // head dimensions 192 and 256 (fa_fwd_wide.cu)
   return a.f16 ? launch_fwd_typed<true>(a, stream) : launch_fwd_typed<false>(a, stream);
 }
 

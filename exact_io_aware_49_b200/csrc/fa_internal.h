@@ -9,7 +9,10 @@
 namespace fa {
 
 // Where the rows of one (sequence, head) unit live.  Units are numbered
-// b * H + h.
+// b * H + h; a launch processes ``units`` of them starting at ``unit0`` (a
+// fixed-length problem split into groups of heads: the tensors then hold only
+// the group, and unit0 keeps (b, h) -- and with them the dropout counters --
+// those of the whole problem).
 //  * Fixed length (cu_q == nullptr): every unit has Nq queries and Nk keys;
 //    tensors are [B, H, N, d], so a unit's tokens are contiguous rows and the
 //    head coordinate of unit u is u itself.
@@ -22,6 +25,8 @@ struct SeqLayout {
   const int* cu_q;
   const int* cu_k;
   int B, H;
+  int units;  // units this launch processes (B * H unless split into groups)
+  int unit0;  // global number of the first of them (0 for packed layouts)
   int Nq, Nk;
   int total_q, total_k;         // rows per head coordinate (fixed: Nq, Nk)
   long long tok_stride;         // elements between consecutive tokens of one head
@@ -42,8 +47,9 @@ struct SeqUnit {
 // rows but never an access outside the tensors or the workspace.
 __device__ __forceinline__ SeqUnit resolve_unit(const SeqLayout& L, int unit) {
   SeqUnit u;
-  u.b = unit / L.H;
-  u.h = unit - u.b * L.H;
+  const int gu = unit + L.unit0;
+  u.b = gu / L.H;
+  u.h = gu - u.b * L.H;
   if (L.cu_q) {
     const int qa = min(max(L.cu_q[u.b], 0), L.total_q);
     const int qb = min(max(L.cu_q[u.b + 1], qa), L.total_q);
@@ -141,6 +147,9 @@ int decode_rows_per_cta();
 int decode_keys_per_tile();
 
 cudaError_t launch_fwd(const FwdArgs& a, cudaStream_t stream);
+// Head dimensions 192 and 256: one 128-row query tile per CTA, 64-key K/V tiles
+// (the K and V tensor maps then have 64-row boxes).
+cudaError_t launch_fwd_wide(const FwdArgs& a, cudaStream_t stream);
 // The three backward stages; fa_bwd runs them in this order.  Only the fields
 // each stage reads need to be set.
 cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream);  // O, dO, LSE -> Dvec, lse2, dQacc = 0

@@ -68,6 +68,196 @@ __device__ __forceinline__ void philox4x32_10_rk(uint32_t c0, uint32_t c1, uint3
   out[3] = c3;
 }
 
+// Philox4x32-10 for calls that share counter words c1, c2, c3 and differ in
+// c0 only (one query row of one head: counter (j >> 3, i, h, b)).  With c2
+// fixed, round 0's second product is the same for every call, and so is round
+// 1's first product (its operand is round 0's new c0 = hi(M1 c2) ^ c1 ^ k0);
+// the per-row part of both rounds is precomputed once:
+//   a2 = c3 ^ k1(0)                       (round 0: c2' = hi(M0 c0) ^ a2)
+//   a3 = lo(M1 c2) ^ k0(1)                (round 1: c0'' = hi(M1 c2') ^ a3)
+//   a4 = hi(M0 c0') ^ k1(1), b1 = lo(M0 c0')   (round 1: c2'' = lo(M0 c0) ^ a4, c3'' = b1)
+// so a call costs 18 multiplies instead of 20 and gives the same words.
+struct PhiloxFixed123 {
+  uint32_t a2, a3, a4, b1;
+};
+
+__device__ __forceinline__ PhiloxFixed123 philox_fix123(uint32_t c1, uint32_t c2, uint32_t c3, const uint32_t* rk) {
+  const uint32_t c0r0 = __umulhi(kPhiloxM1, c2) ^ c1 ^ rk[0];  // round 0's new c0 (fixed)
+  PhiloxFixed123 f;
+  f.a2 = c3 ^ rk[1];
+  f.a3 = (kPhiloxM1 * c2) ^ rk[2];
+  f.a4 = __umulhi(kPhiloxM0, c0r0) ^ rk[3];
+  f.b1 = kPhiloxM0 * c0r0;
+  return f;
+}
+
+__device__ __forceinline__ void philox4x32_10_c0(uint32_t c0, const PhiloxFixed123& f, const uint32_t* rk,
+                                                 uint32_t (&out)[4]) {
+  // round 0 (the c2 product is folded into f)
+  const uint32_t x2 = __umulhi(kPhiloxM0, c0) ^ f.a2;
+  const uint32_t x3 = kPhiloxM0 * c0;
+  // round 1 (the c0 product is folded into f)
+  uint32_t y0 = __umulhi(kPhiloxM1, x2) ^ f.a3;
+  uint32_t y1 = kPhiloxM1 * x2;
+  uint32_t y2 = x3 ^ f.a4;
+  uint32_t y3 = f.b1;
+#pragma unroll
+  for (int r = 2; r < 10; ++r) {
+    const uint32_t hi0 = __umulhi(kPhiloxM0, y0);
+    const uint32_t lo0 = kPhiloxM0 * y0;
+    const uint32_t hi1 = __umulhi(kPhiloxM1, y2);
+    const uint32_t lo1 = kPhiloxM1 * y2;
+    y0 = hi1 ^ y1 ^ rk[2 * r];
+    y1 = lo1;
+    y2 = hi0 ^ y3 ^ rk[2 * r + 1];
+    y3 = lo0;
+  }
+  out[0] = y0;
+  out[1] = y1;
+  out[2] = y2;
+  out[3] = y3;
+}
+
+// kNB calls of philox4x32_10_c0 (counters c0, c0 + 1, ..., c0 + kNB - 1)
+// computed round by round in lockstep: the kNB independent multiply chains are
+// written interleaved, so they overlap in the multiplier pipeline instead of
+// running one after another at its latency.
+template <int kNB>
+__device__ __forceinline__ void philox4x32_10_c0_batch(uint32_t c0, const PhiloxFixed123& f, const uint32_t* rk,
+                                                       uint32_t (&out)[kNB][4]) {
+  uint32_t y0[kNB], y1[kNB], y2[kNB], y3[kNB];
+#pragma unroll
+  for (int n = 0; n < kNB; ++n) {
+    const uint32_t x2 = __umulhi(kPhiloxM0, c0 + n) ^ f.a2;  // round 0
+    const uint32_t x3 = kPhiloxM0 * (c0 + n);
+    y0[n] = __umulhi(kPhiloxM1, x2) ^ f.a3;  // round 1
+    y1[n] = kPhiloxM1 * x2;
+    y2[n] = x3 ^ f.a4;
+    y3[n] = f.b1;
+  }
+#pragma unroll
+  for (int r = 2; r < 10; ++r) {
+#pragma unroll
+    for (int n = 0; n < kNB; ++n) {
+      const uint32_t hi0 = __umulhi(kPhiloxM0, y0[n]);
+      const uint32_t lo0 = kPhiloxM0 * y0[n];
+      const uint32_t hi1 = __umulhi(kPhiloxM1, y2[n]);
+      const uint32_t lo1 = kPhiloxM1 * y2[n];
+      y0[n] = hi1 ^ y1[n] ^ rk[2 * r];
+      y1[n] = lo1;
+      y2[n] = hi0 ^ y3[n] ^ rk[2 * r + 1];
+      y3[n] = lo0;
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < kNB; ++n) {
+    out[n][0] = y0[n];
+    out[n][1] = y1[n];
+    out[n][2] = y2[n];
+    out[n][3] = y3[n];
+  }
+}
+
+// Philox4x32-10 for calls that share counter words c0, c2, c3 and differ in
+// c1 only (one key group of one head: counter (j >> 3, i, h, b) over queries
+// i).  Round 0 then has no varying product (its new c0 is c1 ^ e0), round 1
+// has one (M0 times that c0) and round 2 one (M1 times round 1's new c2); the
+// per-key-group parts are precomputed once:
+//   e0 = hi(M1 c2) ^ k0(0)                   (round 0: c0' = c1 ^ e0)
+//   f2 = lo(M0 c0) ^ k1(1)                   (round 1: c2'' = hi(M0 c0') ^ f2)
+//   f3 = lo(M1 (hi(M0 c0) ^ c3 ^ k1(0))) ^ k0(2)     (round 2: c0 = hi(M1 c2'') ^ f3)
+//   f4 = hi(M0 (hi(M1 c2') ^ lo(M1 c2) ^ k0(1))) ^ k1(2), g1 = lo(M0 ...)
+// so a call costs 16 multiplies instead of 20 and gives the same words.
+struct PhiloxFixed023 {
+  uint32_t e0, f2, f3, f4, g1;
+};
+
+__device__ __forceinline__ PhiloxFixed023 philox_fix023(uint32_t c0, uint32_t c2, uint32_t c3, const uint32_t* rk) {
+  // round 0: c1' = lo(M1 c2), c2' = hi(M0 c0) ^ c3 ^ k1(0), c3' = lo(M0 c0) (all fixed)
+  const uint32_t r0c1 = kPhiloxM1 * c2;
+  const uint32_t r0c2 = __umulhi(kPhiloxM0, c0) ^ c3 ^ rk[1];
+  const uint32_t r0c3 = kPhiloxM0 * c0;
+  // round 1: c0'' = hi(M1 c2') ^ c1' ^ k0(1), c1'' = lo(M1 c2') (fixed)
+  const uint32_t r1c0 = __umulhi(kPhiloxM1, r0c2) ^ r0c1 ^ rk[2];
+  const uint32_t r1c1 = kPhiloxM1 * r0c2;
+  PhiloxFixed023 f;
+  f.e0 = __umulhi(kPhiloxM1, c2) ^ rk[0];
+  f.f2 = r0c3 ^ rk[3];
+  f.f3 = r1c1 ^ rk[4];
+  // round 2: c2 = hi(M0 c0'') ^ c3'' ^ k1(2), c3 = lo(M0 c0'') (the product is fixed)
+  f.f4 = __umulhi(kPhiloxM0, r1c0) ^ rk[5];
+  f.g1 = kPhiloxM0 * r1c0;
+  return f;
+}
+
+__device__ __forceinline__ void philox4x32_10_c1(uint32_t c1, const PhiloxFixed023& f, const uint32_t* rk,
+                                                 uint32_t (&out)[4]) {
+  // round 0: no varying product
+  const uint32_t x0 = c1 ^ f.e0;
+  // round 1: M0 x0 varies
+  const uint32_t y2 = __umulhi(kPhiloxM0, x0) ^ f.f2;
+  const uint32_t y3 = kPhiloxM0 * x0;
+  // round 2: M1 y2 varies
+  uint32_t z0 = __umulhi(kPhiloxM1, y2) ^ f.f3;
+  uint32_t z1 = kPhiloxM1 * y2;
+  uint32_t z2 = y3 ^ f.f4;
+  uint32_t z3 = f.g1;
+#pragma unroll
+  for (int r = 3; r < 10; ++r) {
+    const uint32_t hi0 = __umulhi(kPhiloxM0, z0);
+    const uint32_t lo0 = kPhiloxM0 * z0;
+    const uint32_t hi1 = __umulhi(kPhiloxM1, z2);
+    const uint32_t lo1 = kPhiloxM1 * z2;
+    z0 = hi1 ^ z1 ^ rk[2 * r];
+    z1 = lo1;
+    z2 = hi0 ^ z3 ^ rk[2 * r + 1];
+    z3 = lo0;
+  }
+  out[0] = z0;
+  out[1] = z1;
+  out[2] = z2;
+  out[3] = z3;
+}
+
+// kNB calls of philox4x32_10_c1 with counter words c1[n], in lockstep (see
+// philox4x32_10_c0_batch).
+template <int kNB>
+__device__ __forceinline__ void philox4x32_10_c1_batch(const uint32_t (&c1)[kNB], const PhiloxFixed023& f,
+                                                       const uint32_t* rk, uint32_t (&out)[kNB][4]) {
+  uint32_t z0[kNB], z1[kNB], z2[kNB], z3[kNB];
+#pragma unroll
+  for (int n = 0; n < kNB; ++n) {
+    const uint32_t x0 = c1[n] ^ f.e0;                        // round 0
+    const uint32_t y2 = __umulhi(kPhiloxM0, x0) ^ f.f2;      // round 1
+    const uint32_t y3 = kPhiloxM0 * x0;
+    z0[n] = __umulhi(kPhiloxM1, y2) ^ f.f3;                  // round 2
+    z1[n] = kPhiloxM1 * y2;
+    z2[n] = y3 ^ f.f4;
+    z3[n] = f.g1;
+  }
+#pragma unroll
+  for (int r = 3; r < 10; ++r) {
+#pragma unroll
+    for (int n = 0; n < kNB; ++n) {
+      const uint32_t hi0 = __umulhi(kPhiloxM0, z0[n]);
+      const uint32_t lo0 = kPhiloxM0 * z0[n];
+      const uint32_t hi1 = __umulhi(kPhiloxM1, z2[n]);
+      const uint32_t lo1 = kPhiloxM1 * z2[n];
+      z0[n] = hi1 ^ z1[n] ^ rk[2 * r];
+      z1[n] = lo1;
+      z2[n] = hi0 ^ z3[n] ^ rk[2 * r + 1];
+      z3[n] = lo0;
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < kNB; ++n) {
+    out[n][0] = z0[n];
+    out[n][1] = z1[n];
+    out[n][2] = z2[n];
+    out[n][3] = z3[n];
+  }
+}
+
 __host__ __device__ inline void philox_round_keys(uint64_t seed, uint32_t (&rk)[20]) {
   uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
   for (int r = 0; r < 10; ++r) {
@@ -103,6 +293,54 @@ __device__ __forceinline__ uint32_t keep_mask_2x16(uint32_t w, DropConst k) {
   const uint32_t y = a + k.c2;
   const uint32_t z = (w & y) | ((w | y) & k.m0);
   return prmt(z, 0u, 0xBB99u);
+}
+
+
+// Keep bits of one query row for the 8 * kCalls keys j0 .. j0 + 8 kCalls - 1
+// of a tile (jb0 = j0 / 8), packed into kCalls / 4 words: one Philox call per
+// 8 keys (counter words c1, c2, c3 of the row fixed in ``f``).  The 16-bit
+// pair c of the row's P (keys j0 + 2c, j0 + 2c + 1) uses the low and high half
+// of word c & 3 of call c >> 2; the two-lane test leaves their keep bits at
+// bits 15 and 31.  Pair c = 16 k + 2 s + e is stored in word k at bits
+// 15 - s - 8 e and 31 - s - 8 e (a multiply-high shifts and adds), so that
+// after a left shift by s its bits are the sign bits of bytes 1 and 3 (e = 0)
+// or 0 and 2 (e = 1), which PRMT's sign-replicate mode turns into a 0 / 0xFFFF
+// mask per 16-bit lane (keep_mask_pair).
+template <bool kHighT, int kCalls>
+__device__ __forceinline__ void draw_keep_words(uint32_t jb0, const PhiloxFixed123& f, const uint32_t* rk,
+                                                uint32_t c2, uint32_t (&W)[kCalls / 4]) {
+  static_assert(kCalls % 4 == 0, "four calls per packed word");
+#ifdef FA_FWD_DRAW_NB
+  constexpr int kNB = (kCalls < FA_FWD_DRAW_NB) ? kCalls : FA_FWD_DRAW_NB;
+#else
+  constexpr int kNB = (kCalls < 8) ? kCalls : 8;  // calls in flight together
+#endif
+#pragma unroll
+  for (int k = 0; k < kCalls / 4; ++k) W[k] = 0u;
+#pragma unroll
+  for (int g0 = 0; g0 < kCalls; g0 += kNB) {
+    uint32_t w[kNB][4];
+    philox4x32_10_c0_batch<kNB>(jb0 + g0, f, rk, w);
+#pragma unroll
+    for (int n = 0; n < kNB; ++n) {
+      const int g = g0 + n;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        // bit 15 / 31: the low / high 16-bit draw is >= t (see keep_mask_2x16)
+        const uint32_t y = (w[n][e] & 0x7FFF7FFFu) + c2;
+        const uint32_t zm = (kHighT ? (w[n][e] & y) : (w[n][e] | y)) & 0x80008000u;
+        const int sh = 2 * (g & 3) + (e >> 1) + 8 * (e & 1);
+        W[g >> 2] = (sh == 0) ? (W[g >> 2] | zm) : mad_hi_u32(zm, 1u << (32 - sh), W[g >> 2]);
+      }
+    }
+  }
+}
+
+// 0 / 0xFFFF lane mask of 16-bit pair c from the packed keep words.
+template <int kWords>
+__device__ __forceinline__ uint32_t keep_mask_pair(const uint32_t (&W)[kWords], int c) {
+  const int cc = c & 15;
+  return prmt(W[c >> 4] << (cc >> 1), 0u, (cc & 1) ? 0xAA88u : 0xBB99u);
 }
 
 }  // namespace fa

@@ -268,6 +268,44 @@ fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const
                         size_t workspace_bytes, void* stream);
 
 /*
+ * One training step of attention (forward, then backward) on HOST buffers,
+ * with the host<->device copies overlapped with the kernels.  The pages ask
+ * that end-to-end throughput, not only kernel speed, be measured ("Flash
+ * Attention" glossary, Practical Limits and Common Pitfalls); this call is
+ * that end-to-end path.
+ *   Q, K, V, dO : host, [B, H, N, d] of ``dtype``, contiguous (page-locked for
+ *                 the copies to overlap; pageable memory works but serialises)
+ *   O, LSE      : host outputs, [B, H, N, d] and fp32 [B, H, N]
+ *   dQ, dK, dV  : host outputs, [B, H, N, d]
+ *   groups      : the B*H (b, h) units are cut into this many groups of
+ *                 consecutive units (at most B*H; a smaller last group);
+ *                 group g is copied in on streams[0], computed (fa_fwd and
+ *                 the three backward stages, the same kernels and results as
+ *                 fa_fwd / fa_bwd) on streams[1] and copied out on
+ *                 streams[2], so group g+1's copy-in and group g-1's copy-out
+ *                 overlap group g's kernels.  Dropout counters keep the whole
+ *                 problem's (b, h).
+ *   workspace   : device, 256-byte aligned, at least
+ *                 fa_fwd_bwd_host_workspace_size(B, H, N, d, groups) bytes:
+ *                 three staging slots of one group's tensors plus one
+ *                 group's backward workspace.  Caller-owned.
+ *   streams     : three CUDA streams (cudaStream_t), copy-in, compute,
+ *                 copy-out; the same stream may be given more than once (the
+ *                 step then runs without overlap).
+ * Everything is enqueued asynchronously and starts after the work already
+ * enqueued on streams[2] (so calls in a row on the same streams reuse the
+ * staging slots safely); the outputs are complete when streams[2] has
+ * reached the end of this call's work (synchronise it).
+ * Validation as fa_bwd (FA_ERR_INVALID_ARG for null pointers, groups <= 0, a
+ * workspace too small or misaligned, an unknown dtype).
+ */
+size_t fa_fwd_bwd_host_workspace_size(int B, int H, int N, int d, int groups);
+fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const void* dO, void* O, float* LSE,
+                          void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal, float scale,
+                          float p_drop, uint64_t seed, fa_dtype dtype, int groups, void* workspace,
+                          size_t workspace_bytes, void* const* streams);
+
+/*
  * Backward pass for callers that cannot allocate device memory.  (The pages
  * have no counterpart: this is an integration convenience of this library.)
  * Some callers may not call cudaMalloc at all -- a plugin running inside a

@@ -3,6 +3,7 @@ every entry point include/*.h declares, and rejects bad arguments before it
 makes any CUDA call.  Every call here carries at least one invalid argument,
 so nothing is ever launched."""
 
+import ctypes
 import glob
 import os
 import re
@@ -63,11 +64,23 @@ def _fwd(lib, Q=A, K=A, V=A, O=A, L=A, B=1, H=1, N=128, d=64, causal=0, scale=0.
     (dict(B=0), 1), (dict(H=-1), 1), (dict(N=0), 1), (dict(d=0), 1),
     (dict(p=1.0), 1), (dict(p=-0.1), 1), (dict(p=float("nan")), 1),
     (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("inf")), 1),
-    (dict(d=48), 2), (dict(d=80), 2), (dict(d=256), 2),
+    (dict(d=48), 2), (dict(d=80), 2), (dict(d=160), 2), (dict(d=512), 2),
     (dict(B=1 << 16, H=1 << 8, N=1 << 7), 2),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, want):
     assert _fwd(lib, **kw) == want
+
+
+@pytest.mark.parametrize("d", [192, 256])
+def test_wide_heads_forward_only(lib, d):
+    """d = 192 / 256 pass the forward's validation (a null output still stops
+    the call first); the backward, the host-buffer step and the decode reject
+    them as unsupported."""
+    assert _fwd(lib, d=d, O=0) == 1
+    ws = lib.fa_bwd_workspace_size(1, 1, 128, d)
+    assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, A, ws, None) == 2
+    st = (ctypes.c_void_p * 3)()
+    assert lib.fa_fwd_bwd_host(A, A, A, A, A, A, A, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, 0, 1, A, 1 << 40, st) == 2
 
 
 def _bwd(lib, ws=A, ws_bytes=None, B=1, H=1, N=128, d=64, p=0.0, **ptrs):

@@ -17,7 +17,7 @@ bf16, f16, f32, i32, u8 = torch.bfloat16, torch.float16, torch.float32, torch.in
 
 # calls that compute sizes on the host; the recorder forwards them to the real library
 _HOST_CALLS = {"fa_bwd_workspace_size", "fa_bwd_qk_workspace_size", "fa_bwd_varlen_workspace_size",
-               "fa_decode_num_splits", "fa_decode_workspace_size"}
+               "fa_decode_num_splits", "fa_decode_workspace_size", "fa_fwd_bwd_host_workspace_size"}
 
 
 class FakeCuda:
@@ -65,6 +65,8 @@ class Recorder:
             for a, t in zip(args, fn.argtypes):
                 if t is ctypes.c_void_p:
                     assert a is None or isinstance(a, (int, ctypes.c_void_p)), (name, a)
+                elif isinstance(t, type) and issubclass(t, ctypes._Pointer):
+                    assert isinstance(a, ctypes.Array) and a._type_ is t._type_, (name, a)
                 else:
                     assert not isinstance(a, ctypes.c_void_p), (name, a)
                     t(a)  # raises TypeError for a value the C type cannot take
@@ -82,6 +84,7 @@ def rec(monkeypatch):
     monkeypatch.setattr(binding, "load_library", lambda path=None: r)
     monkeypatch.setattr(binding, "_stream", lambda t: ctypes.c_void_p(0))
     monkeypatch.setattr(binding, "_guard", lambda t: contextlib.nullcontext())
+    monkeypatch.setattr(binding, "_on_device", lambda d: contextlib.nullcontext())
     return r
 
 
@@ -226,4 +229,34 @@ def test_decode_calls_and_output_checks(rec):
     with pytest.raises(ValueError, match="cuda:1"):
         binding.fa_decode_paged(q, FakeCuda((40, page, H_kv, d), bf16, index=1), vc, table, lens, 200, True,
                                 num_splits=2, out=o, lse=lse, workspace=ws)
+    assert len(rec.calls) == 1
+
+
+class FakeStream:
+    def __init__(self, handle):
+        self.cuda_stream = handle
+
+
+def test_host_step_calls_and_checks(rec):
+    from exact_io_aware_49_b200 import binding
+    B, H, N, d = 1, 4, 300, 128
+    q, k, v, do = (torch.zeros(B, H, N, d, dtype=bf16) for _ in range(4))
+    need = binding.fa_fwd_bwd_host_workspace_size(B, H, N, d, 3)
+    ws = FakeCuda((need,), u8)
+    streams = [FakeStream(s) for s in (11, 22, 33)]
+    o, lse, dq, dk, dv = binding.fa_fwd_bwd_host(q, k, v, do, True, None, 0.1, 5, groups=3, device="cuda:0",
+                                                 workspace=ws, streams=streams)
+    (name, args), = rec.calls
+    assert name == "fa_fwd_bwd_host"
+    assert args[9:13] == (B, H, N, d) and args[18] == 3 and args[20] == need
+    assert [args[21][i] for i in range(3)] == [11, 22, 33]
+    assert tuple(o.shape) == (B, H, N, d) and tuple(lse.shape) == (B, H, N) and not o.is_cuda
+    with pytest.raises(ValueError):  # device tensors are not host buffers
+        binding.fa_fwd_bwd_host(FakeCuda((B, H, N, d), bf16), k, v, do, True, workspace=ws, streams=streams,
+                                device="cuda:0")
+    with pytest.raises(ValueError):  # too small a workspace is caught before the call
+        binding.fa_fwd_bwd_host(q, k, v, do, True, groups=3, device="cuda:0", workspace=FakeCuda((need - 1,), u8),
+                                streams=streams)
+    with pytest.raises(ValueError):
+        binding.fa_fwd_bwd_host(q, k, v, do, True, groups=3, device="cuda:0", workspace=ws, streams=streams[:2])
     assert len(rec.calls) == 1

@@ -104,3 +104,79 @@ def test_decode(d, page):
 def test_no_device_wait_timed_out():
     from exact_io_aware_49_b200 import fa_last_device_error
     assert fa_last_device_error() == 0
+
+
+# ---------------------------------------------------------------- head dimensions 192 and 256
+
+@pytest.mark.parametrize("d", [192, 256])
+@pytest.mark.parametrize("B,H,Nq,Nk,causal,p,dtype", [
+    (1, 2, 1000, 1000, True, 0.1, torch.bfloat16),    # ragged N, several 64-key tiles, dropout
+    (2, 1, 256, 256, False, 0.0, torch.bfloat16),
+    (1, 2, 333, 333, True, 0.0, torch.float16),
+    (1, 1, 130, 130, False, 0.7, torch.bfloat16),     # threshold above 0x8000
+    (1, 1, 1, 1, True, 0.0, torch.bfloat16),          # a single row and key
+    (1, 2, 300, 1000, True, 0.1, torch.bfloat16),     # Nq < Nk: bottom-right causal alignment
+    (1, 1, 1000, 300, True, 0.0, torch.bfloat16),     # Nq > Nk: leading rows see no key
+])
+def test_wide_forward(d, B, H, Nq, Nk, causal, p, dtype):
+    """The wide-head forward kernel (one 128-row query tile per CTA, 64-key
+    tiles, S double-buffered in tensor memory) against the oracle."""
+    from exact_io_aware_49_b200 import fa_fwd, fa_last_device_error
+    gen = torch.Generator().manual_seed(d * 10 + Nq + Nk)
+    q = _draw((B, H, Nq, d), gen, dtype)
+    k, v = (_draw((B, H, Nk, d), gen, dtype) for _ in range(2))
+    scale, seed = d ** -0.5, 13
+    o, lse = fa_fwd(q.cuda(), k.cuda(), v.cuda(), causal, scale, p, seed)
+    torch.cuda.synchronize()
+    assert fa_last_device_error() == 0
+    bits = 11 if dtype == torch.float16 else 8
+    for b in range(B):
+        for h in range(H):
+            args = [x[b, h].to(torch.float64).numpy() for x in (q, k, v)]
+            want_o, want_l = attention.forward(*args, causal=causal, scale=scale, p_drop=p, seed=seed, b=b, h=h)
+            pu.check_o(pu.f64(o[b, h].cpu()), want_o, f"O {(b, h)}", bits=bits)
+            pu.check_lse(pu.f64(lse[b, h].cpu()), want_l, f"LSE {(b, h)}")
+
+
+@pytest.mark.parametrize("d", [192, 256])
+def test_wide_forward_mask_and_guard_bands(d):
+    """Q = 0 and V[j] = e_(j - w0) on a window of keys: O[i, c] != 0 exactly
+    where key w0 + c is kept for row i (bit-exact dropout mask through the wide
+    kernel), and the canary bands around O and LSE stay untouched."""
+    from exact_io_aware_49_b200 import binding
+    from oracle import philox
+    B, H, N, p, seed = 1, 2, 700, 0.1, 3
+    gen = torch.Generator().manual_seed(d)
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    k = _draw((B, H, N, d), gen)
+    v = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    w0 = 0 if d == 192 else 500
+    n_c = min(d, N - w0)
+    v[:, :, w0:w0 + n_c, :n_c] = torch.eye(n_c, dtype=torch.bfloat16)
+    band = 4096
+    o_buf = torch.full((2 * band + B * H * N * d,), 12345, dtype=torch.int16, device="cuda")
+    l_buf = torch.full((2 * band + B * H * N,), -7.0, dtype=torch.float32, device="cuda")
+    o = o_buf[band:band + B * H * N * d].view(torch.bfloat16).view(B, H, N, d)
+    lse = l_buf[band:band + B * H * N].view(B, H, N)
+    binding.fa_fwd(q.cuda(), k.cuda(), v.cuda(), True, d ** -0.5, p, seed, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert bool((o_buf[:band] == 12345).all()) and bool((o_buf[-band:] == 12345).all())
+    assert bool((l_buf[:band] == -7.0).all()) and bool((l_buf[-band:] == -7.0).all())
+    got = (o[..., :n_c] != 0).cpu().numpy()
+    rows, cols = np.arange(N), np.arange(w0, w0 + n_c)
+    for h in range(H):
+        want = philox.keep_mask(seed, 0, h, rows, cols, p)
+        valid = cols[None, :] <= rows[:, None]
+        np.testing.assert_array_equal(got[0, h][valid], want[valid])
+        assert not got[0, h][~valid].any()
+
+
+def test_wide_backward_is_not_built():
+    """The backward and decode kernels stop at d = 128: those calls report
+    FA_ERR_UNSUPPORTED instead of computing."""
+    from exact_io_aware_49_b200 import FAError, fa_bwd, fa_fwd
+    q = torch.randn(1, 1, 128, 192, device="cuda").to(torch.bfloat16)
+    o, lse = fa_fwd(q, q, q, True)
+    with pytest.raises(FAError) as e:
+        fa_bwd(q, q, q, o, q, lse, True)
+    assert e.value.status == 2
