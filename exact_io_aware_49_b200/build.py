@@ -18,7 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB_NAME = "libfa_sm100.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
-SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_fwd_wide.cu", "fa_bwd.cu", "fa_decode.cu", "fa_mask.cu", "fa_noalloc.cu"]
+SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_fwd_wide.cu", "fa_bwd.cu", "fa_bwd_wide.cu", "fa_decode.cu", "fa_mask.cu",
+           "fa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

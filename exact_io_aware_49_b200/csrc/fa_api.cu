@@ -90,12 +90,12 @@ fa_status check_scalars(int d, float scale, float p_drop) {
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
   // 32 and 96 run on the 64- and 128-column kernels: the tensor maps read the
   // columns past d as zeros and only d columns are stored; 192 and 256 run on
-  // the wide forward kernel (the backward and decode kernels stop at 128)
+  // the wide kernels (fa_fwd_wide.cu, fa_bwd_wide.cu; not the paged decode)
   if (d != 32 && d != 64 && d != 96 && d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
-// Head dimensions the backward and decode kernels take.
+// Head dimensions of the 64- / 128-column kernels (the rest run on the wide ones).
 bool narrow_head(int d) { return d <= 128; }
 
 uint32_t drop_threshold(float p_drop) {
@@ -196,9 +196,9 @@ size_t workspace_bytes(const Problem& pb) {
   return round_up(acc, 256) + 2 * round_up(vec, 256) + round_up(order_bytes(pb), 256);
 }
 
-bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base) {
+bool encode_q_like(const Problem& pb, CUtensorMap* tm, const void* base, int box_rows = 128) {
   return encode_map(tm, base, pb.d, pb.seq.total_q, pb.groups(), pb.seq.tok_stride, pb.seq.q_head_stride,
-                    elem_type(pb.f16));
+                    elem_type(pb.f16), box_rows);
 }
 
 bool encode_k_like(const Problem& pb, CUtensorMap* tm, const void* base, int box_rows = 128) {
@@ -241,7 +241,6 @@ fa_status fwd_run(const Problem& pb, const void* Q, const void* K, const void* V
 }
 
 fa_status check_workspace(const Problem& pb, const void* workspace, size_t bytes) {
-  if (!narrow_head(pb.d)) return FA_ERR_UNSUPPORTED;  // no backward kernel for d > 128
   if (!workspace || misaligned(workspace, 256)) return FA_ERR_INVALID_ARG;
   if (bytes < workspace_bytes(pb)) return FA_ERR_INVALID_ARG;
   return FA_OK;
@@ -280,6 +279,7 @@ fa_status prepare_run(const Problem& pb, const void* O, const void* dO, const fl
 
 fa_status tiles_run(const Problem& pb, const void* Q, const void* K, const void* V, const void* dO, void* dK,
                     void* dV, void* workspace, size_t bytes, void* stream) {
+  if (!narrow_head(pb.d)) return FA_ERR_UNSUPPORTED;  // wide heads: bwd_run's two-kernel path only
   if (!Q || !K || !V || !dO || !dK || !dV) return FA_ERR_INVALID_ARG;
   if (misaligned(Q, 16) || misaligned(K, 16) || misaligned(V, 16) || misaligned(dO, 16) || misaligned(dK, 16) ||
       misaligned(dV, 16))
@@ -304,6 +304,7 @@ fa_status tiles_run(const Problem& pb, const void* Q, const void* K, const void*
 }
 
 fa_status finish_run(const Problem& pb, void* dQ, const void* workspace, size_t bytes, void* stream) {
+  if (!narrow_head(pb.d)) return FA_ERR_UNSUPPORTED;
   if (!dQ || misaligned(dQ, 16)) return FA_ERR_INVALID_ARG;
   fa_status st = check_workspace(pb, workspace, bytes);
   if (st != FA_OK) return st;
@@ -311,6 +312,26 @@ fa_status finish_run(const Problem& pb, void* dQ, const void* workspace, size_t 
   bwd_args(pb, &a, const_cast<void*>(workspace));
   a.dQ = dQ;
   return fa::launch_bwd_finish(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Head dimensions 192 / 256: the dK, dV kernel (64-query tiles against a
+// 128-key tile) and the dQ kernel (64-key tiles against a 128-query tile),
+// after the preprocess; dQ is written directly (no accumulator, no convert).
+fa_status wide_tiles_run(const Problem& pb, const void* Q, const void* K, const void* V, const void* dO, void* dQ,
+                         void* dK, void* dV, void* workspace, void* stream) {
+  fa::BwdArgs a;
+  bwd_args(pb, &a, workspace);
+  CUtensorMap kv[4], qm[4];  // Q, K, V, dO
+  if (!encode_q_like(pb, &kv[0], Q, 64) || !encode_k_like(pb, &kv[1], K, 128) || !encode_k_like(pb, &kv[2], V, 128) ||
+      !encode_q_like(pb, &kv[3], dO, 64) || !encode_q_like(pb, &qm[0], Q, 128) || !encode_k_like(pb, &qm[1], K, 64) ||
+      !encode_k_like(pb, &qm[2], V, 64) || !encode_q_like(pb, &qm[3], dO, 128))
+    return FA_ERR_CUDA;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  a.err = error_word_ptr();
+  if (!a.err) return FA_ERR_CUDA;
+  return fa::launch_bwd_wide(a, kv, qm, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status bwd_run(const Problem& pb, const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -323,6 +344,7 @@ fa_status bwd_run(const Problem& pb, const void* Q, const void* K, const void* V
   fa_status st = check_workspace(pb, workspace, bytes);
   if (st != FA_OK) return st;
   if ((st = prepare_run(pb, O, dO, LSE, workspace, bytes, stream)) != FA_OK) return st;
+  if (!narrow_head(pb.d)) return wide_tiles_run(pb, Q, K, V, dO, dQ, dK, dV, workspace, stream);
   if ((st = tiles_run(pb, Q, K, V, dO, dK, dV, workspace, bytes, stream)) != FA_OK) return st;
   return finish_run(pb, dQ, workspace, bytes, stream);
 }
@@ -547,7 +569,6 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
   Problem whole;
   fa_status st = fixed_problem(&whole, B, H, N, N, d, causal, scale, p_drop, seed, dtype == FA_DTYPE_F16);
   if (st != FA_OK) return st;
-  if (!narrow_head(d)) return FA_ERR_UNSUPPORTED;  // the backward stops at d = 128
   HostPlan hp;
   if (!host_plan(B, H, N, d, groups, &hp)) return FA_ERR_INVALID_ARG;
   if (!Q || !K || !V || !dO || !O || !LSE || !dQ || !dK || !dV || !streams) return FA_ERR_INVALID_ARG;

@@ -46,10 +46,10 @@
 #include "sm100.cuh"
 
 #ifndef FA_FWD_KEEP_FMT
-#define FA_FWD_KEEP_FMT 0  // 0: 4 packed words a row, 1: 32 words (byte signs)
+#define FA_FWD_KEEP_FMT 1  // 0: 4 packed words a row, 1: 32 words (byte signs)
 #endif
 #ifndef FA_FWD_DRAW_NB
-#define FA_FWD_DRAW_NB 8
+#define FA_FWD_DRAW_NB 4
 #endif
 
 namespace fa {
@@ -365,6 +365,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                                static_cast<uint32_t>(su.b), p.philox_rk);
       const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
       const bool hi_t = p.drop_t > 0x8000u;
+      const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
       // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
       // last key, and under the causal mask the row's position i + Nk - Nq);
       // tiles from t_mask on are the first that can hold a masked key for
@@ -393,7 +394,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             draw_keep_words<false, kBN / 8>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, W);
           asm volatile("" : "+r"(W[0]), "+r"(W[1]), "+r"(W[2]), "+r"(W[3]));  // not sunk past the wait
         }
-#else
+#elif FA_FWD_KEEP_FMT == 1
         uint32_t kz[32];
         if (DROPOUT) {
           if (hi_t)
@@ -402,6 +403,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             draw_keep_bytes<false, FA_FWD_DRAW_NB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
           reg_fence32(kz);
         }
+#else
+        // Philox words of the tile's first 32 keys, before S is ready; the
+        // exponential loop below draws each next 32 keys' words while it
+        // exponentiates the current ones
+        uint32_t wn[4][4];
+        if (DROPOUT) philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, wn);
 #endif
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -458,8 +465,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
+#if FA_FWD_KEEP_FMT == 2
+        uint32_t wc[4][4];
+#endif
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
+#if FA_FWD_KEEP_FMT == 2
+          if (DROPOUT && (c & 15) == 0) {
+            // this chunk's words, then the next chunk's Philox calls (independent
+            // of the exponentials that follow, so they overlap them)
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
+            if (c + 16 < kBN / 2)
+              philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + (c + 16) / 4), phx, p.philox_rk, wn);
+          }
+#endif
           float x0, x1;
           f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
           const float p0 = ex2_approx(x0);
@@ -473,8 +495,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // dropped keys: zero the 16-bit P (the row sum l keeps them)
 #if FA_FWD_KEEP_FMT == 0
           if (DROPOUT) pk[c] &= keep_mask_pair(W, c);
-#else
+#elif FA_FWD_KEEP_FMT == 1
           if (DROPOUT) pk[c] &= prmt(kz[c >> 1], 0u, (c & 1) ? 0xBBAAu : 0x9988u);
+#else
+          if (DROPOUT) {
+            // keep test on the FMA pipe: the float 2^23 + u16 is exact, and
+            // sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0
+            const uint32_t wv = wc[(c & 15) >> 2][c & 3];
+            float k0, k1;
+            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k0) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7610u))),
+                "f"(drop_bias));
+            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7632u))),
+                "f"(drop_bias));
+            float q0, q1;
+            f2_unpack(mul_f2(pp, f2_pack(k0, k1)), q0, q1);
+            pk[c] = pack2<F16>(q0, q1);
+          }
 #endif
         }
         {

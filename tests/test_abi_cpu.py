@@ -72,15 +72,17 @@ def test_fwd_rejects_bad_arguments(lib, kw, want):
 
 
 @pytest.mark.parametrize("d", [192, 256])
-def test_wide_heads_forward_only(lib, d):
-    """d = 192 / 256 pass the forward's validation (a null output still stops
-    the call first); the backward, the host-buffer step and the decode reject
-    them as unsupported."""
+def test_wide_heads_validation(lib, d):
+    """d = 192 / 256 pass the forward's and backward's validation (a null
+    pointer still stops the call first); the staged backward entry points and
+    the paged decode, which have no wide-head kernels, reject them."""
     assert _fwd(lib, d=d, O=0) == 1
     ws = lib.fa_bwd_workspace_size(1, 1, 128, d)
-    assert lib.fa_bwd(A, A, A, A, A, A, A, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, A, ws, None) == 2
-    st = (ctypes.c_void_p * 3)()
-    assert lib.fa_fwd_bwd_host(A, A, A, A, A, A, A, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, 0, 1, A, 1 << 40, st) == 2
+    assert lib.fa_bwd(A, A, A, A, A, A, 0, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, A, ws, None) == 1
+    assert lib.fa_bwd_tiles(A, A, A, A, A, A, 1, 1, 128, d, 1, 0.125, 0.0, 0, A, ws, None) == 2
+    assert lib.fa_bwd_finish(A, 1, 1, 128, d, 0.125, A, ws, None) == 2
+    assert lib.fa_decode_paged(A, A, A, A, A, A, A, 1, 8, 2, 1, d, 4, 64, 2, 128, 1, 0.125, 1, 0, A, 1 << 30,
+                               None) == 2
 
 
 def _bwd(lib, ws=A, ws_bytes=None, B=1, H=1, N=128, d=64, p=0.0, **ptrs):
@@ -104,7 +106,7 @@ def test_workspace_size_is_linear_in_n(lib):
 
 @pytest.mark.parametrize("kw,want", [
     (dict(ws=0), 1), (dict(ws=A + 16), 1), (dict(dQ=0), 1), (dict(dO=A + 2), 1), (dict(L=0), 1),
-    (dict(ws_bytes=1000), 1), (dict(p=1.5), 1), (dict(d=256), 2), (dict(N=64, ws_bytes=100), 1),
+    (dict(ws_bytes=1000), 1), (dict(p=1.5), 1), (dict(d=320), 2), (dict(N=64, ws_bytes=100), 1),
 ])
 def test_bwd_rejects_bad_arguments(lib, kw, want):
     assert _bwd(lib, **kw) == want

@@ -171,12 +171,69 @@ def test_wide_forward_mask_and_guard_bands(d):
         assert not got[0, h][~valid].any()
 
 
-def test_wide_backward_is_not_built():
-    """The backward and decode kernels stop at d = 128: those calls report
-    FA_ERR_UNSUPPORTED instead of computing."""
-    from exact_io_aware_49_b200 import FAError, fa_bwd, fa_fwd
-    q = torch.randn(1, 1, 128, 192, device="cuda").to(torch.bfloat16)
-    o, lse = fa_fwd(q, q, q, True)
-    with pytest.raises(FAError) as e:
-        fa_bwd(q, q, q, o, q, lse, True)
-    assert e.value.status == 2
+@pytest.mark.parametrize("d", [192, 256])
+@pytest.mark.parametrize("B,H,Nq,Nk,causal,p,det,dtype", [
+    (1, 2, 1000, 1000, True, 0.1, False, torch.bfloat16),  # ragged N, dropout
+    (2, 1, 256, 256, False, 0.0, False, torch.bfloat16),
+    (1, 1, 333, 333, True, 0.7, False, torch.float16),     # threshold above 0x8000
+    (1, 2, 200, 700, True, 0.1, True, torch.bfloat16),     # Nq < Nk (deterministic is the only dQ order here)
+    (1, 1, 700, 200, True, 0.0, False, torch.bfloat16),    # Nq > Nk: leading rows see no key
+])
+def test_wide_backward(d, B, H, Nq, Nk, causal, p, det, dtype):
+    """The wide-head backward (a dK / dV kernel over 64-query tiles and a dQ
+    kernel over 64-key tiles) against the oracle; dQ is written by one CTA per
+    row, so two calls agree bit for bit."""
+    from exact_io_aware_49_b200 import fa_bwd, fa_fwd, fa_last_device_error
+    gen = torch.Generator().manual_seed(d + 7 * Nq + Nk)
+    q, do = (_draw((B, H, Nq, d), gen, dtype) for _ in range(2))
+    k, v = (_draw((B, H, Nk, d), gen, dtype) for _ in range(2))
+    scale, seed = d ** -0.5, 17
+    qd, kd, vd, dod = (x.cuda() for x in (q, k, v, do))
+    o, lse = fa_fwd(qd, kd, vd, causal, scale, p, seed)
+    dq, dk, dv = fa_bwd(qd, kd, vd, o, dod, lse, causal, scale, p, seed, deterministic=det)
+    dq2, dk2, dv2 = fa_bwd(qd, kd, vd, o, dod, lse, causal, scale, p, seed, deterministic=det)
+    torch.cuda.synchronize()
+    assert fa_last_device_error() == 0
+    assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    bits = 11 if dtype == torch.float16 else 8
+
+    def one(bh):
+        b, h = bh
+        args = [x[b, h].to(torch.float64).numpy() for x in (q, k, v, do)]
+        kw = dict(causal=causal, scale=scale, p_drop=p, seed=seed, b=b, h=h)
+        want_o, want_l = attention.forward(*args[:3], **kw)
+        pu.check_o(pu.f64(o[b, h].cpu()), want_o, f"O {(b, h)}", bits=bits)
+        pu.check_lse(pu.f64(lse[b, h].cpu()), want_l, f"LSE {(b, h)}")
+        want = attention.backward(*args, **kw)[:3]
+        for got, w, name in zip((dq, dk, dv), want, ("dQ", "dK", "dV")):
+            pu.check_grad(pu.f64(got[b, h].cpu()), w, f"{name} {(b, h)}")
+
+    pu.map_heads(one, [(b, h) for b in range(B) for h in range(H)])
+
+
+@pytest.mark.parametrize("d", [192, 256])
+def test_wide_backward_mask_probe(d):
+    """Bit-exact dropout mask through the wide dK / dV kernel: Q = 0 and dO
+    rows one-hot over a window of d queries make dV[j, c] non-zero exactly
+    where key j is kept for query w0 + c."""
+    from exact_io_aware_49_b200 import fa_bwd, fa_fwd
+    from oracle import philox
+    B, H, N, p, seed = 1, 2, 500, 0.1, 23
+    gen = torch.Generator().manual_seed(d + 1)
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16, device="cuda")
+    k, v = (_draw((B, H, N, d), gen).cuda() for _ in range(2))
+    o, lse = fa_fwd(q, k, v, True, d ** -0.5, p, seed)
+    cols = np.arange(N)
+    for w0 in (0, N - min(d, N)):
+        n_c = min(d, N - w0)
+        do = torch.zeros(B, H, N, d, dtype=torch.bfloat16, device="cuda")
+        idx = torch.arange(n_c, device="cuda")
+        do[:, :, w0 + idx, idx] = 1.0
+        _, _, dv = fa_bwd(q, k, v, o, do, lse, True, d ** -0.5, p, seed)
+        got = (dv[0, :, :, :n_c] != 0).cpu().numpy()
+        rows = np.arange(w0, w0 + n_c)
+        for h in range(H):
+            want = philox.keep_mask(seed, 0, h, rows, cols, p).T
+            valid = cols[:, None] <= rows[None, :]
+            np.testing.assert_array_equal(got[h][valid], want[valid])
+            assert not got[h][~valid].any()
