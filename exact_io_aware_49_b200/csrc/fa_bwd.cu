@@ -238,14 +238,16 @@ __device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, ui
 }
 
 // dV (+)= P^T dO : A = P^T (TMEM, 16-bit pairs), B = dO tile (MN-major), K = 128 queries, N = D.
+// P^T of query columns [64 g, 64 g + 64) lies over that group's own S^T
+// columns: 32 TMEM columns from tmem_p + 64 g.
 template <int D, bool F16>
 __device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem, bool accumulate) {
   do_smem = opaque_u32(do_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_ts(tmem_d, tmem_p + kk * 8, sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(tmem_d, tmem_p + (kk / 4) * 64 + (kk % 4) * 8,
+           sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // dK (+)= dS^T Q : A = dS^T (smem, K-major over queries), B = Q tile (MN-major), N = D.
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S^T [0,128) (P^T over [0,64)), dP^T / dQ [128,256), dK, dV after.
+  // TMEM columns: S^T [0,128) (P^T of query columns 64g.. over [64g, 64g+32)), dP^T / dQ [128,256), dK, dV after.
   constexpr uint32_t kColS = 0, kColDP = 128, kColDK = 256, kColDV = 256 + D;
   const uint32_t sm_k = smem_u32(smem + L::kK), sm_v = smem_u32(smem + L::kV);
   const uint32_t sm_q = smem_u32(smem + L::kQ), sm_do = smem_u32(smem + L::kDO);
@@ -601,7 +603,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c)
         pk[c] = DROPOUT ? pack2_relu<F16>(P[2 * c], P[2 * c + 1]) : pack2<F16>(P[2 * c], P[2 * c + 1]);
-      tmem_st32(t_row + kColS + 32 * g, pk);
+      // over this group's own S^T columns: the other group may still be
+      // reading its half of S^T from the same TMEM lanes
+      tmem_st32(t_row + kColS + 64 * g, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -95,6 +95,23 @@ def test_full_size_benchmark_shape_repeatable():
     assert torch.isfinite(a[0].float()).all()
 
 
+@pytest.mark.parametrize("name", ["causal_dropout_N4096_d128", "causal_dropout_N32768_d128"])
+def test_default_mode_dk_dv_repeatable(name):
+    """dK and dV of a key tile come from one CTA, so even the default
+    backward (dQ in atomic order) gives them bit for bit on every call.  A
+    P^T store over S^T columns that the other elementwise warpgroup has not
+    read yet would corrupt 32 x 32 blocks of P^T at random and break this."""
+    from exact_io_aware_49_b200 import fa_fwd
+    w = wl.BY_NAME[name]
+    q, k, v, do = (x.cuda() for x in wl.draw_inputs(w))
+    o, lse = fa_fwd(q, k, v, w.causal, w.scale, w.p_drop, w.seed)
+    first = _grads(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, False)
+    for _ in range(3):
+        again = _grads(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, False)
+        for a, b in zip(first[1:], again[1:]):
+            assert torch.equal(_bits(a), _bits(b))
+
+
 def test_no_device_wait_timed_out():
     from exact_io_aware_49_b200 import fa_last_device_error
     assert fa_last_device_error() == 0

@@ -228,6 +228,11 @@ class Backward(Protocol):
         self.s_reading, self.dp_reading = set(), set()
         self.p_written, self.ds_written = {}, {}
         self.ds_readers, self.dq_reading, self.staging, self.dv_last = 0, False, None, -1
+        # TMEM columns within the S^T block: warp w (group g = w // 4, lanes of
+        # quadrant w % 4) reads S^T columns [64 g, 64 g + 64) and writes its
+        # P^T over [64 g, 64 g + 32); the slip puts it at [32 g, 32 g + 32),
+        # over the other group's unread S^T
+        self.s_loaded = [-1] * 8
 
     def producer(self):
         self.loads.append(("kv", None))
@@ -306,8 +311,14 @@ class Backward(Protocol):
             if self.tm_s != ("S", it) or self.qst[s] != it:
                 self.errors.append(f"warp {w} tile {it}: S cols {self.tm_s}, vectors of {self.qst[s]}")
             self.s_reading.add(w)
+            self.s_loaded[w] = it
             yield None
             self.s_reading.discard(w)
+            g, partner = w // 4, (w + 4) % 8
+            p_cols = range(32 * g, 32 * g + 32) if self.slip == "shared_p_cols" else range(64 * g, 64 * g + 32)
+            partner_cols = range(64 * (1 - g), 64 * (1 - g) + 64)
+            if self.s_loaded[partner] < it and set(p_cols) & set(partner_cols):
+                self.errors.append(f"warp {w} tile {it}: P^T written over S^T warp {partner} has not read")
             self.p_written.setdefault(it, set()).add(w)
             if len(self.p_written[it]) == 8:
                 self.tm_s = ("P", it)
@@ -535,7 +546,7 @@ def test_forward_slip_is_caught():
     assert any(Forward(rng, 6, 6, 1, 2, 0.0, slip="early_stage_reuse").check() for _ in range(40))
 
 
-@pytest.mark.parametrize("slip", ["no_dqfree_wait", "no_dostage_wait"])
+@pytest.mark.parametrize("slip", ["no_dqfree_wait", "no_dostage_wait", "shared_p_cols"])
 def test_backward_slips_are_caught(slip):
     rng = random.Random(4)
     assert any(Backward(rng, 4, slip=slip).check() for _ in range(40))
