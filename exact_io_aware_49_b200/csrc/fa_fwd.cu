@@ -19,16 +19,19 @@
 //  * warp roles: warps 0-3 and 4-7 are the softmax warpgroups of Q0 and Q1
 //    (one thread per query row: causal mask on the diagonal tile, running
 //    max / sum, exp2, Philox dropout, P to TMEM, and the epilogue); warp 8
-//    issues the MMAs; warp 9 issues the TMA loads.  While one warpgroup turns
-//    S into P, the tensor core works on the other query tile;
+//    issues the MMAs (the whole warp runs the loop, so descriptors are
+//    warp-uniform values, and one elected lane issues); warp 9 issues the
+//    TMA loads.  While one warpgroup turns S into P, the tensor core works
+//    on the other query tile;
 //  * the O rescale is lazy: the stale maximum is kept until a row's maximum
 //    grows by more than 8 (log2 units).  l and O share the stale maximum, so
 //    the result is unchanged; P stays <= 2^8;
 //  * dropout never stores a mask: keep decisions come from Philox keyed on
-//    (seed, b, h, i, j), computed as 0.0 / 1.0 multipliers with one byte
-//    permute and one saturating add per element (the integer ALU pipe, which
-//    runs at half rate, is the bottleneck of this path); kept P are left
-//    unscaled and 1/(1-p) is folded into the final normalisation.
+//    (seed, b, h, i, j), drawn for a whole tile before its scores are read
+//    (16 calls per row and 128-key tile, 4 in lockstep, while the tensor core
+//    computes S) and applied with a byte permute and an AND per pair of P;
+//    kept P are left unscaled and 1/(1-p) is folded into the final
+//    normalisation.
 //  * a causal CTA processes only key tiles up to its diagonal; the grid puts
 //    the heaviest query blocks first;
 //  * queries and keys may differ in number (Nq != Nk, causal alignment
@@ -45,28 +48,22 @@
 #include "philox.cuh"
 #include "sm100.cuh"
 
-#ifndef FA_FWD_KEEP_FMT
-#define FA_FWD_KEEP_FMT 1  // 0: 4 packed words a row, 1: 32 words (byte signs)
-#endif
-#ifndef FA_FWD_DRAW_NB
-#define FA_FWD_DRAW_NB 4
-#endif
-
 namespace fa {
 namespace {
 
-// byte-sign format: kz[m] holds pair 2m's keep bits in the signs of bytes 0, 1
-// and pair 2m + 1's in bytes 2, 3
+// Keep bits of one row for the 128 keys of a tile (calls jb0 .. jb0 + 15, one
+// Philox call per 8 keys, kNB calls in lockstep), in byte-sign form: kz[m]
+// holds pair 2m's keep bits in the signs of bytes 0, 1 and pair 2m + 1's in
+// bytes 2, 3.  Each Philox word carries two 16-bit draws; the two-lane test of
+// keep_mask_2x16 leaves their keep bits at bits 15 and 31, and one byte
+// permute gathers the four bits of two words.
 template <bool kHighT, int kNB>
 __device__ __forceinline__ void draw_keep_bytes(uint32_t jb0, const PhiloxFixed123& f, const uint32_t* rk,
                                                 uint32_t c2, uint32_t (&kz)[32]) {
 #pragma unroll
   for (int g0 = 0; g0 < 16; g0 += kNB) {
     uint32_t w[kNB][4];
-    if (kNB == 1)
-      philox4x32_10_c0(jb0 + g0, f, rk, w[0]);
-    else
-      philox4x32_10_c0_batch<kNB>(jb0 + g0, f, rk, w);
+    philox4x32_10_c0_batch<kNB>(jb0 + g0, f, rk, w);
 #pragma unroll
     for (int n = 0; n < kNB; ++n) {
       uint32_t z[4];
@@ -86,6 +83,7 @@ constexpr int kBN = 128;             // keys per tile
 constexpr int kFwdThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
+constexpr int kDrawNB = 4;           // Philox calls in lockstep
 // Register split (setmaxnreg): the kernel launches with kFwdLaunchRegs per
 // thread; softmax warpgroups grow to kSoftmaxRegs, the control warpgroup
 // (MMA, TMA, two idle warps) shrinks to kControlRegs.  The split must fit the
@@ -152,26 +150,32 @@ struct FwdParams {
   int group, BH;
 };
 
-// S_q = Q_q * K^T : M = 128 query rows, N = 128 keys, K = D (both K-major).
+// S_q = Q_q K^T : M = 128 query rows, N = 128 keys, K = D (both K-major).
+// a0 / b0 are the descriptors of the Q tile and the K stage; each K-step
+// adds its box / swizzle-atom offset (bytes / 16) to the start address.
 template <int D, bool F16>
-__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(bool leader, uint32_t tmem_s, uint64_t a0, uint64_t b0) {
   constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * FwdSmem<D>::kBoxBytes + (kk % 4) * 32;
-    mma_ss(tmem_s, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc, kk > 0);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = static_cast<uint32_t>(((kk / 4) * FwdSmem<D>::kBoxBytes + (kk % 4) * 32) >> 4);
+      mma_ss(tmem_s, a0 + off, b0 + off, idesc, kk > 0);
+    }
   }
 }
 
-// O_q (+)= P_q * V : M = 128, N = D, K = 128 keys.  P (16-bit, packed in
-// pairs) lives in TMEM over S_q; V is MN-major in shared memory (D contiguous).
+// O_q (+)= P_q V : M = 128, N = D, K = 128 keys.  P (16-bit, packed in pairs)
+// lives in TMEM over S_q; V is MN-major in shared memory (D contiguous,
+// 64-column boxes kBoxBytes apart), b0 the descriptor of its stage.
 template <int D, bool F16>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+__device__ __forceinline__ void issue_pv(bool leader, uint32_t tmem_o, uint32_t tmem_p, uint64_t b0, bool accumulate) {
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk) {
-    const uint64_t bdesc = sdesc_sw128(v_smem + kk * 2048, FwdSmem<D>::kBoxBytes, 1024);
-    mma_ts(tmem_o, tmem_p + kk * 8, bdesc, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < kBN / 16; ++kk)
+      mma_ts(tmem_o, tmem_p + kk * 8, b0 + static_cast<uint32_t>((kk * 2048) >> 4), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -302,44 +306,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nt_all > 0) {
-      bool ok = mbar_wait(bar.q, 0, abort_flag, p.err) && mbar_wait(&bar.kfull[0], 0, abort_flag, p.err);
+    // Per key tile t and query tile q: O_q += P_{q,t} V_t, then S_{q,t+1}
+    // into the columns P_{q,t} occupied (the tensor core runs the products in
+    // issue order).  The whole warp runs the loop, so descriptors and
+    // counters are warp-uniform values; one elected lane issues the MMAs and
+    // commits.
+    if (nt_all > 0) {
+      const bool leader = elect_one();
+      // descriptor bases; a tile, stage, box or K-step offset (bytes / 16) is
+      // added to the start-address field
+      const uint64_t dq0 = sdesc_sw128(sm_q, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sm_k, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sm_v, L::kBoxBytes, 1024);
+      // every lane waits; the vote keeps the warp's decision uniform
+#define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
+      bool ok = FA_WAIT(bar.q, 0) && FA_WAIT(&bar.kfull[0], 0);
       if (ok) {
         tc_fence_after();
         for (int q = 0; q < nq; ++q) {
           if ((q ? nt1 : nt0) == 0) continue;  // a query tile that sees no key
-          issue_qk<D, F16>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k);
-          mma_commit(&bar.s_ready[q]);
+          issue_qk<D, F16>(leader, tmem + q * 128, dq0 + static_cast<uint32_t>((q * L::kTileBytes) >> 4), dk0);
+          if (leader) mma_commit(&bar.s_ready[q]);
         }
       }
       for (int t = 0; ok && t < nt_all; ++t) {
         const int s = t % S;
-        if (!mbar_wait(&bar.vfull[s], (t / S) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&bar.vfull[s], (t / S) & 1)) { ok = false; break; }
         bool next_k_ready = false;
         const int s1 = (t + 1) % S;
         for (int q = 0; q < nq; ++q) {
           const int ntq = q ? nt1 : nt0;
           if (t >= ntq) continue;
-          if (!mbar_wait(&bar.p_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!FA_WAIT(&bar.p_ready[q], t & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D, F16>(tmem + 256 + q * D, tmem + q * 128, sm_v + s * L::kTileBytes, t > 0);
+          issue_pv<D, F16>(leader, tmem + 256 + q * D, tmem + q * 128,
+                           dv0 + static_cast<uint32_t>((s * L::kTileBytes) >> 4), t > 0);
           if (t == ntq - 1) {
-            mma_commit(&bar.o_ready[q]);
+            if (leader) mma_commit(&bar.o_ready[q]);
           } else {
             if (!next_k_ready) {
-              if (!mbar_wait(&bar.kfull[s1], ((t + 1) / S) & 1, abort_flag, p.err)) { ok = false; break; }
+              if (!FA_WAIT(&bar.kfull[s1], ((t + 1) / S) & 1)) { ok = false; break; }
               tc_fence_after();
               next_k_ready = true;
             }
-            issue_qk<D, F16>(tmem + q * 128, sm_q + q * L::kTileBytes, sm_k + s1 * L::kTileBytes);
-            mma_commit(&bar.s_ready[q]);
+            issue_qk<D, F16>(leader, tmem + q * 128, dq0 + static_cast<uint32_t>((q * L::kTileBytes) >> 4),
+                             dk0 + static_cast<uint32_t>((s1 * L::kTileBytes) >> 4));
+            if (leader) mma_commit(&bar.s_ready[q]);
           }
         }
         if (!ok) break;
-        mma_commit(&bar.kvempty[s]);
+        if (leader) mma_commit(&bar.kvempty[s]);
       }
+#undef FA_WAIT
       if (!ok) {
-        mma_commit(bar.drain);  // wait for MMAs already issued before TMEM is freed
+        if (leader) mma_commit(bar.drain);  // wait for MMAs already issued before TMEM is freed
         mbar_wait_drain(bar.drain, 0);
       }
     }
@@ -365,7 +385,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                                static_cast<uint32_t>(su.b), p.philox_rk);
       const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
       const bool hi_t = p.drop_t > 0x8000u;
-      const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
       // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
       // last key, and under the causal mask the row's position i + Nk - Nq);
       // tiles from t_mask on are the first that can hold a masked key for
@@ -385,31 +404,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // keep bits of the tile's 128 keys, drawn before S is ready: while the
         // tensor core computes S the warp would only wait, and the 16 Philox
         // calls run 8 at a time in lockstep (the S row's registers are free)
-#if FA_FWD_KEEP_FMT == 0
-        uint32_t W[4] = {0u, 0u, 0u, 0u};
-        if (DROPOUT) {
-          if (hi_t)
-            draw_keep_words<true, kBN / 8>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, W);
-          else
-            draw_keep_words<false, kBN / 8>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, W);
-          asm volatile("" : "+r"(W[0]), "+r"(W[1]), "+r"(W[2]), "+r"(W[3]));  // not sunk past the wait
-        }
-#elif FA_FWD_KEEP_FMT == 1
         uint32_t kz[32];
         if (DROPOUT) {
           if (hi_t)
-            draw_keep_bytes<true, FA_FWD_DRAW_NB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
+            draw_keep_bytes<true, kDrawNB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
           else
-            draw_keep_bytes<false, FA_FWD_DRAW_NB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
+            draw_keep_bytes<false, kDrawNB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
           reg_fence32(kz);
         }
-#else
-        // Philox words of the tile's first 32 keys, before S is ready; the
-        // exponential loop below draws each next 32 keys' words while it
-        // exponentiates the current ones
-        uint32_t wn[4][4];
-        if (DROPOUT) philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, wn);
-#endif
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -465,25 +467,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
-#if FA_FWD_KEEP_FMT == 2
-        uint32_t wc[4][4];
-#endif
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
-#if FA_FWD_KEEP_FMT == 2
-          if (DROPOUT && (c & 15) == 0) {
-            // this chunk's words, then the next chunk's Philox calls (independent
-            // of the exponentials that follow, so they overlap them)
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
-            if (c + 16 < kBN / 2)
-              philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + (c + 16) / 4), phx, p.philox_rk, wn);
-          }
-#endif
+          const float sv0 = s[2 * c], sv1 = s[2 * c + 1];
           float x0, x1;
-          f2_unpack(fma_f2(f2_pack(s[2 * c], s[2 * c + 1]), sl2x2, negm2), x0, x1);
+          f2_unpack(fma_f2(f2_pack(sv0, sv1), sl2x2, negm2), x0, x1);
           const float p0 = ex2_approx(x0);
           const float p1 = ex2_approx(x1);
           const uint64_t pp = f2_pack(p0, p1);
@@ -493,31 +481,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             rs0 = add_f2(rs0, pp);
           pk[c] = pack2<F16>(p0, p1);
           // dropped keys: zero the 16-bit P (the row sum l keeps them)
-#if FA_FWD_KEEP_FMT == 0
-          if (DROPOUT) pk[c] &= keep_mask_pair(W, c);
-#elif FA_FWD_KEEP_FMT == 1
           if (DROPOUT) pk[c] &= prmt(kz[c >> 1], 0u, (c & 1) ? 0xBBAAu : 0x9988u);
-#else
-          if (DROPOUT) {
-            // keep test on the FMA pipe: the float 2^23 + u16 is exact, and
-            // sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0
-            const uint32_t wv = wc[(c & 15) >> 2][c & 3];
-            float k0, k1;
-            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k0) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7610u))),
-                "f"(drop_bias));
-            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7632u))),
-                "f"(drop_bias));
-            float q0, q1;
-            f2_unpack(mul_f2(pp, f2_pack(k0, k1)), q0, q1);
-            pk[c] = pack2<F16>(q0, q1);
-          }
-#endif
         }
         {
           float a0, a1;
           f2_unpack(add_f2(rs0, rs1), a0, a1);
           l += a0 + a1;
         }
+
         if (rescale && t > 0) {
           // O accumulator of this row, after the S row is consumed (fewer live
           // registers); every earlier PV MMA completed before S_t was committed

@@ -255,6 +255,17 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// One lane of a converged warp (the lowest active one) gets true.  The MMA
+// issuers run their loops with the whole warp, so that descriptors and loop
+// state are warp-uniform values, and issue each tcgen05 op from this lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 format (version 1).
 // lbo/sbo are byte offsets (leading / stride dimension).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
