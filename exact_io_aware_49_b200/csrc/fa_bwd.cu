@@ -215,10 +215,12 @@ struct BwdParams {
   int group, BH;
 };
 
-// The MMA issuer rebuilds its shared-memory descriptors from the tile base
-// addresses at each use instead of keeping all of them live across its loop
-// (its warpgroup runs with few registers): an opaque copy of each base stops
-// the compiler from hoisting the descriptors out of the loop.
+// MMA helpers.  The MMA warp runs its loop with all 32 lanes, so addresses
+// and descriptors are warp-uniform values; ``leader`` (one elected lane)
+// issues.  The descriptors are rebuilt from the tile base addresses at each
+// use instead of being kept live across the loop (the warpgroup runs with few
+// registers): an opaque copy of each base stops the compiler from hoisting
+// them out of the loop.
 __device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
   asm volatile("mov.b32 %0, %0;" : "+r"(x));
   return x;
@@ -226,54 +228,64 @@ __device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
 
 // D[tmem] (+)= A[K-major tile] * B[K-major tile]^T, M = N = 128, K = D.
 template <int D, bool F16>
-__device__ __forceinline__ void mma_tile_kk(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+__device__ __forceinline__ void mma_tile_kk(bool leader, uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
   a_smem = opaque_u32(a_smem);
   b_smem = opaque_u32(b_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
-    mma_ss(tmem_d, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc, kk > 0);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
+      mma_ss(tmem_d, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc, kk > 0);
+    }
   }
 }
 
-// dV (+)= P^T dO : A = P^T (TMEM, 16-bit pairs), B = dO tile (MN-major), K = 128 queries, N = D.
-// P^T of query columns [64 g, 64 g + 64) lies over that group's own S^T
-// columns: 32 TMEM columns from tmem_p + 64 g.
+// dV (+)= P^T dO : A = P^T (TMEM, 16-bit pairs), B = dO tile (MN-major),
+// K = 128 queries, N = D.  P^T of query columns [64 g, 64 g + 64) lies over
+// that group's own S^T columns: 32 TMEM columns from tmem_p + 64 g.
 template <int D, bool F16>
-__device__ __forceinline__ void mma_dv(uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem, bool accumulate) {
+__device__ __forceinline__ void mma_dv(bool leader, uint32_t tmem_d, uint32_t tmem_p, uint32_t do_smem,
+                                       bool accumulate) {
   do_smem = opaque_u32(do_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_ts(tmem_d, tmem_p + (kk / 4) * 64 + (kk % 4) * 8,
-           sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(tmem_d, tmem_p + (kk / 4) * 64 + (kk % 4) * 8,
+             sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 // dK (+)= dS^T Q : A = dS^T (smem, K-major over queries), B = Q tile (MN-major), N = D.
 template <int D, bool F16>
-__device__ __forceinline__ void mma_dk(uint32_t tmem_d, uint32_t ds_smem, uint32_t q_smem, bool accumulate) {
+__device__ __forceinline__ void mma_dk(bool leader, uint32_t tmem_d, uint32_t ds_smem, uint32_t q_smem,
+                                       bool accumulate) {
   ds_smem = opaque_u32(ds_smem);
   q_smem = opaque_u32(q_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t a_off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
-    mma_ss(tmem_d, sdesc_sw128(ds_smem + a_off, 16, 1024), sdesc_sw128(q_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
-           idesc, (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t a_off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
+      mma_ss(tmem_d, sdesc_sw128(ds_smem + a_off, 16, 1024),
+             sdesc_sw128(q_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
   }
 }
 
 // dQ_i = dS K : A = dS (the dS^T tile read MN-major, M = queries), B = K tile (MN-major), N = D.
 template <int D, bool F16>
-__device__ __forceinline__ void mma_dq(uint32_t tmem_d, uint32_t ds_smem, uint32_t k_smem) {
+__device__ __forceinline__ void mma_dq(bool leader, uint32_t tmem_d, uint32_t ds_smem, uint32_t k_smem) {
   ds_smem = opaque_u32(ds_smem);
   k_smem = opaque_u32(k_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, true, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_ss(tmem_d, sdesc_sw128(ds_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
-           sdesc_sw128(k_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ss(tmem_d, sdesc_sw128(ds_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
+             sdesc_sw128(k_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
 }
 
 __device__ __forceinline__ void bwd_teardown(uint32_t tmem, bool dealloc) {
@@ -393,53 +405,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mbar_wait_drain(&bars[kDOFull0 + (it & 1)], (it >> 1) & 1);
         }
       }
-    } else if (warp == kBwdMmaWarp && lane == 0) {
+    } else if (warp == kBwdMmaWarp) {
       // ---------------------------------------------------------------- MMA issuer
-      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err) &&
-                mbar_wait(&bars[kQFull0], 0, abort_flag, p.err);
+      // the whole warp runs the loop; one elected lane issues and commits
+      const bool leader = elect_one();
+#define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
+      bool ok = FA_WAIT(&bars[kKVFull], 0) && FA_WAIT(&bars[kQFull0], 0);
       if (ok) {
         tc_fence_after();
-        mma_tile_kk<D, F16>(tmem + kColS, sm_k, sm_q);
-        mma_commit(&bars[kSReady]);
-        ok = mbar_wait(&bars[kDOFull0], 0, abort_flag, p.err);
+        mma_tile_kk<D, F16>(leader, tmem + kColS, sm_k, sm_q);
+        if (leader) mma_commit(&bars[kSReady]);
+        ok = FA_WAIT(&bars[kDOFull0], 0);
         if (ok) {
           tc_fence_after();
-          mma_tile_kk<D, F16>(tmem + kColDP, sm_v, sm_do);
-          mma_commit(&bars[kDPReady]);
+          mma_tile_kk<D, F16>(leader, tmem + kColDP, sm_v, sm_do);
+          if (leader) mma_commit(&bars[kDPReady]);
         }
       }
       for (int it = 0; ok && it < nq; ++it) {
         const int s = it & 1, s1 = (it + 1) & 1;
         const bool more = it + 1 < nq;
-        if (!mbar_wait(&bars[kPReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&bars[kPReady], it & 1)) { ok = false; break; }
         tc_fence_after();
-        mma_dv<D, F16>(tmem + kColDV, tmem + kColS, sm_do + s * L::kTile, it > 0);
+        mma_dv<D, F16>(leader, tmem + kColDV, tmem + kColS, sm_do + s * L::kTile, it > 0);
         if (more) {
-          if (!mbar_wait(&bars[kQFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!FA_WAIT(&bars[kQFull0 + s1], ((it + 1) >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
-          mma_tile_kk<D, F16>(tmem + kColS, sm_k, sm_q + s1 * L::kTile);
-          mma_commit(&bars[kSReady]);
+          mma_tile_kk<D, F16>(leader, tmem + kColS, sm_k, sm_q + s1 * L::kTile);
+          if (leader) mma_commit(&bars[kSReady]);
         }
-        if (!mbar_wait(&bars[kDSReady], it & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&bars[kDSReady], it & 1)) { ok = false; break; }
         tc_fence_after();
         // dQ first: the dK MMA runs while the drain lifts dQ out of TMEM
-        mma_dq<D, F16>(tmem + kColDP, sm_ds, sm_k);
-        mma_commit(&bars[kDQReady]);
-        mma_dk<D, F16>(tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
-        mma_commit(&bars[kEmpty0 + s]);
-        mma_commit(&bars[kDSFree]);
+        mma_dq<D, F16>(leader, tmem + kColDP, sm_ds, sm_k);
+        if (leader) mma_commit(&bars[kDQReady]);
+        mma_dk<D, F16>(leader, tmem + kColDK, sm_ds, sm_q + s * L::kTile, it > 0);
+        if (leader) {
+          mma_commit(&bars[kEmpty0 + s]);
+          mma_commit(&bars[kDSFree]);
+        }
         if (more) {
-          if (!mbar_wait(&bars[kDQFree], it & 1, abort_flag, p.err) ||
-              !mbar_wait(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!FA_WAIT(&bars[kDQFree], it & 1) || !FA_WAIT(&bars[kDOFull0 + s1], ((it + 1) >> 1) & 1)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          mma_tile_kk<D, F16>(tmem + kColDP, sm_v, sm_do + s1 * L::kTile);
-          mma_commit(&bars[kDPReady]);
+          mma_tile_kk<D, F16>(leader, tmem + kColDP, sm_v, sm_do + s1 * L::kTile);
+          if (leader) mma_commit(&bars[kDPReady]);
         }
       }
+#undef FA_WAIT
       if (ok) {
-        mma_commit(&bars[kDKDVReady]);
+        if (leader) mma_commit(&bars[kDKDVReady]);
       } else {
-        mma_commit(&bars[kDrain]);
+        if (leader) mma_commit(&bars[kDrain]);
         mbar_wait_drain(&bars[kDrain], 0);
       }
     }

@@ -306,15 +306,11 @@ __device__ __forceinline__ uint32_t keep_mask_2x16(uint32_t w, DropConst k) {
 // after a left shift by s its bits are the sign bits of bytes 1 and 3 (e = 0)
 // or 0 and 2 (e = 1), which PRMT's sign-replicate mode turns into a 0 / 0xFFFF
 // mask per 16-bit lane (keep_mask_pair).
-template <bool kHighT, int kCalls>
+template <bool kHighT, int kCalls, int kNB = (kCalls < 8) ? kCalls : 8>  // kNB: calls in flight together
 __device__ __forceinline__ void draw_keep_words(uint32_t jb0, const PhiloxFixed123& f, const uint32_t* rk,
                                                 uint32_t c2, uint32_t (&W)[kCalls / 4]) {
   static_assert(kCalls % 4 == 0, "four calls per packed word");
-#ifdef FA_FWD_DRAW_NB
-  constexpr int kNB = (kCalls < FA_FWD_DRAW_NB) ? kCalls : FA_FWD_DRAW_NB;
-#else
-  constexpr int kNB = (kCalls < 8) ? kCalls : 8;  // calls in flight together
-#endif
+  static_assert(kCalls % kNB == 0, "whole lockstep batches");
 #pragma unroll
   for (int k = 0; k < kCalls / 4; ++k) W[k] = 0u;
 #pragma unroll
