@@ -27,11 +27,12 @@
 //    grows by more than 8 (log2 units).  l and O share the stale maximum, so
 //    the result is unchanged; P stays <= 2^8;
 //  * dropout never stores a mask: keep decisions come from Philox keyed on
-//    (seed, b, h, i, j), drawn for a whole tile before its scores are read
-//    (16 calls per row and 128-key tile, 4 in lockstep, while the tensor core
-//    computes S) and applied with a byte permute and an AND per pair of P;
-//    kept P are left unscaled and 1/(1-p) is folded into the final
-//    normalisation.
+//    (seed, b, h, i, j), 16 calls per row and 128-key tile, 4 in lockstep
+//    (the first 4 while the tensor core computes S, the others inside the
+//    exponential loop), tested on the FMA pipe: one byte permute makes the
+//    exact float 2^23 + u of a 16-bit draw u, one saturating add turns it into
+//    the 0.0 / 1.0 keep multiplier.  Kept P are left unscaled and 1/(1-p) is
+//    folded into the final normalisation.
 //  * a causal CTA processes only key tiles up to its diagonal; the grid puts
 //    the heaviest query blocks first;
 //  * queries and keys may differ in number (Nq != Nk, causal alignment
@@ -51,39 +52,11 @@
 namespace fa {
 namespace {
 
-// Keep bits of one row for the 128 keys of a tile (calls jb0 .. jb0 + 15, one
-// Philox call per 8 keys, kNB calls in lockstep), in byte-sign form: kz[m]
-// holds pair 2m's keep bits in the signs of bytes 0, 1 and pair 2m + 1's in
-// bytes 2, 3.  Each Philox word carries two 16-bit draws; the two-lane test of
-// keep_mask_2x16 leaves their keep bits at bits 15 and 31, and one byte
-// permute gathers the four bits of two words.
-template <bool kHighT, int kNB>
-__device__ __forceinline__ void draw_keep_bytes(uint32_t jb0, const PhiloxFixed123& f, const uint32_t* rk,
-                                                uint32_t c2, uint32_t (&kz)[32]) {
-#pragma unroll
-  for (int g0 = 0; g0 < 16; g0 += kNB) {
-    uint32_t w[kNB][4];
-    philox4x32_10_c0_batch<kNB>(jb0 + g0, f, rk, w);
-#pragma unroll
-    for (int n = 0; n < kNB; ++n) {
-      uint32_t z[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t y = (w[n][e] & 0x7FFF7FFFu) + c2;
-        z[e] = kHighT ? (w[n][e] & y) : (w[n][e] | y);
-      }
-      kz[2 * (g0 + n)] = prmt(z[0], z[1], 0x7531u);
-      kz[2 * (g0 + n) + 1] = prmt(z[2], z[3], 0x7531u);
-    }
-  }
-}
-
 constexpr int kBM = 128;             // query rows per tile
 constexpr int kBN = 128;             // keys per tile
 constexpr int kFwdThreads = 384;     // 2 softmax warpgroups + 1 control warpgroup
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
-constexpr int kDrawNB = 4;           // Philox calls in lockstep
 // Register split (setmaxnreg): the kernel launches with kFwdLaunchRegs per
 // thread; softmax warpgroups grow to kSoftmaxRegs, the control warpgroup
 // (MMA, TMA, two idle warps) shrinks to kControlRegs.  The split must fit the
@@ -383,8 +356,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // parts of its first two rounds that do not depend on j are fixed here
       const PhiloxFixed123 phx = philox_fix123(static_cast<uint32_t>(i), static_cast<uint32_t>(su.h),
                                                static_cast<uint32_t>(su.b), p.philox_rk);
-      const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
-      const bool hi_t = p.drop_t > 0x8000u;
+      const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
       // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
       // last key, and under the causal mask the row's position i + Nk - Nq);
       // tiles from t_mask on are the first that can hold a masked key for
@@ -401,17 +373,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       const int ntq = q ? nt1 : nt0;
       for (int t = 0; t < ntq; ++t) {
-        // keep bits of the tile's 128 keys, drawn before S is ready: while the
-        // tensor core computes S the warp would only wait, and the 16 Philox
-        // calls run 8 at a time in lockstep (the S row's registers are free)
-        uint32_t kz[32];
-        if (DROPOUT) {
-          if (hi_t)
-            draw_keep_bytes<true, kDrawNB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
-          else
-            draw_keep_bytes<false, kDrawNB>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, drop_c2, kz);
-          reg_fence32(kz);
-        }
+        // dropout draws: the Philox words of the tile's first 32 keys (4 calls
+        // in lockstep) before S is ready, while the tensor core computes S;
+        // the exponential loop draws each next 32 keys' words while it
+        // exponentiates the current ones
+        uint32_t wn[4][4];
+        if (DROPOUT) philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, wn);
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -467,8 +434,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
+        uint32_t wc[4][4];
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
+          if (DROPOUT && (c & 15) == 0) {
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
+            if (c + 16 < kBN / 2)
+              philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + (c + 16) / 4), phx, p.philox_rk, wn);
+          }
           const float sv0 = s[2 * c], sv1 = s[2 * c + 1];
           float x0, x1;
           f2_unpack(fma_f2(f2_pack(sv0, sv1), sl2x2, negm2), x0, x1);
@@ -479,9 +455,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             rs1 = add_f2(rs1, pp);
           else
             rs0 = add_f2(rs0, pp);
-          pk[c] = pack2<F16>(p0, p1);
-          // dropped keys: zero the 16-bit P (the row sum l keeps them)
-          if (DROPOUT) pk[c] &= prmt(kz[c >> 1], 0u, (c & 1) ? 0xBBAAu : 0x9988u);
+          if (DROPOUT) {
+            // keep test on the FMA pipe: the float 2^23 + u16 is exact, and
+            // sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0;
+            // dropped keys get P = 0 (the row sum l keeps them)
+            const uint32_t wv = wc[(c & 15) >> 2][c & 3];
+            float k0, k1;
+            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k0) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7610u))),
+                "f"(drop_bias));
+            asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7632u))),
+                "f"(drop_bias));
+            float q0, q1;
+            f2_unpack(mul_f2(pp, f2_pack(k0, k1)), q0, q1);
+            pk[c] = pack2<F16>(q0, q1);
+          } else {
+            pk[c] = pack2<F16>(p0, p1);
+          }
+          if (c == kBN / 4 - 1) tmem_st32(t_s, pk);  // the first half of P (S is all in registers)
         }
         {
           float a0, a1;
@@ -504,7 +494,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st32(t_o + c * 32, orow);
           }
         }
-        tmem_st32(t_s, pk);
         tmem_st32(t_s + 32, pk + 32);
         tmem_st_wait();
         tc_fence_before();
