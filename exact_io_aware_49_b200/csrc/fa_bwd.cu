@@ -559,16 +559,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const PhiloxFixed023 phx = philox_fix023(static_cast<uint32_t>((kj * 128 + r) >> 3), static_cast<uint32_t>(su.h),
                                              static_cast<uint32_t>(su.b), p.philox_rk);
     uint32_t zbn[2] = {0u, 0u};
-    auto keep_half = [&](int qi_next, int half) {
-      const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g + 32 * half);
-      zbn[half] = hi_t ? keep_bits_32<true>(phx, q0, p.philox_rk, dk.c2, lane)
-                       : keep_bits_32<false>(phx, q0, p.philox_rk, dk.c2, lane);
+    // both 32-query words of the group's 64 columns (8 Philox calls in lockstep)
+    auto keep_tile = [&](int qi_next) {
+      const uint32_t q0 = static_cast<uint32_t>(qi_next * 128 + 64 * g);
+      if (hi_t)
+        keep_bits<true, 2>(phx, q0, p.philox_rk, dk.c2, lane, zbn);
+      else
+        keep_bits<false, 2>(phx, q0, p.philox_rk, dk.c2, lane, zbn);
     };
     // keep bits of this thread's 64 query columns, computed one tile ahead
     // (at the end of the previous tile, while the warp would wait for S^T)
     if (DROPOUT) {
-      keep_half(qi_of(0), 0);
-      keep_half(qi_of(0), 1);
+      keep_tile(qi_of(0));
     }
     // masking: query i = qi * 128 + c sees this thread's key j = kj * 128 + r
     // iff i + Nk - Nq >= j, i.e. c >= lo0 - qi * 128; query tiles up to qi_mask
@@ -665,8 +667,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kDSReady]);
       if (DROPOUT && it + 1 < nq) {
-        keep_half(qi_of(it + 1), 0);
-        keep_half(qi_of(it + 1), 1);
+        keep_tile(qi_of(it + 1));
       }
     }
     if (ok && mbar_wait(&bars[kDKDVReady], 0, abort_flag, p.err)) {

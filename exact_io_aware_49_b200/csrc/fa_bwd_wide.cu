@@ -304,10 +304,10 @@ __global__ void __launch_bounds__(kWThreads, 1)
     uint32_t zb[2] = {0u, 0u};
     if (DROPOUT) {
       const uint32_t q0 = static_cast<uint32_t>(qt * 64);
-      zb[0] = hi_t ? keep_bits_32<true>(phx, q0, p.philox_rk, dk.c2, lane)
-                   : keep_bits_32<false>(phx, q0, p.philox_rk, dk.c2, lane);
-      zb[1] = hi_t ? keep_bits_32<true>(phx, q0 + 32, p.philox_rk, dk.c2, lane)
-                   : keep_bits_32<false>(phx, q0 + 32, p.philox_rk, dk.c2, lane);
+      if (hi_t)
+        keep_bits<true, 2>(phx, q0, p.philox_rk, dk.c2, lane, zb);
+      else
+        keep_bits<false, 2>(phx, q0, p.philox_rk, dk.c2, lane, zb);
     }
     if (!mbar_wait(&b_full[s], (it / S) & 1, abort_flag, p.err) || !mbar_wait(b_s, it & 1, abort_flag, p.err)) {
       ok = false;

@@ -339,48 +339,57 @@ __device__ __forceinline__ uint32_t keep_mask_pair(const uint32_t (&W)[kWords], 
   return prmt(W[c >> 4] << (cc >> 1), 0u, (cc & 1) ? 0xAA88u : 0xBB99u);
 }
 
-// Keep bits of the dropout mask for this lane's key row and 32 consecutive
-// queries q0 .. q0+31: bit l of the result is keep(key, q0 + l).  ``phx``
+// Keep bits of the dropout mask for this lane's key row and 32 kWords
+// consecutive queries: bit l of W[w] is keep(key, q0 + 32 w + l).  ``phx``
 // holds the per-key-group part of the Philox rounds (counter words key >> 3,
 // h, b are fixed, the query varies).
 //
 // The Philox counter (key >> 3, query, h, b) yields 8 keys x 1 query per call,
 // so lane l8 of each group of 8 consecutive keys evaluates queries
-// q0 + 8 j + l8 (j = 0..3).  Per output word the two 16-bit draws are tested
-// against t with three integer ops (the same two-lane test as the mask
-// export), and a multiply-high on the FMA pipe moves the two keep bits to
-// bits 2e and 16 + 2e of an accumulator.  That gives, per lane, four bytes
-// whose bit k' is keep(key 8 g + k', query q0 + 8 j + l8); a three-stage
-// butterfly of lane shuffles then transposes each 8 x 8 bit block so that lane
-// k' holds bit l = keep(its key, query q0 + 8 j + l).
-template <bool kHighT>
-__device__ __forceinline__ uint32_t keep_bits_32(const PhiloxFixed023& phx, uint32_t q0, const uint32_t* rk,
-                                                 uint32_t c2, int lane) {
+// q0 + 32 w + 8 j + l8 (j = 0..3) for word w.  Per Philox output word the two
+// 16-bit draws are tested against t with three integer ops (the same two-lane
+// test as the mask export), and a multiply-high on the FMA pipe moves the two
+// keep bits to bits 2e and 16 + 2e of an accumulator.  That gives, per lane,
+// four bytes whose bit k' is keep(key 8 g + k', query q0 + 32 w + 8 j + l8); a
+// three-stage butterfly of lane shuffles then transposes each 8 x 8 bit block
+// so that lane k' holds bit l = keep(its key, query q0 + 32 w + 8 j + l).  The
+// 4 kWords Philox calls run in lockstep and the words' butterflies are
+// interleaved, for more independent work per warp.
+template <bool kHighT, int kWords>
+__device__ __forceinline__ void keep_bits(const PhiloxFixed023& phx, uint32_t q0, const uint32_t* rk, uint32_t c2,
+                                          int lane, uint32_t (&W)[kWords]) {
+  constexpr int kCalls = 4 * kWords;
   const uint32_t l8 = static_cast<uint32_t>(lane & 7);
-  uint32_t W = 0;
-  uint32_t cq[4];
+  uint32_t cq[kCalls];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) cq[j] = q0 + 8 * j + l8;
-  uint32_t w4[4][4];
-  philox4x32_10_c1_batch<4>(cq, phx, rk, w4);  // the 4 calls in lockstep
+  for (int j = 0; j < kCalls; ++j) cq[j] = q0 + 8 * j + l8;
+  uint32_t wv[kCalls][4];
+  philox4x32_10_c1_batch<kCalls>(cq, phx, rk, wv);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint32_t acc = 0;
+  for (int w = 0; w < kWords; ++w) {
+    W[w] = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t y = (w4[j][e] & 0x7FFF7FFFu) + c2;
-      const uint32_t zm = (kHighT ? (w4[j][e] & y) : (w4[j][e] | y)) & 0x80008000u;  // keep bits at 15 and 31
-      acc = mad_hi_u32(zm, 1u << (17 + 2 * e), acc);                                  // -> bits 2e and 16 + 2e
+    for (int j = 0; j < 4; ++j) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = wv[4 * w + j][e];
+        const uint32_t y = (x & 0x7FFF7FFFu) + c2;
+        const uint32_t zm = (kHighT ? (x & y) : (x | y)) & 0x80008000u;  // keep bits at 15 and 31
+        acc = mad_hi_u32(zm, 1u << (17 + 2 * e), acc);                    // -> bits 2e and 16 + 2e
+      }
+      W[w] |= ((acc | (acc >> 15)) & 0xFFu) << (8 * j);
     }
-    W |= ((acc | (acc >> 15)) & 0xFFu) << (8 * j);
   }
 #pragma unroll
   for (int sh = 4; sh >= 1; sh >>= 1) {
     const uint32_t lo = (sh == 4) ? 0x0F0F0F0Fu : ((sh == 2) ? 0x33333333u : 0x55555555u);
-    const uint32_t y = __shfl_xor_sync(0xffffffffu, W, sh);
-    W = (l8 & sh) ? ((W & ~lo) | ((y >> sh) & lo)) : ((W & lo) | ((y << sh) & ~lo));
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) {
+      const uint32_t y = __shfl_xor_sync(0xffffffffu, W[w], sh);
+      W[w] = (l8 & sh) ? ((W[w] & ~lo) | ((y >> sh) & lo)) : ((W[w] & lo) | ((y << sh) & ~lo));
+    }
   }
-  return W;
 }
 
 // Marks dropped entries by setting the sign bit of P: for 4 columns whose keep
