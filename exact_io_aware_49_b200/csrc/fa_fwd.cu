@@ -27,11 +27,13 @@
 //    grows by more than 8 (log2 units).  l and O share the stale maximum, so
 //    the result is unchanged; P stays <= 2^8;
 //  * dropout never stores a mask: keep decisions come from Philox keyed on
-//    (seed, b, h, i, j), 16 calls per row and 128-key tile, 4 in lockstep
-//    (the first 4 while the tensor core computes S, the others inside the
-//    exponential loop), tested on the FMA pipe: one byte permute makes the
-//    exact float 2^23 + u of a 16-bit draw u, one saturating add turns it into
-//    the 0.0 / 1.0 keep multiplier.  Kept P are left unscaled and 1/(1-p) is
+//    (seed, b, h, i, j), 16 calls per row and 128-key tile, 4 in lockstep.
+//    The first 8 (d = 128) or 4 (d = 64) run while the tensor core computes
+//    S and become byte-sign masks (an integer test, an AND per pair of P);
+//    the others run inside the exponential loop, one chunk of 32 keys ahead,
+//    and are tested on the FMA pipe: one byte permute makes the exact float
+//    2^23 + u of a 16-bit draw u, one saturating add turns it into the
+//    0.0 / 1.0 keep multiplier.  Kept P are left unscaled and 1/(1-p) is
 //    folded into the final normalisation.
 //  * a causal CTA processes only key tiles up to its diagonal; the grid puts
 //    the heaviest query blocks first;
@@ -357,6 +359,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const PhiloxFixed123 phx = philox_fix123(static_cast<uint32_t>(i), static_cast<uint32_t>(su.h),
                                                static_cast<uint32_t>(su.b), p.philox_rk);
       const float drop_bias = -(8388608.0f + static_cast<float>(p.drop_t) - 1.0f);
+      // dropout: Philox calls drawn before S is ready (while the tensor core
+      // computes S); the rest run inside the exponential loop.  At d = 128 the
+      // wait for S is long enough for 8, at d = 64 for 4.
+      constexpr int kPre = (D == 128) ? 8 : 4;
+      const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
+      const uint32_t drop_m0 = make_drop_const(p.drop_t).m0;
       // masking: key j = t * kBN + c is visible to this row iff j <= lim0 (the
       // last key, and under the causal mask the row's position i + Nk - Nq);
       // tiles from t_mask on are the first that can hold a masked key for
@@ -373,12 +381,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       const int ntq = q ? nt1 : nt0;
       for (int t = 0; t < ntq; ++t) {
-        // dropout draws: the Philox words of the tile's first 32 keys (4 calls
-        // in lockstep) before S is ready, while the tensor core computes S;
-        // the exponential loop draws each next 32 keys' words while it
-        // exponentiates the current ones
-        uint32_t wn[4][4];
-        if (DROPOUT) philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8)), phx, p.philox_rk, wn);
+        // dropout draws: the first kPre calls (8 kPre keys, 4 in lockstep)
+        // before S is ready, while the tensor core computes S.  Their keep
+        // test is the two-lane integer test of keep_mask_2x16 (m0 selects the
+        // threshold side at run time), gathered into byte-sign words: kz[2g]
+        // holds keys 8g .. 8g+3 in the signs of its bytes, kz[2g+1] keys
+        // 8g+4 .. 8g+7.
+        uint32_t kz[2 * kPre];
+        if (DROPOUT) {
+#pragma unroll
+          for (int g0 = 0; g0 < kPre; g0 += 4) {
+            uint32_t w[4][4];
+            philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + g0), phx, p.philox_rk, w);
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+              uint32_t z[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t y = (w[n][e] & 0x7FFF7FFFu) + drop_c2;
+                z[e] = (w[n][e] & y) | ((w[n][e] | y) & drop_m0);
+              }
+              kz[2 * (g0 + n)] = prmt(z[0], z[1], 0x7531u);
+              kz[2 * (g0 + n) + 1] = prmt(z[2], z[3], 0x7531u);
+            }
+          }
+        }
         if (!mbar_wait(&bar.s_ready[q], t & 1, abort_flag, p.err)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[128];
@@ -434,16 +461,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
         uint64_t rs0 = 0ull, rs1 = 0ull;
-        uint32_t wc[4][4];
+        // the other calls inside the exponential loop, 4 at a time, 32 keys
+        // ahead of the pairs that use them (chunk k = pairs 16k .. 16k + 15)
+        uint32_t wn[4][4], wc[4][4];
 #pragma unroll
         for (int c = 0; c < kBN / 2; ++c) {
           if (DROPOUT && (c & 15) == 0) {
+            const int k = c >> 4;  // chunk of this pair
+            if (k >= kPre / 4) {
 #pragma unroll
-            for (int n = 0; n < 4; ++n)
+              for (int n = 0; n < 4; ++n)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
-            if (c + 16 < kBN / 2)
-              philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + (c + 16) / 4), phx, p.philox_rk, wn);
+                for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
+            }
+            // chunk k + kPre / 4 is drawn while this chunk is exponentiated
+            // (chunk kPre / 4 during the chunk before it)
+            const int kd = (k + 1 >= kPre / 4) ? k + 1 : -1;
+            if (kd >= kPre / 4 && kd < kBN / 32)
+              philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + 4 * kd), phx, p.philox_rk, wn);
           }
           const float sv0 = s[2 * c], sv1 = s[2 * c + 1];
           float x0, x1;
@@ -455,7 +490,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             rs1 = add_f2(rs1, pp);
           else
             rs0 = add_f2(rs0, pp);
-          if (DROPOUT) {
+          if (DROPOUT && c < 4 * kPre) {
+            // keys of the calls drawn before S: the byte signs of kz spread
+            // over 16-bit lanes (PRMT sign mode) zero the dropped P
+            pk[c] = pack2<F16>(p0, p1) & prmt(kz[c >> 1], 0u, (c & 1) ? 0xBBAAu : 0x9988u);
+          } else if (DROPOUT) {
             // keep test on the FMA pipe: the float 2^23 + u16 is exact, and
             // sat((2^23 + u) - (2^23 + t - 1)) is 1.0 when u >= t, else 0.0;
             // dropped keys get P = 0 (the row sum l keeps them)
