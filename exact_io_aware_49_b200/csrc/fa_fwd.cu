@@ -474,8 +474,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) wc[n][e] = wn[n][e];
             }
-            // chunk k + kPre / 4 is drawn while this chunk is exponentiated
-            // (chunk kPre / 4 during the chunk before it)
+            // the next chunk's words are drawn while this chunk is
+            // exponentiated (chunks from kPre / 4 on come from here)
             const int kd = (k + 1 >= kPre / 4) ? k + 1 : -1;
             if (kd >= kPre / 4 && kd < kBN / 32)
               philox4x32_10_c0_batch<4>(static_cast<uint32_t>(t * (kBN / 8) + 4 * kd), phx, p.philox_rk, wn);
