@@ -103,8 +103,11 @@ def test_backward_applies_oracle_mask_every_query(causal, N, d, p, seed):
     _backward_mask_windows(2, 3, N, d, causal, p, seed, list(range(0, N, d)))
 
 
+@pytest.mark.parametrize("causal,p", [(True, 0.1), (False, 0.7)])
 @pytest.mark.parametrize("B,H,N,seed", [(4, 16, 4096, 2), (1, 32, 32768, 4)])
-def test_backward_applies_oracle_mask_full_size(B, H, N, seed):
-    """The two dropout workloads' shapes (d = 128, causal, p = 0.1): sampled
-    windows at the start, in the middle and at the end, on every head."""
-    _backward_mask_windows(B, H, N, 128, True, 0.1, seed, [0, N // 2 - 64, N - 128])
+def test_backward_applies_oracle_mask_full_size(B, H, N, seed, causal, p):
+    """The two dropout workloads' shapes (d = 128): sampled windows at the
+    start, in the middle and at the end, on every head; the workloads' own
+    causal p = 0.1 and a non-causal p = 0.7 case (every key visible, most of
+    them dropped)."""
+    _backward_mask_windows(B, H, N, 128, causal, p, seed, [0, N // 2 - 64, N - 128])
