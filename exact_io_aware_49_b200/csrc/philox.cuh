@@ -45,29 +45,6 @@ __device__ __forceinline__ void philox4x32_10(uint32_t c0, uint32_t c1, uint32_t
   out[3] = c3;
 }
 
-// The same generator with its round keys precomputed (they are the same for
-// every thread of a launch): rk[2r], rk[2r + 1] = (k0 + r W0, k1 + r W1) mod
-// 2^32 for rounds r = 0..9.  ``rk`` points at kernel parameter space, so each
-// key is an operand read from the constant bank, not a register.
-__device__ __forceinline__ void philox4x32_10_rk(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
-                                                 const uint32_t* rk, uint32_t (&out)[4]) {
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    const uint32_t hi0 = __umulhi(kPhiloxM0, c0);
-    const uint32_t lo0 = kPhiloxM0 * c0;
-    const uint32_t hi1 = __umulhi(kPhiloxM1, c2);
-    const uint32_t lo1 = kPhiloxM1 * c2;
-    c0 = hi1 ^ c1 ^ rk[2 * r];
-    c1 = lo1;
-    c2 = hi0 ^ c3 ^ rk[2 * r + 1];
-    c3 = lo0;
-  }
-  out[0] = c0;
-  out[1] = c1;
-  out[2] = c2;
-  out[3] = c3;
-}
-
 // Philox4x32-10 for calls that share counter words c1, c2, c3 and differ in
 // c0 only (one query row of one head: counter (j >> 3, i, h, b)).  With c2
 // fixed, round 0's second product is the same for every call, and so is round
