@@ -14,7 +14,7 @@ FLOPs per step: forward 4*B*H*N^2*d/2 (causal), backward 2.5x the forward.
             CUDA events on the launching stream (max over ranks)
   e2e       the same through the C ABI's host-buffer call fa_fwd_bwd_host:
             each step copies Q, K, V, dO host->device from pinned memory and
-            O, LSE, dQ, dK, dV back, in 8 groups of heads whose copies overlap
+            O, LSE, dQ, dK, dV back, in 16 groups of heads whose copies overlap
             the kernels of the neighbouring groups on three streams
   roofline  the kernel with the largest share of the step, achieved TFLOP/s
             from its own CUDA events against the measured bf16 burst peak
@@ -69,7 +69,7 @@ FWD_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_fwd.cu")
 DECODE_SOURCE = os.path.join(ROOT, "exact_io_aware_49_b200", "csrc", "fa_decode.cu")
 DECODE_WORKLOAD = "decode_paged_B16_L32768_H32_Hkv8_d128"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-E2E_GROUPS = 8  # head groups of the host-buffer step (copies of one overlap the kernels of the next)
+E2E_GROUPS = 16  # head groups of the host-buffer step (copies of one overlap the kernels of the next)
 
 
 def _peaks():
