@@ -20,8 +20,10 @@
 //   * S^T = K_tile Q^T   (tcgen05, A = K tile, B = Q rows, fp32 in TMEM:
 //     lane = key, column = query row);
 //   * softmax over keys, i.e. across TMEM lanes: each of 128 threads holds
-//     one key's 16 scores, a 16-shuffle reduce-scatter per warp and one
-//     exchange through shared memory give every row's tile max and sum; the
+//     one key's scores of the CTA's rows (4, 8 or 16 columns: the kernel is
+//     instantiated for the row count, the products keep N = 16), a
+//     reduce-scatter of shuffles per warp and one exchange through shared
+//     memory give every row's tile max and sum; the
 //     O rescale is lazy (stale max kept until a row's max grows by more than
 //     8 in log2 units, as in the forward kernel); P goes to shared memory as
 //     16-bit [16 rows x 128 keys];
@@ -75,50 +77,83 @@ struct DecSmem {
   static constexpr int kUsed = kMisc + 16;
 };
 
-// Reduce-scatter of 16 per-lane values over a warp: afterwards the lanes with
-// bit 0 clear hold the warp-wide max (kMax) or sum of column
-// col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1).
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce_scatter16(float (&v)[16], int lane) {
-  float a[8], b4[4], c2[2];
-  const bool up16 = lane & 16, up8 = lane & 8, up4 = lane & 4, up2 = lane & 2;
+// Reduce-scatter of kRows per-lane values over a warp (kRows = 4, 8 or 16):
+// log2(kRows) exchange steps (lane bits 4, 3, ...) each halve the values a
+// lane holds, then plain butterfly steps over the remaining lane bits finish
+// the reduction.  Afterwards every lane holds the warp-wide max (kMax) or sum
+// of column scatter_col<kRows>(lane).
+template <bool kMax, int kRows>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[kRows], int lane) {
+  static_assert(kRows == 4 || kRows == 8 || kRows == 16, "rows per CTA");
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float send = up16 ? v[k] : v[k + 8];
-    const float keep = up16 ? v[k + 8] : v[k];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-    a[k] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
+  for (int lvl = 0; (kRows >> lvl) > 1; ++lvl) {
+    const int half = kRows >> (lvl + 1);
+    const int sh = 16 >> lvl;
+    const bool up = lane & sh;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float send = up8 ? a[k] : a[k + 4];
-    const float keep = up8 ? a[k + 4] : a[k];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-    b4[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+    for (int k = 0; k < half; ++k) {
+      const float send = up ? v[k] : v[k + half];
+      const float keep = up ? v[k + half] : v[k];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, sh);
+      v[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
   }
+  float d = v[0];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float send = up4 ? b4[k] : b4[k + 2];
-    const float keep = up4 ? b4[k + 2] : b4[k];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-    c2[k] = kMax ? fmaxf(keep, recv) : keep + recv;
+  for (int sh = 16 / kRows; sh >= 1; sh >>= 1) {
+    const float recv = __shfl_xor_sync(0xffffffffu, d, sh);
+    d = kMax ? fmaxf(d, recv) : d + recv;
   }
-  float d;
-  {
-    const float send = up2 ? c2[0] : c2[1];
-    const float keep = up2 ? c2[1] : c2[0];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-    d = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
-  const float recv = __shfl_xor_sync(0xffffffffu, d, 1);
-  return kMax ? fmaxf(d, recv) : d + recv;
+  return d;
 }
 
+template <int kRows>
 __device__ __forceinline__ int scatter_col(int lane) {
-  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+  constexpr int kShift = (kRows == 16) ? 1 : ((kRows == 8) ? 2 : 3);
+  return (lane >> kShift) & (kRows - 1);
 }
 
-template <int D, bool F16>
+// kN consecutive TMEM columns of this warp's 32 lanes (32x32b shape, kN = 4, 8, 16).
+template <int kN>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[kN]) {
+  if constexpr (kN == 16) {
+    tmem_ld16(taddr, r);
+  } else if constexpr (kN == 8) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+  } else {
+    static_assert(kN == 4, "columns");
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+  }
+}
+
+template <int kN>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[kN]) {
+  if constexpr (kN == 16) {
+    tmem_st16(taddr, r);
+  } else if constexpr (kN == 8) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+  } else {
+    static_assert(kN == 4, "columns");
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+  }
+}
+
+// Keeps the consumers of r after the preceding tmem_ld_wait() (see reg_fence32).
+template <int kN>
+__device__ __forceinline__ void reg_fence_cols(uint32_t (&r)[kN]) {
+#pragma unroll
+  for (int k = 0; k < kN; ++k) asm volatile("" : "+r"(r[k]));
+}
+
+template <int D, bool F16, int kRows>
 __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                   const __grid_constant__ CUtensorMap tmV,
                                                                   const __grid_constant__ DecodeParams p) {
@@ -178,6 +213,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
     }
     *reinterpret_cast<uint4*>(qsm + (c8 / 8) * (kMaxRows * 128) + r * 128 + (((c8 % 8) ^ (r & 7)) << 4)) = v;
   }
+  // P rows from kRows on are never written by the softmax: zero both buffers
+  // once, so the P V product reads zeros there
+  if (kRows < kMaxRows)
+    for (int idx = tid; idx < 2 * L::kPBytes / 16; idx += kDecThreads)
+      *reinterpret_cast<uint4*>(smem + L::kP + idx * 16) = make_uint4(0u, 0u, 0u, 0u);
   if (D == 64) {
     // the second V box of every stage stays zero
     for (int idx = tid; idx < S * (L::kBox / 16); idx += kDecThreads) {
@@ -201,17 +241,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      auto issue = [&](int it) {
-        const int st = it % S;
+      // a tile's page ids are read from the block table one refill ahead of
+      // its copies, so the copies never wait for those reads
+      constexpr int kMaxPagesPerTile = kTileKeys / 16;
+      auto pages_of = [&](int it) {
         const int first = (t_begin + it) * kTileKeys;
-        const int pages_here = min(kTileKeys / p.page, (Lk - first + p.page - 1) / p.page);
-        // read the tile's page ids first: the copies below are ordered after
-        // every earlier memory access, so interleaving would serialise the reads
-        constexpr int kMaxPagesPerTile = kTileKeys / 16;
-        int pids[kMaxPagesPerTile];
+        return min(kTileKeys / p.page, (Lk - first + p.page - 1) / p.page);
+      };
+      auto read_pids = [&](int it, int (&ids)[kMaxPagesPerTile]) {
+        const int first = (t_begin + it) * kTileKeys;
+        const int pages_here = pages_of(it);
         const int* bt = p.block_table + static_cast<size_t>(b) * p.max_pages + first / p.page;
 #pragma unroll
-        for (int pg = 0; pg < kMaxPagesPerTile; ++pg) pids[pg] = (pg < pages_here) ? bt[pg] : 0;
+        for (int pg = 0; pg < kMaxPagesPerTile; ++pg) ids[pg] = (pg < pages_here) ? bt[pg] : 0;
+      };
+      auto issue = [&](int it, const int (&pids)[kMaxPagesPerTile]) {
+        const int st = it % S;
+        const int pages_here = pages_of(it);
         // K and V complete separately: S^T needs only K, so it starts while V is still arriving
         mbar_expect_tx(&kfull[st], static_cast<uint32_t>(pages_here * (D / 64) * p.page * 128));
         mbar_expect_tx(&vfull[st], static_cast<uint32_t>(pages_here * (D / 64) * p.page * 128));
@@ -231,7 +277,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       constexpr uint32_t idesc_s = idesc_f32acc(128, kMaxRows, false, false, F16);
       constexpr uint32_t idesc_o = idesc_f32acc(128, kMaxRows, true, false, F16);
       int issued = 0;
-      for (; issued < min(S - 1, n); ++issued) issue(issued);
+      int pids_next[kMaxPagesPerTile];
+      for (; issued < min(S - 1, n); ++issued) {
+        read_pids(issued, pids_next);
+        issue(issued, pids_next);
+      }
+      if (issued < n) read_pids(issued, pids_next);
       bool ok = true;
       int consumed = 0;  // tiles whose copies have landed
       // S^T = K Q^T of tile it into its TMEM buffer: M = 128 keys, N = 16 rows, K = D (both K-major)
@@ -253,18 +304,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       };
       ok = issue_s(0);
       for (int it = 0; ok && it < n; ++it) {
-        // the next tile's S^T runs while the softmax warps work on this one; its
-        // buffer was last read by the softmax of tile it - 1 (p_ready seen below)
-        if (it + 1 < n && !issue_s(it + 1)) { ok = false; break; }
         // refill the stage of tile it - 1 once its P V product has read it
+        // (before waiting for the next tile's K, so the copies go out early)
         if (issued < n) {
           if (it >= 1 && !mbar_wait(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
-          issue(issued);
+          issue(issued, pids_next);
           ++issued;
+          if (issued < n) read_pids(issued, pids_next);
         }
+        // the next tile's S^T runs while the softmax warps work on this one; its
+        // buffer was last read by the softmax of tile it - 1 (p_ready seen below)
+        if (it + 1 < n && !issue_s(it + 1)) { ok = false; break; }
         if (!mbar_wait(&p_ready[it & 1], (it >> 1) & 1, abort_flag, p.err) ||
             !mbar_wait(&vfull[it % S], (it / S) & 1, abort_flag, p.err)) {
           ok = false;
@@ -294,18 +347,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
   } else {
     // ------------------------------------------------------------ softmax warps
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m_st[kMaxRows], l_r[kMaxRows];  // per row: stale max (log2 units) and sum, same in every thread
+    // only the first kRows >= R columns of S^T and O^T carry rows of this CTA
+    float m_st[kRows], l_r[kRows];  // per row: stale max (log2 units) and sum, same in every thread
 #pragma unroll
-    for (int c = 0; c < kMaxRows; ++c) {
+    for (int c = 0; c < kRows; ++c) {
       m_st[c] = -CUDART_INF_F;
       l_r[c] = 0.f;
     }
-    const int col = scatter_col(lane);
+    const int col = scatter_col<kRows>(lane);
     // last visible position of each row: the cached length, and under the
     // causal mask the row's own position Lk - Nq + i; rows past R see nothing
-    int lim[kMaxRows];
+    int lim[kRows];
 #pragma unroll
-    for (int c = 0; c < kMaxRows; ++c) {
+    for (int c = 0; c < kRows; ++c) {
       const int i = (r0 + c) % p.Nq;
       lim[c] = (c >= R) ? -1 : (p.causal ? min(Lk - 1, Lk - p.Nq + i) : Lk - 1);
     }
@@ -321,22 +375,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       ok = named_bar_and(1, 128, mbar_wait(&s_ready[it & 1], (it >> 1) & 1, abort_flag, p.err));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[16];
-      tmem_ld16(tmem + (it & 1) * 16 + lane_base, sr);
+      uint32_t sr[kRows];
+      tmem_ld_cols<kRows>(tmem + (it & 1) * 16 + lane_base, sr);
       tmem_ld_wait();
-      reg_fence16(sr);
-      float s[16];
+      reg_fence_cols<kRows>(sr);
+      float s[kRows];
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) s[c] = (pos <= lim[c]) ? __uint_as_float(sr[c]) * p.scale_log2 : -CUDART_INF_F;
+      for (int c = 0; c < kRows; ++c) s[c] = (pos <= lim[c]) ? __uint_as_float(sr[c]) * p.scale_log2 : -CUDART_INF_F;
       // tile max per row: reduce over this warp's keys, then over the 4 warps
       float* rmax = red + ((it & 1) * 2 + 0) * kMaxRows * 4;
       float* rsum = red + ((it & 1) * 2 + 1) * kMaxRows * 4;
       {
-        float v[16];
+        float v[kRows];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = s[c];
-        const float wm = warp_reduce_scatter16<true>(v, lane);
-        if (!(lane & 1)) rmax[col * 4 + warp] = wm;
+        for (int c = 0; c < kRows; ++c) v[c] = s[c];
+        const float wm = warp_reduce_scatter<true, kRows>(v, lane);
+        if ((lane & (32 / kRows - 1)) == 0) rmax[col * 4 + warp] = wm;
       }
       // V rows of positions past the sequence (or of pages not loaded) may
       // hold anything, NaN included, and 0 * NaN would reach O through the
@@ -357,10 +411,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       const bool p_free = (it < 2) || mbar_wait(&pv_done[it & 1], ((it - 2) >> 1) & 1, abort_flag, p.err);
       ok = named_bar_and(1, 128, p_free && v_ok);
       if (!ok) break;
-      float alpha[kMaxRows];
+      float alpha[kRows];
       bool rescale = false;  // the same in every thread: computed from the same shared values
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) {
+      for (int c = 0; c < kRows; ++c) {
         const float4 w4 = *reinterpret_cast<const float4*>(rmax + c * 4);
         const float m_tile = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
         const float m_new = fmaxf(m_st[c], m_tile);
@@ -371,9 +425,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
           rescale = true;
         }
       }
-      float pv[16];
+      float pv[kRows];
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) {
+      for (int c = 0; c < kRows; ++c) {
         const float mu = (m_st[c] == -CUDART_INF_F) ? 0.f : m_st[c];
         pv[c] = ex2_approx(s[c] - mu);  // 0 for masked keys
       }
@@ -381,18 +435,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       {
         const int box = j / 64, kin = j % 64;
 #pragma unroll
-        for (int c = 0; c < kMaxRows; ++c) {
+        for (int c = 0; c < kRows; ++c) {
           const uint32_t bits = pack2<F16>(pv[c], 0.f);
           *reinterpret_cast<uint16_t*>(psm + box * (kMaxRows * 128) + c * 128 + (((kin >> 3) ^ (c & 7)) << 4) +
                                        (kin & 7) * 2) = static_cast<uint16_t>(bits & 0xFFFFu);
         }
       }
       {
-        float v[16];
+        float v[kRows];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = pv[c];
-        const float ws = warp_reduce_scatter16<false>(v, lane);
-        if (!(lane & 1)) rsum[col * 4 + warp] = ws;
+        for (int c = 0; c < kRows; ++c) v[c] = pv[c];
+        const float ws = warp_reduce_scatter<false, kRows>(v, lane);
+        if ((lane & (32 / kRows - 1)) == 0) rsum[col * 4 + warp] = ws;
       }
       // rescale O^T (lane = dimension) when a row's max moved: the previous
       // P V product must have finished
@@ -401,19 +455,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
       ok = named_bar_and(1, 128, prev_done);  // also: every row sum partial is written
       if (!ok) break;
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) {
+      for (int c = 0; c < kRows; ++c) {
         const float4 w4 = *reinterpret_cast<const float4*>(rsum + c * 4);
         l_r[c] = l_r[c] * alpha[c] + ((w4.x + w4.y) + (w4.z + w4.w));
       }
       if (rescale && it > 0) {
         tc_fence_after();
-        uint32_t orow[16];
-        tmem_ld16(tm_o + lane_base, orow);
+        uint32_t orow[kRows];
+        tmem_ld_cols<kRows>(tm_o + lane_base, orow);
         tmem_ld_wait();
-        reg_fence16(orow);
+        reg_fence_cols<kRows>(orow);
 #pragma unroll
-        for (int c = 0; c < kMaxRows; ++c) orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha[c]);
-        tmem_st16(tm_o + lane_base, orow);
+        for (int c = 0; c < kRows; ++c) orow[c] = __float_as_uint(__uint_as_float(orow[c]) * alpha[c]);
+        tmem_st_cols<kRows>(tm_o + lane_base, orow);
         tmem_st_wait();
       }
       fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
@@ -425,22 +479,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
     if (ok && n > 0)
       ok = named_bar_and(1, 128, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.err));
     if (ok) {
-      float o[16];
+      float o[kRows];
       if (n > 0) {
         tc_fence_after();
-        uint32_t orow[16];
-        tmem_ld16(tm_o + lane_base, orow);
+        uint32_t orow[kRows];
+        tmem_ld_cols<kRows>(tm_o + lane_base, orow);
         tmem_ld_wait();
-        reg_fence16(orow);
+        reg_fence_cols<kRows>(orow);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) o[c] = __uint_as_float(orow[c]);
+        for (int c = 0; c < kRows; ++c) o[c] = __uint_as_float(orow[c]);
       } else {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) o[c] = 0.f;
+        for (int c = 0; c < kRows; ++c) o[c] = 0.f;
       }
       const int dim = warp * 32 + lane;
 #pragma unroll
-      for (int c = 0; c < kMaxRows; ++c) {
+      for (int c = 0; c < kRows; ++c) {
         if (c >= R) continue;
         const int rr = r0 + c;
         const int h = g * p.group + rr / p.Nq, i = rr - (rr / p.Nq) * p.Nq;
@@ -514,9 +568,9 @@ __global__ void __launch_bounds__(256) fa_decode_merge_kernel(const float* __res
   }
 }
 
-template <int D, bool F16>
+template <int D, bool F16, int kRows>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
-  auto kern = fa_decode_kernel<D, F16>;
+  auto kern = fa_decode_kernel<D, F16, kRows>;
   const int smem = DecSmem<D>::kUsed + 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -535,9 +589,19 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+template <int D, bool F16>
+cudaError_t launch_decode_rows(const DecodeArgs& a, cudaStream_t stream) {
+  // the softmax handles only as many S^T / O^T columns as a CTA has rows
+  // (query heads per key/value head times queries, up to 16 per CTA)
+  const int rows = a.p.row_chunks > 1 ? kMaxRows : a.p.rows;
+  if (rows <= 4) return launch_decode_t<D, F16, 4>(a, stream);
+  if (rows <= 8) return launch_decode_t<D, F16, 8>(a, stream);
+  return launch_decode_t<D, F16, 16>(a, stream);
+}
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  if (a.d <= 64) return a.f16 ? launch_decode_t<64, true>(a, stream) : launch_decode_t<64, false>(a, stream);
-  return a.f16 ? launch_decode_t<128, true>(a, stream) : launch_decode_t<128, false>(a, stream);
+  if (a.d <= 64) return a.f16 ? launch_decode_rows<64, true>(a, stream) : launch_decode_rows<64, false>(a, stream);
+  return a.f16 ? launch_decode_rows<128, true>(a, stream) : launch_decode_rows<128, false>(a, stream);
 }
 
 int decode_rows_per_cta() { return kMaxRows; }
