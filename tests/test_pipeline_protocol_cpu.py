@@ -431,13 +431,14 @@ class Decode(Protocol):
             issued += 1
         yield from self.issue_s(0)
         for it in range(n):
-            if it + 1 < n:
-                yield from self.issue_s(it + 1)
+            # the freed stage is refilled before the wait for the next tile's K
             if issued < n:
                 if it >= 1 and self.slip != "no_refill_wait":
                     yield ("wait", self.pv_done[(it - 1) & 1], (it - 1) >> 1)
                 self.load(issued)
                 issued += 1
+            if it + 1 < n:
+                yield from self.issue_s(it + 1)
             if self.slip == "single_p_ready":
                 yield ("wait", self.p_ready[0], it)
             else:
