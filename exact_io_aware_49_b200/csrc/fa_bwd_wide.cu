@@ -64,30 +64,39 @@ __device__ __forceinline__ void wide_bwd_teardown(uint32_t tmem, bool dealloc) {
   if (dealloc) tmem_dealloc(tmem, 512);
 }
 
+// MMA helpers.  The MMA warps run their loops with all 32 lanes, so
+// descriptors are warp-uniform values; ``leader`` (one elected lane) issues.
+// Operands are descriptors of the tile's first box; each K-step adds its box
+// / swizzle-atom offset (bytes / 16) to the start-address field.
+
 // D[tmem] (+)= A * B^T over K = D (both K-major): A has 128 rows in 128-row
-// boxes, B has 64 rows in 64-row boxes; N = 64.
+// boxes, B has 64 rows in 64-row boxes; N = 64.  a0 / b0: sdesc_sw128(x, 16, 1024).
 template <int D, bool F16>
-__device__ __forceinline__ void mma_rows128_x_rows64(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+__device__ __forceinline__ void mma_rows128_x_rows64(bool leader, uint32_t tmem_d, uint64_t a0, uint64_t b0) {
   constexpr uint32_t idesc = idesc_f32acc(128, 64, false, false, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t a = a_smem + (kk / 4) * kBox128 + (kk % 4) * 32;
-    const uint32_t b = b_smem + (kk / 4) * kBox64 + (kk % 4) * 32;
-    mma_ss(tmem_d, sdesc_sw128(a, 16, 1024), sdesc_sw128(b, 16, 1024), idesc, kk > 0);
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(tmem_d, a0 + static_cast<uint32_t>(((kk / 4) * kBox128 + (kk % 4) * 32) >> 4),
+             b0 + static_cast<uint32_t>(((kk / 4) * kBox64 + (kk % 4) * 32) >> 4), idesc, kk > 0);
   }
 }
 
 // D[tmem] (+)= A[tmem, 16-bit pairs] * B over K = 64 rows of B, N = NC columns
-// of B starting at box ``box0`` (B MN-major in 64-row boxes 8 KB apart).
+// of B (B MN-major in 64-row boxes 8 KB apart); b0: sdesc_sw128(first box, kBox64, 1024).
 template <int NC, bool F16>
-__device__ __forceinline__ void mma_tmemA_x_rows64(uint32_t tmem_d, uint32_t tmem_a, uint32_t b_smem, int box0,
+__device__ __forceinline__ void mma_tmemA_x_rows64(bool leader, uint32_t tmem_d, uint32_t tmem_a, uint64_t b0,
                                                    bool accumulate) {
   constexpr uint32_t idesc = idesc_f32acc(128, NC, false, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk)
-    mma_ts(tmem_d, tmem_a + kk * 8, sdesc_sw128(b_smem + box0 * kBox64 + kk * 2048, kBox64, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ts(tmem_d, tmem_a + kk * 8, b0 + static_cast<uint32_t>((kk * 2048) >> 4), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
+
+__device__ __forceinline__ uint64_t desc_off(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // ============================================================ kernel 1: dK, dV
 
@@ -235,48 +244,61 @@ __global__ void __launch_bounds__(kWThreads, 1)
     return;
   }
   if (warp == kWMma) {
-    if (lane == 0) {
-      bool ok = mbar_wait(b_kv, 0, abort_flag, p.err) && mbar_wait(&b_full[0], 0, abort_flag, p.err);
+    {
+      const bool leader = elect_one();
+      const uint64_t dk_k = sdesc_sw128(sm_k, 16, 1024), dk_v = sdesc_sw128(sm_v, 16, 1024);
+      const uint64_t dk_q = sdesc_sw128(sm_q, 16, 1024), dk_do = sdesc_sw128(sm_do, 16, 1024);
+      const uint64_t dk_ds = sdesc_sw128(sm_ds, 16, 1024);
+      const uint64_t dmn_q = sdesc_sw128(sm_q, kBox64, 1024), dmn_do = sdesc_sw128(sm_do, kBox64, 1024);
+      const uint32_t col_off = hc * (NC / 64) * kBox64;  // this CTA's output columns
+      // every lane waits; the vote keeps the warp's decision uniform
+#define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
+      bool ok = FA_WAIT(b_kv, 0) && FA_WAIT(&b_full[0], 0);
       if (ok) {
         tc_fence_after();
-        mma_rows128_x_rows64<D, F16>(tmem + kColS, sm_k, sm_q);
-        mma_commit(b_s);
-        mma_rows128_x_rows64<D, F16>(tmem + kColDP, sm_v, sm_do);
-        mma_commit(b_dp);
+        mma_rows128_x_rows64<D, F16>(leader, tmem + kColS, dk_k, dk_q);
+        if (leader) mma_commit(b_s);
+        mma_rows128_x_rows64<D, F16>(leader, tmem + kColDP, dk_v, dk_do);
+        if (leader) mma_commit(b_dp);
       }
       for (int it = 0; ok && it < nq; ++it) {
         const int s = it % S;
-        if (!mbar_wait(b_p, it & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(b_p, it & 1)) { ok = false; break; }
         tc_fence_after();
         // dV += P^T dO (this CTA's columns)
-        mma_tmemA_x_rows64<NC, F16>(tmem + kColDV, tmem + kColS, sm_do + s * L::kQS, hc * (NC / 64), it > 0);
-        if (!mbar_wait(b_ds, it & 1, abort_flag, p.err)) { ok = false; break; }
+        mma_tmemA_x_rows64<NC, F16>(leader, tmem + kColDV, tmem + kColS, desc_off(dmn_do, s * L::kQS + col_off),
+                                    it > 0);
+        if (!FA_WAIT(b_ds, it & 1)) { ok = false; break; }
         tc_fence_after();
         // dK += dS^T Q : A = dS^T (128 keys x 64 queries, K-major), B = Q columns (MN-major)
         {
           constexpr uint32_t idesc = idesc_f32acc(128, NC, false, true, F16);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kColDK, sdesc_sw128(sm_ds + kk * 32, 16, 1024),
-                   sdesc_sw128(sm_q + s * L::kQS + hc * (NC / 64) * kBox64 + kk * 2048, kBox64, 1024), idesc,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + kColDK, desc_off(dk_ds, kk * 32), desc_off(dmn_q, s * L::kQS + col_off + kk * 2048),
+                     idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
         }
-        mma_commit(b_dsfree);
-        mma_commit(&b_empty[s]);
+        if (leader) {
+          mma_commit(b_dsfree);
+          mma_commit(&b_empty[s]);
+        }
         if (it + 1 < nq) {
           const int s1 = (it + 1) % S;
-          if (!mbar_wait(&b_full[s1], ((it + 1) / S) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!FA_WAIT(&b_full[s1], ((it + 1) / S) & 1)) { ok = false; break; }
           tc_fence_after();
-          mma_rows128_x_rows64<D, F16>(tmem + kColS, sm_k, sm_q + s1 * L::kQS);
-          mma_commit(b_s);
-          mma_rows128_x_rows64<D, F16>(tmem + kColDP, sm_v, sm_do + s1 * L::kQS);
-          mma_commit(b_dp);
+          mma_rows128_x_rows64<D, F16>(leader, tmem + kColS, dk_k, desc_off(dk_q, s1 * L::kQS));
+          if (leader) mma_commit(b_s);
+          mma_rows128_x_rows64<D, F16>(leader, tmem + kColDP, dk_v, desc_off(dk_do, s1 * L::kQS));
+          if (leader) mma_commit(b_dp);
         }
       }
+#undef FA_WAIT
       if (ok) {
-        mma_commit(b_dkdv);
+        if (leader) mma_commit(b_dkdv);
       } else {
-        mma_commit(b_drain);
+        if (leader) mma_commit(b_drain);
         mbar_wait_drain(b_drain, 0);
       }
     }
@@ -552,28 +574,34 @@ __global__ void __launch_bounds__(kWThreads, 1)
     return;
   }
   if (warp == kWMma) {
-    if (lane == 0) {
-      bool ok = mbar_wait(b_qdo, 0, abort_flag, p.err);
+    {
+      const bool leader = elect_one();
+      const uint64_t dk_q = sdesc_sw128(sm_q, 16, 1024), dk_do = sdesc_sw128(sm_do, 16, 1024);
+      const uint64_t dk_k = sdesc_sw128(sm_k, 16, 1024), dk_v = sdesc_sw128(sm_v, 16, 1024);
+      const uint64_t dmn_k = sdesc_sw128(sm_k, kBox64, 1024);
+      // every lane waits; the vote keeps the warp's decision uniform
+#define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
+      bool ok = FA_WAIT(b_qdo, 0);
       for (int t = 0; ok && t < nt; ++t) {
         const int s = t % S;
-        if (!mbar_wait(&b_kfull[s], (t / S) & 1, abort_flag, p.err) ||
-            !mbar_wait(&b_vfull[s], (t / S) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&b_kfull[s], (t / S) & 1) || !FA_WAIT(&b_vfull[s], (t / S) & 1)) { ok = false; break; }
         tc_fence_after();
         // S = Q K^T and dP = dO V^T (the previous tile's dS was read by its dQ product, issued before)
-        mma_rows128_x_rows64<D, F16>(tmem + kColS, sm_q, sm_k + s * L::kKS);
-        mma_commit(b_s);
-        mma_rows128_x_rows64<D, F16>(tmem + kColDP, sm_do, sm_v + s * L::kKS);
-        mma_commit(b_dp);
-        if (!mbar_wait(b_ds, t & 1, abort_flag, p.err)) { ok = false; break; }
+        mma_rows128_x_rows64<D, F16>(leader, tmem + kColS, dk_q, desc_off(dk_k, s * L::kKS));
+        if (leader) mma_commit(b_s);
+        mma_rows128_x_rows64<D, F16>(leader, tmem + kColDP, dk_do, desc_off(dk_v, s * L::kKS));
+        if (leader) mma_commit(b_dp);
+        if (!FA_WAIT(b_ds, t & 1)) { ok = false; break; }
         tc_fence_after();
         // dQ += dS K : A = dS in TMEM, B = K tile (MN-major, D columns)
-        mma_tmemA_x_rows64<D, F16>(tmem + kColDQ, tmem + kColS, sm_k + s * L::kKS, 0, t > 0);
-        mma_commit(&b_empty[s]);
+        mma_tmemA_x_rows64<D, F16>(leader, tmem + kColDQ, tmem + kColS, desc_off(dmn_k, s * L::kKS), t > 0);
+        if (leader) mma_commit(&b_empty[s]);
       }
+#undef FA_WAIT
       if (ok) {
-        mma_commit(b_dq);
+        if (leader) mma_commit(b_dq);
       } else {
-        mma_commit(b_drain);
+        if (leader) mma_commit(b_drain);
         mbar_wait_drain(b_drain, 0);
       }
     }

@@ -94,29 +94,35 @@ struct WideParams {
   int group, BH;
 };
 
-// S = Q K^T : M = 128 query rows, N = 64 keys, K = D (both K-major).
+// S = Q K^T : M = 128 query rows, N = 64 keys, K = D (both K-major).  a0 /
+// b0 are the descriptors of the Q tile and the K stage; each K-step adds its
+// box / swizzle-atom offset (bytes / 16) to the start-address field.  The
+// whole MMA warp calls this; ``leader`` (one elected lane) issues.
 template <int D, bool F16>
-__device__ __forceinline__ void wide_qk(uint32_t tmem_s, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void wide_qk(bool leader, uint32_t tmem_s, uint64_t a0, uint64_t b0) {
   using L = WideSmem<D>;
   constexpr uint32_t idesc = idesc_f32acc(128, kWBN, false, false, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t qa = q_smem + (kk / 4) * L::kQBox + (kk % 4) * 32;
-    const uint32_t ka = k_smem + (kk / 4) * L::kKVBox + (kk % 4) * 32;
-    mma_ss(tmem_s, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), idesc, kk > 0);
+    for (int kk = 0; kk < D / 16; ++kk)
+      mma_ss(tmem_s, a0 + static_cast<uint32_t>(((kk / 4) * L::kQBox + (kk % 4) * 32) >> 4),
+             b0 + static_cast<uint32_t>(((kk / 4) * L::kKVBox + (kk % 4) * 32) >> 4), idesc, kk > 0);
   }
 }
 
 // O (+)= P V : M = 128, N = D, K = 64 keys; P (16-bit pairs) in TMEM over S,
-// V MN-major in shared memory (64-column boxes 8 KB apart).
+// V MN-major in shared memory (64-column boxes 8 KB apart), b0 the descriptor
+// of its stage.
 template <int D, bool F16>
-__device__ __forceinline__ void wide_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
-  using L = WideSmem<D>;
+__device__ __forceinline__ void wide_pv(bool leader, uint32_t tmem_o, uint32_t tmem_p, uint64_t b0,
+                                        bool accumulate) {
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
+  if (leader) {
 #pragma unroll
-  for (int kk = 0; kk < kWBN / 16; ++kk)
-    mma_ts(tmem_o, tmem_p + kk * 8, sdesc_sw128(v_smem + kk * 2048, L::kKVBox, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < kWBN / 16; ++kk)
+      mma_ts(tmem_o, tmem_p + kk * 8, b0 + static_cast<uint32_t>((kk * 2048) >> 4), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 __device__ __forceinline__ void wide_teardown(uint32_t tmem, bool dealloc) {
@@ -233,38 +239,53 @@ __global__ void __launch_bounds__(kWThreads, 1)
   }
   if (warp == kWMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nt > 0) {
-      bool ok = mbar_wait(bar.q, 0, abort_flag, p.err);
+    // The whole warp runs the loop, so descriptors and counters are
+    // warp-uniform values; one elected lane issues the MMAs and commits.
+    if (nt > 0) {
+      const bool leader = elect_one();
+      const uint64_t dq0 = sdesc_sw128(sm_q, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sm_k, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sm_v, L::kKVBox, 1024);
+      // every lane waits; the vote keeps the warp's decision uniform
+#define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
+      bool ok = FA_WAIT(bar.q, 0);
       // S_0 and S_1 ahead of the loop
       for (int t = 0; ok && t < min(2, nt); ++t) {
-        if (!mbar_wait(&bar.kfull[t % S], (t / S) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&bar.kfull[t % S], (t / S) & 1)) { ok = false; break; }
         tc_fence_after();
-        wide_qk<D, F16>(tmem + 64 * t, sm_q, sm_k + (t % S) * L::kKVTile);
-        mma_commit(&bar.s_full[t]);
-        mma_commit(&bar.kempty[t % S]);
+        wide_qk<D, F16>(leader, tmem + 64 * t, dq0, dk0 + static_cast<uint32_t>(((t % S) * L::kKVTile) >> 4));
+        if (leader) {
+          mma_commit(&bar.s_full[t]);
+          mma_commit(&bar.kempty[t % S]);
+        }
       }
       for (int t = 0; ok && t < nt; ++t) {
         const int b = t & 1, s = t % S;
-        if (!mbar_wait(&bar.p_ready[b], (t >> 1) & 1, abort_flag, p.err) ||
-            !mbar_wait(&bar.vfull[s], (t / S) & 1, abort_flag, p.err)) { ok = false; break; }
+        if (!FA_WAIT(&bar.p_ready[b], (t >> 1) & 1) || !FA_WAIT(&bar.vfull[s], (t / S) & 1)) { ok = false; break; }
         tc_fence_after();
-        wide_pv<D, F16>(tmem + kColO, tmem + 64 * b, sm_v + s * L::kKVTile, t > 0);
-        mma_commit(bar.pv_done);
-        mma_commit(&bar.vempty[s]);
+        wide_pv<D, F16>(leader, tmem + kColO, tmem + 64 * b, dv0 + static_cast<uint32_t>((s * L::kKVTile) >> 4),
+                        t > 0);
+        if (leader) {
+          mma_commit(bar.pv_done);
+          mma_commit(&bar.vempty[s]);
+        }
         if (t + 2 < nt) {
           // S_{t+2} into the buffer P_t occupies: issued after the P V product reading it
           const int s2 = (t + 2) % S;
-          if (!mbar_wait(&bar.kfull[s2], ((t + 2) / S) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!FA_WAIT(&bar.kfull[s2], ((t + 2) / S) & 1)) { ok = false; break; }
           tc_fence_after();
-          wide_qk<D, F16>(tmem + 64 * b, sm_q, sm_k + s2 * L::kKVTile);
-          mma_commit(&bar.s_full[b]);
-          mma_commit(&bar.kempty[s2]);
+          wide_qk<D, F16>(leader, tmem + 64 * b, dq0, dk0 + static_cast<uint32_t>((s2 * L::kKVTile) >> 4));
+          if (leader) {
+            mma_commit(&bar.s_full[b]);
+            mma_commit(&bar.kempty[s2]);
+          }
         }
       }
+#undef FA_WAIT
       if (ok) {
-        mma_commit(bar.o_ready);
+        if (leader) mma_commit(bar.o_ready);
       } else {
-        mma_commit(bar.drain);  // MMAs already issued finish before TMEM is freed
+        if (leader) mma_commit(bar.drain);  // MMAs already issued finish before TMEM is freed
         mbar_wait_drain(bar.drain, 0);
       }
     }
