@@ -31,8 +31,8 @@
 //     dimension, column = query row);
 //   * warp 4 streams the tiles (1 to 8 pages each, located through the block
 //     table) with TMA through a 3-stage (d = 128) / 4-stage (d = 64) mbarrier
-//     ring and issues the MMAs; warps 0-3 do the softmax, the rescale and the
-//     epilogue.
+//     ring and issues the MMAs (the whole warp runs the loop, one elected lane
+//     issues); warps 0-3 do the softmax, the rescale and the epilogue.
 // For d = 64 the V tile carries a second, all-zero 64-column box so the P V
 // product keeps M = 128 (dimensions 64..127 come out as zeros).
 // grid = (split, key/value head x block of up to 16 query rows, sequence): all
@@ -238,9 +238,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA + MMA
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+    // The whole warp runs the loop, so descriptors and counters are
+    // warp-uniform values; one elected lane issues the copies, the MMAs and
+    // the commits.
+    if (n > 0) {
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
       // a tile's page ids are read from the block table one refill ahead of
       // its copies, so the copies never wait for those reads
       constexpr int kMaxPagesPerTile = kTileKeys / 16;
@@ -256,6 +262,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         for (int pg = 0; pg < kMaxPagesPerTile; ++pg) ids[pg] = (pg < pages_here) ? bt[pg] : 0;
       };
       auto issue = [&](int it, const int (&pids)[kMaxPagesPerTile]) {
+        if (!leader) return;
         const int st = it % S;
         const int pages_here = pages_of(it);
         // K and V complete separately: S^T needs only K, so it starts while V is still arriving
@@ -273,7 +280,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
           }
         }
       };
-      const uint32_t q_addr = smem_u32(qsm);
+      // descriptor bases; a stage, box, buffer or K-step offset (bytes / 16)
+      // is added to the start-address field
+      const uint64_t dk0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t dq0 = sdesc_sw128(smem_u32(qsm), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(smem) + L::kKBytes, L::kBox, 1024);
+      const uint64_t dp0 = sdesc_sw128(smem_u32(smem + L::kP), 16, 1024);
       constexpr uint32_t idesc_s = idesc_f32acc(128, kMaxRows, false, false, F16);
       constexpr uint32_t idesc_o = idesc_f32acc(128, kMaxRows, true, false, F16);
       int issued = 0;
@@ -283,23 +295,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         issue(issued, pids_next);
       }
       if (issued < n) read_pids(issued, pids_next);
+      // every lane waits; the vote keeps the warp's decision uniform
+#define FA_WAIT(bar_, parity) __all_sync(0xffffffffu, mbar_wait((bar_), (parity), abort_flag, p.err))
       bool ok = true;
       int consumed = 0;  // tiles whose copies have landed
       // S^T = K Q^T of tile it into its TMEM buffer: M = 128 keys, N = 16 rows, K = D (both K-major)
       auto issue_s = [&](int it) -> bool {
         const int st = it % S;
-        if (!mbar_wait(&kfull[st], (it / S) & 1, abort_flag, p.err)) return false;
+        if (!FA_WAIT(&kfull[st], (it / S) & 1)) return false;
         consumed = it + 1;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + st * L::kStage);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk / 4) * L::kBox + (kk % 4) * 32;
-          const uint32_t off_q = (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
-          mma_ss(tmem + (it & 1) * 16, sdesc_sw128(k_addr + off_k, 16, 1024), sdesc_sw128(q_addr + off_q, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off_k = st * L::kStage + (kk / 4) * L::kBox + (kk % 4) * 32;
+            const uint32_t off_q = (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
+            mma_ss(tmem + (it & 1) * 16, dk0 + (off_k >> 4), dq0 + (off_q >> 4), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_ready[it & 1]);
         }
-        mma_commit(&s_ready[it & 1]);
         return true;
       };
       ok = issue_s(0);
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         // refill the stage of tile it - 1 once its P V product has read it
         // (before waiting for the next tile's K, so the copies go out early)
         if (issued < n) {
-          if (it >= 1 && !mbar_wait(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag, p.err)) {
+          if (it >= 1 && !FA_WAIT(&pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1)) {
             ok = false;
             break;
           }
@@ -318,29 +332,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) fa_decode_kernel(const __grid_
         // the next tile's S^T runs while the softmax warps work on this one; its
         // buffer was last read by the softmax of tile it - 1 (p_ready seen below)
         if (it + 1 < n && !issue_s(it + 1)) { ok = false; break; }
-        if (!mbar_wait(&p_ready[it & 1], (it >> 1) & 1, abort_flag, p.err) ||
-            !mbar_wait(&vfull[it % S], (it / S) & 1, abort_flag, p.err)) {
+        if (!FA_WAIT(&p_ready[it & 1], (it >> 1) & 1) || !FA_WAIT(&vfull[it % S], (it / S) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
         // O^T += V^T P^T: M = 128 dimensions (V read MN-major), N = 16 rows, K = 128 keys
-        const uint32_t v_addr = smem_u32(smem + (it % S) * L::kStage) + L::kKBytes;
-        const uint32_t p_addr = smem_u32(smem + L::kP + (it & 1) * L::kPBytes);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-          const uint32_t off_p = (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
-          mma_ss(tm_o, sdesc_sw128(v_addr + kk * 2048, L::kBox, 1024), sdesc_sw128(p_addr + off_p, 16, 1024),
-                 idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+            const uint32_t off_v = (it % S) * L::kStage + kk * 2048;
+            const uint32_t off_p = (it & 1) * L::kPBytes + (kk / 4) * (kMaxRows * 128) + (kk % 4) * 32;
+            mma_ss(tm_o, dv0 + (off_v >> 4), dp0 + (off_p >> 4), idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&pv_done[it & 1]);
         }
-        mma_commit(&pv_done[it & 1]);
       }
+#undef FA_WAIT
       if (!ok) {
         // copies and products in flight finish before shared and tensor memory go away
-        mma_commit(drain);
+        if (leader) mma_commit(drain);
         mbar_wait_drain(drain, 0);
-        for (int it2 = consumed; it2 < issued; ++it2) mbar_wait_drain(&kfull[it2 % S], (it2 / S) & 1);
-        for (int it2 = max(0, consumed - 1); it2 < issued; ++it2) mbar_wait_drain(&vfull[it2 % S], (it2 / S) & 1);
+        if (leader) {
+          for (int it2 = consumed; it2 < issued; ++it2) mbar_wait_drain(&kfull[it2 % S], (it2 / S) & 1);
+          for (int it2 = max(0, consumed - 1); it2 < issued; ++it2)
+            mbar_wait_drain(&vfull[it2 % S], (it2 / S) & 1);
+        }
       }
     }
     __syncwarp();
