@@ -19,9 +19,12 @@
 //    of fa_fwd.cu; since S_{t+1} was issued before O += P_{t-1} V_{t-1}, a
 //    rescale of O first waits for that product (a barrier committed after
 //    every P V product);
-//  * draws the dropout keep bits in the softmax thread before waiting for S
-//    (8 Philox calls per 64-key tile, in lockstep).
-// Warps: 0-3 softmax, 4 MMA issue, 5 TMA loads.
+//  * with dropout, a fourth group of warps draws the keep bits (one thread
+//    per query row, 8 Philox calls per 64-key tile in lockstep) up to two
+//    tiles ahead into a two-buffer shared-memory ring that the softmax warps
+//    read; with one softmax warp per sub-partition the draw then overlaps
+//    the softmax instead of preceding it.
+// Warps: 0-3 softmax, 4 MMA issue, 5 TMA loads, 6-9 keep words (dropout only).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,8 +41,10 @@ namespace {
 constexpr int kWBM = 128;        // query rows per CTA
 constexpr int kWBN = 64;         // keys per tile
 constexpr int kWThreads = 192;   // 4 softmax warps, MMA warp, TMA warp
+constexpr int kWThreadsDrop = 320;  // + 4 keep-word warps (dropout)
 constexpr int kWMmaWarp = 4;
 constexpr int kWLoadWarp = 5;
+constexpr int kWKeepWarp0 = 6;
 constexpr float kWRescaleTau = 8.0f;  // lazy-rescale threshold, log2 units
 
 template <int D>
@@ -51,16 +56,20 @@ struct WideSmem {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + (D / 64) * kQBox;
   static constexpr int kV = kK + kStages * kKVTile;
-  static constexpr int kBar = kV + kStages * kKVTile;
-  // barriers: q, kfull[S], kempty[S], vfull[S], vempty[S], s_full[2], p_ready[2], pv_done, o_ready, drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  // dropout keep words drawn by the keep-word warps: [buffer][word 0..1][row]
+  static constexpr int kKeep = kV + kStages * kKVTile;
+  static constexpr int kBar = kKeep + 2 * 2 * 128 * 4;
+  // barriers: q, kfull[S], kempty[S], vfull[S], vempty[S], s_full[2], p_ready[2], pv_done, o_ready, drain,
+  // keep_full[2], keep_empty[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 7 + 4;
   // tmem slot, abort flag, the unit's first query row and head coordinate
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
 
 struct WideBars {
-  uint64_t *q, *kfull, *kempty, *vfull, *vempty, *s_full, *p_ready, *pv_done, *o_ready, *drain;
+  uint64_t *q, *kfull, *kempty, *vfull, *vempty, *s_full, *p_ready, *pv_done, *o_ready, *drain, *keep_full,
+      *keep_empty;
 };
 
 template <int D>
@@ -79,6 +88,8 @@ __device__ __forceinline__ WideBars wide_bars(uint8_t* smem) {
   r.pv_done = r.s_full + 4;
   r.o_ready = r.s_full + 5;
   r.drain = r.s_full + 6;
+  r.keep_full = r.s_full + 7;
+  r.keep_empty = r.s_full + 9;
   return r;
 }
 
@@ -125,15 +136,16 @@ __device__ __forceinline__ void wide_pv(bool leader, uint32_t tmem_o, uint32_t t
   }
 }
 
+template <bool DROPOUT>
 __device__ __forceinline__ void wide_teardown(uint32_t tmem, bool dealloc) {
   tc_fence_before();
-  asm volatile("bar.sync 1, %0;" ::"n"(kWThreads) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"n"(DROPOUT ? kWThreadsDrop : kWThreads) : "memory");
   tc_fence_after();
   if (dealloc) tmem_dealloc(tmem, 512);
 }
 
 template <int D, bool CAUSAL, bool DROPOUT, bool F16>
-__global__ void __launch_bounds__(kWThreads, 1)
+__global__ void __launch_bounds__(DROPOUT ? kWThreadsDrop : kWThreads, 1)
     fa_fwd_wide_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ WideParams p) {
   using L = WideSmem<D>;
@@ -182,6 +194,10 @@ __global__ void __launch_bounds__(kWThreads, 1)
     mbar_init(bar.pv_done, 1);
     mbar_init(bar.o_ready, 1);
     mbar_init(bar.drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar.keep_full[b], 4);
+      mbar_init(&bar.keep_empty[b], 4);
+    }
     *abort_flag = 0;
     reinterpret_cast<int*>(smem + L::kMisc)[2] = su.q0;
     reinterpret_cast<int*>(smem + L::kMisc)[3] = su.g;
@@ -234,7 +250,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
       }
     }
     __syncwarp();
-    wide_teardown(tmem, false);
+    wide_teardown<DROPOUT>(tmem, false);
     return;
   }
   if (warp == kWMmaWarp) {
@@ -290,7 +306,36 @@ __global__ void __launch_bounds__(kWThreads, 1)
       }
     }
     __syncwarp();
-    wide_teardown(tmem, true);
+    wide_teardown<DROPOUT>(tmem, true);
+    return;
+  }
+
+  if (DROPOUT && warp >= kWKeepWarp0) {
+    // ---------------------------------------------------------- keep words
+    // One thread per query row draws its 8 Philox calls per 64-key tile (in
+    // lockstep) up to two tiles ahead of the softmax, into a two-buffer ring.
+    const int kr = (warp - kWKeepWarp0) * 32 + lane;
+    const PhiloxFixed123 kphx = philox_fix123(static_cast<uint32_t>(qt * kWBM + kr), static_cast<uint32_t>(su.h),
+                                              static_cast<uint32_t>(su.b), p.philox_rk);
+    const uint32_t kc2 = make_drop_const(p.drop_t).c2;
+    const bool khi = p.drop_t > 0x8000u;
+    uint32_t* ring = reinterpret_cast<uint32_t*>(smem + L::kKeep);
+    for (int t = 0; t < nt; ++t) {
+      const int b = t & 1;
+      // the softmax warps have read the buffer's previous tile (t - 2)
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.keep_empty[b], ((t - 2) >> 1) & 1, abort_flag, p.err)))
+        break;
+      uint32_t W[2];
+      if (khi)
+        draw_keep_words<true, kWBN / 8>(static_cast<uint32_t>(t * (kWBN / 8)), kphx, p.philox_rk, kc2, W);
+      else
+        draw_keep_words<false, kWBN / 8>(static_cast<uint32_t>(t * (kWBN / 8)), kphx, p.philox_rk, kc2, W);
+      ring[(b * 2 + 0) * 128 + kr] = W[0];
+      ring[(b * 2 + 1) * 128 + kr] = W[1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.keep_full[b]);
+    }
+    wide_teardown<DROPOUT>(tmem, false);
     return;
   }
 
@@ -300,10 +345,6 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const uint32_t t_o = t_lane + kColO;
   const float sl2 = p.scale_log2;
-  const PhiloxFixed123 phx = philox_fix123(static_cast<uint32_t>(i), static_cast<uint32_t>(su.h),
-                                           static_cast<uint32_t>(su.b), p.philox_rk);
-  const uint32_t drop_c2 = make_drop_const(p.drop_t).c2;
-  const bool hi_t = p.drop_t > 0x8000u;
   // masking: key j = t * kWBN + c is visible iff j <= lim0; tiles from t_mask
   // on can hold a masked key for some row of the tile
   const int lim0 = CAUSAL ? min(su.nk - 1, i + delta) : su.nk - 1;
@@ -317,11 +358,13 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const int b = t & 1;
     uint32_t W[2] = {0u, 0u};
     if (DROPOUT) {
-      if (hi_t)
-        draw_keep_words<true, kWBN / 8>(static_cast<uint32_t>(t * (kWBN / 8)), phx, p.philox_rk, drop_c2, W);
-      else
-        draw_keep_words<false, kWBN / 8>(static_cast<uint32_t>(t * (kWBN / 8)), phx, p.philox_rk, drop_c2, W);
-      asm volatile("" : "+r"(W[0]), "+r"(W[1]));  // not sunk past the wait
+      // this row's keep words from the keep-word warps' ring
+      if (!mbar_wait(&bar.keep_full[b], (t >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+      const uint32_t* ring = reinterpret_cast<const uint32_t*>(smem + L::kKeep);
+      W[0] = ring[(b * 2 + 0) * 128 + r];
+      W[1] = ring[(b * 2 + 1) * 128 + r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.keep_empty[b]);
     }
     if (!mbar_wait(&bar.s_full[b], (t >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
     tc_fence_after();
@@ -442,7 +485,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     }
     if (row_ok) *lse_g = (l > 0.f) ? (m + lg2_approx(l)) * 0.69314718055994531f : -CUDART_INF_F;
   }
-  wide_teardown(tmem, false);
+  wide_teardown<DROPOUT>(tmem, false);
 }
 
 template <int D, bool CAUSAL, bool DROPOUT, bool F16>
@@ -467,7 +510,7 @@ cudaError_t launch_wide_t(const FwdArgs& a, cudaStream_t stream) {
   if (p.group < 1) p.group = 1;
   if (p.group > p.BH) p.group = p.BH;
   dim3 grid(static_cast<unsigned>(p.BH) * n_qt);
-  kern<<<grid, kWThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
+  kern<<<grid, DROPOUT ? kWThreadsDrop : kWThreads, smem, stream>>>(a.tmQ, a.tmK, a.tmV, p);
   return cudaGetLastError();
 }
 
