@@ -233,10 +233,11 @@ __device__ __forceinline__ void mma_tile_kk(bool leader, uint32_t tmem_d, uint32
   b_smem = opaque_u32(b_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, 128, false, false, F16);
   if (leader) {
+    const uint64_t da = sdesc_sw128(a_smem, 16, 1024), db = sdesc_sw128(b_smem, 16, 1024);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
-      mma_ss(tmem_d, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc, kk > 0);
+      const uint32_t off = ((kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32) >> 4;
+      mma_ss(tmem_d, da + off, db + off, idesc, kk > 0);
     }
   }
 }
@@ -250,10 +251,11 @@ __device__ __forceinline__ void mma_dv(bool leader, uint32_t tmem_d, uint32_t tm
   do_smem = opaque_u32(do_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
   if (leader) {
+    const uint64_t db = sdesc_sw128(do_smem, BwdSmem<D>::kBox, 1024);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_ts(tmem_d, tmem_p + (kk / 4) * 64 + (kk % 4) * 8,
-             sdesc_sw128(do_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+      mma_ts(tmem_d, tmem_p + (kk / 4) * 64 + (kk % 4) * 8, db + static_cast<uint32_t>((kk * 2048) >> 4), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -265,11 +267,11 @@ __device__ __forceinline__ void mma_dk(bool leader, uint32_t tmem_d, uint32_t ds
   q_smem = opaque_u32(q_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, false, true, F16);
   if (leader) {
+    const uint64_t da = sdesc_sw128(ds_smem, 16, 1024), db = sdesc_sw128(q_smem, BwdSmem<D>::kBox, 1024);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t a_off = (kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32;
-      mma_ss(tmem_d, sdesc_sw128(ds_smem + a_off, 16, 1024),
-             sdesc_sw128(q_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+      const uint32_t a_off = ((kk / 4) * BwdSmem<D>::kBox + (kk % 4) * 32) >> 4;
+      mma_ss(tmem_d, da + a_off, db + static_cast<uint32_t>((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
     }
   }
 }
@@ -281,10 +283,12 @@ __device__ __forceinline__ void mma_dq(bool leader, uint32_t tmem_d, uint32_t ds
   k_smem = opaque_u32(k_smem);
   constexpr uint32_t idesc = idesc_f32acc(128, D, true, true, F16);
   if (leader) {
+    const uint64_t da = sdesc_sw128(ds_smem, BwdSmem<D>::kBox, 1024), db = sdesc_sw128(k_smem, BwdSmem<D>::kBox, 1024);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_ss(tmem_d, sdesc_sw128(ds_smem + kk * 2048, BwdSmem<D>::kBox, 1024),
-             sdesc_sw128(k_smem + kk * 2048, BwdSmem<D>::kBox, 1024), idesc, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk * 2048) >> 4;
+      mma_ss(tmem_d, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
+    }
   }
 }
 
