@@ -355,9 +355,10 @@ bool dtype_ok(fa_dtype dtype) { return dtype == FA_DTYPE_BF16 || dtype == FA_DTY
 
 // Device layout of fa_fwd_bwd_host's workspace: kHostSlots staging slots of
 // the per-group tensors (Q, K, V, dO in; O, dQ, dK, dV out: [units, N, d]
-// 16-bit each; LSE [units, N] fp32), then the backward workspace of one group
-// (the groups run one after another on the compute stream and share it).
-constexpr int kHostSlots = 3;
+// 16-bit each; LSE [units, N] fp32), then two backward workspaces of one
+// group (even groups compute on the caller's compute stream, odd groups on a
+// second one; the groups of one stream run in order and share its workspace).
+constexpr int kHostSlots = 4;
 
 struct HostPlan {
   int units_total;   // B * H
@@ -558,7 +559,7 @@ fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void*
 size_t fa_fwd_bwd_host_workspace_size(int B, int H, int N, int d, int groups) {
   HostPlan hp;
   if (!host_plan(B, H, N, d, groups, &hp)) return 0;
-  return kHostSlots * hp.slot + hp.bwd;
+  return kHostSlots * hp.slot + 2 * hp.bwd;
 }
 
 fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const void* dO, void* O, float* LSE,
@@ -572,13 +573,23 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
   HostPlan hp;
   if (!host_plan(B, H, N, d, groups, &hp)) return FA_ERR_INVALID_ARG;
   if (!Q || !K || !V || !dO || !O || !LSE || !dQ || !dK || !dV || !streams) return FA_ERR_INVALID_ARG;
-  if (!workspace || misaligned(workspace, 256) || workspace_bytes_ < kHostSlots * hp.slot + hp.bwd)
+  if (!workspace || misaligned(workspace, 256) || workspace_bytes_ < kHostSlots * hp.slot + 2 * hp.bwd)
     return FA_ERR_INVALID_ARG;
   cudaStream_t s_in = static_cast<cudaStream_t>(streams[0]);
-  cudaStream_t s_cmp = static_cast<cudaStream_t>(streams[1]);
+  cudaStream_t s_cmp0 = static_cast<cudaStream_t>(streams[1]);
   cudaStream_t s_out = static_cast<cudaStream_t>(streams[2]);
+  // odd groups compute on a second stream of the call's own, so that one
+  // group's kernels start while the last wave of the previous group's runs
+  // (only when the caller asked for overlap with three distinct streams)
+  cudaStream_t s_cmp1 = s_cmp0;
+  bool own_stream = false;
+  if (s_cmp0 != s_in && s_cmp0 != s_out && hp.groups > 1) {
+    if (cudaStreamCreateWithFlags(&s_cmp1, cudaStreamNonBlocking) != cudaSuccess) return FA_ERR_CUDA;
+    own_stream = true;
+  }
   char* ws = static_cast<char*>(workspace);
-  char* bwd_ws = ws + kHostSlots * hp.slot;
+  char* bwd_ws0 = ws + kHostSlots * hp.slot;  // one backward workspace per compute stream
+  char* bwd_ws1 = bwd_ws0 + hp.bwd;
   const size_t row = static_cast<size_t>(N) * d * 2;  // bytes of one unit of a 16-bit tensor
   // events: copy-in done, compute done, copy-out done, per group
   const int ng = hp.groups;
@@ -591,7 +602,8 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
   // call's last copies still reading the staging slots this call refills)
   if (st == FA_OK && (cudaEventRecord(ev[3 * ng], s_out) != cudaSuccess ||
                       cudaStreamWaitEvent(s_in, ev[3 * ng], 0) != cudaSuccess ||
-                      cudaStreamWaitEvent(s_cmp, ev[3 * ng], 0) != cudaSuccess))
+                      cudaStreamWaitEvent(s_cmp0, ev[3 * ng], 0) != cudaSuccess ||
+                      cudaStreamWaitEvent(s_cmp1, ev[3 * ng], 0) != cudaSuccess))
     st = FA_ERR_CUDA;
   const char* src_in[4] = {static_cast<const char*>(Q), static_cast<const char*>(K), static_cast<const char*>(V),
                            static_cast<const char*>(dO)};
@@ -605,6 +617,8 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
                     slot + 7 * hp.tensor};  // O, dQ, dK, dV
     float* lse = reinterpret_cast<float*>(slot + 8 * hp.tensor);
     cudaEvent_t ev_in = ev[3 * g], ev_cmp = ev[3 * g + 1], ev_out = ev[3 * g + 2];
+    cudaStream_t s_cmp = (g & 1) ? s_cmp1 : s_cmp0;
+    char* bwd_ws = (g & 1) ? bwd_ws1 : bwd_ws0;
     // copy-in: the slot's inputs are free once the group that used it last has computed
     if (g >= kHostSlots && cudaStreamWaitEvent(s_in, ev[3 * (g - kHostSlots) + 1], 0) != cudaSuccess) {
       st = FA_ERR_CUDA;
@@ -650,8 +664,9 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
       st = FA_ERR_CUDA;
     if (st == FA_OK && cudaEventRecord(ev_out, s_out) != cudaSuccess) st = FA_ERR_CUDA;
   }
-  // events may be destroyed while work that records them is still queued
+  // events and the stream may be destroyed while work on them is still queued
   for (int k = 0; k < made; ++k) cudaEventDestroy(ev[k]);
+  if (own_stream) cudaStreamDestroy(s_cmp1);
   delete[] ev;
   return st;
 }

@@ -281,17 +281,20 @@ fa_status fa_bwd_finish(void* dQ, int B, int H, int N, int d, float scale, const
  *                 consecutive units (at most B*H; a smaller last group);
  *                 group g is copied in on streams[0], computed (fa_fwd and
  *                 the three backward stages, the same kernels and results as
- *                 fa_fwd / fa_bwd) on streams[1] and copied out on
- *                 streams[2], so group g+1's copy-in and group g-1's copy-out
- *                 overlap group g's kernels.  Dropout counters keep the whole
- *                 problem's (b, h).
+ *                 fa_fwd / fa_bwd) on streams[1] (odd groups: on a second
+ *                 compute stream the call creates and releases itself, so
+ *                 one group's kernels start while the previous group's last
+ *                 wave runs) and copied out on streams[2], so group g+1's
+ *                 copy-in and group g-1's copy-out overlap group g's kernels.
+ *                 Dropout counters keep the whole problem's (b, h).
  *   workspace   : device, 256-byte aligned, at least
  *                 fa_fwd_bwd_host_workspace_size(B, H, N, d, groups) bytes:
- *                 three staging slots of one group's tensors plus one
- *                 group's backward workspace.  Caller-owned.
+ *                 four staging slots of one group's tensors plus two of one
+ *                 group's backward workspaces.  Caller-owned.
  *   streams     : three CUDA streams (cudaStream_t), copy-in, compute,
  *                 copy-out; the same stream may be given more than once (the
- *                 step then runs without overlap).
+ *                 step then runs without overlap, and without the second
+ *                 compute stream).
  * Everything is enqueued asynchronously and starts after the work already
  * enqueued on streams[2] (so calls in a row on the same streams reuse the
  * staging slots safely); the outputs are complete when streams[2] has
