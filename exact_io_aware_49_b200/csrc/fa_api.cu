@@ -322,8 +322,9 @@ fa_status wide_tiles_run(const Problem& pb, const void* Q, const void* K, const 
   fa::BwdArgs a;
   bwd_args(pb, &a, workspace);
   CUtensorMap kv[4], qm[4];  // Q, K, V, dO
-  if (!encode_q_like(pb, &kv[0], Q, 64) || !encode_k_like(pb, &kv[1], K, 128) || !encode_k_like(pb, &kv[2], V, 128) ||
-      !encode_q_like(pb, &kv[3], dO, 64) || !encode_q_like(pb, &qm[0], Q, 128) || !encode_k_like(pb, &qm[1], K, 64) ||
+  const int kv_rows = fa::wide_kv_query_rows(pb.d);
+  if (!encode_q_like(pb, &kv[0], Q, kv_rows) || !encode_k_like(pb, &kv[1], K, 128) ||
+      !encode_k_like(pb, &kv[2], V, 128) || !encode_q_like(pb, &kv[3], dO, kv_rows) || !encode_q_like(pb, &qm[0], Q, 128) || !encode_k_like(pb, &qm[1], K, 64) ||
       !encode_k_like(pb, &qm[2], V, 64) || !encode_q_like(pb, &qm[3], dO, 128))
     return FA_ERR_CUDA;
   a.dQ = dQ;

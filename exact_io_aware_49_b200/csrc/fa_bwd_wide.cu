@@ -12,7 +12,9 @@
 // kernels that each keep one kind of output on chip:
 //  1. dK, dV: one CTA per (unit, 128-key tile[, half of the d columns at
 //     d = 256]) keeps K and V in shared memory and dK, dV in tensor memory
-//     while it streams 64-query tiles of Q and dO: S^T = K Q^T and
+//     while it streams query tiles of Q and dO through two stages (64
+//     queries at d = 192, 32 at d = 256, where the resident K and V leave
+//     room for only 64 KB of stages): S^T = K Q^T and
 //     dP^T = V dO^T over the full d, P^T (masked, dropout-marked) back into
 //     TMEM, dS^T into shared memory, dV += P^T dO and dK += dS^T Q for its
 //     output columns (the two halves at d = 256 recompute S^T and dP^T);
@@ -71,26 +73,28 @@ __device__ __forceinline__ void wide_bwd_teardown(uint32_t tmem, bool dealloc) {
 
 // D[tmem] (+)= A * B^T over K = D (both K-major): A has 128 rows in 128-row
 // boxes, B has 64 rows in 64-row boxes; N = 64.  a0 / b0: sdesc_sw128(x, 16, 1024).
-template <int D, bool F16>
+template <int D, bool F16, int NB = 64>
 __device__ __forceinline__ void mma_rows128_x_rows64(bool leader, uint32_t tmem_d, uint64_t a0, uint64_t b0) {
-  constexpr uint32_t idesc = idesc_f32acc(128, 64, false, false, F16);
+  // B has NB rows (64 or 32) in NB-row boxes; N = NB
+  constexpr uint32_t idesc = idesc_f32acc(128, NB, false, false, F16);
   if (leader) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk)
       mma_ss(tmem_d, a0 + static_cast<uint32_t>(((kk / 4) * kBox128 + (kk % 4) * 32) >> 4),
-             b0 + static_cast<uint32_t>(((kk / 4) * kBox64 + (kk % 4) * 32) >> 4), idesc, kk > 0);
+             b0 + static_cast<uint32_t>(((kk / 4) * (NB * 128) + (kk % 4) * 32) >> 4), idesc, kk > 0);
   }
 }
 
 // D[tmem] (+)= A[tmem, 16-bit pairs] * B over K = 64 rows of B, N = NC columns
 // of B (B MN-major in 64-row boxes 8 KB apart); b0: sdesc_sw128(first box, kBox64, 1024).
-template <int NC, bool F16>
+template <int NC, bool F16, int NB = 64>
 __device__ __forceinline__ void mma_tmemA_x_rows64(bool leader, uint32_t tmem_d, uint32_t tmem_a, uint64_t b0,
                                                    bool accumulate) {
+  // K = NB rows of B (64 or 32)
   constexpr uint32_t idesc = idesc_f32acc(128, NC, false, true, F16);
   if (leader) {
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
+    for (int kk = 0; kk < NB / 16; ++kk)
       mma_ts(tmem_d, tmem_a + kk * 8, b0 + static_cast<uint32_t>((kk * 2048) >> 4), idesc,
              (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -104,16 +108,19 @@ template <int D>
 struct KvSmem {
   static constexpr int kCols = (D == 256) ? 128 : D;     // output columns per CTA
   static constexpr int kSplit = D / kCols;                // CTAs per key tile
-  static constexpr int kStages = (D == 256) ? 1 : 2;
+  static constexpr int kQT = (D == 256) ? 32 : 64;        // queries per stage
+  static constexpr int kStages = 2;
+  static constexpr int kBoxQ = kQT * 128;                 // one 64-column box of a Q or dO stage
   static constexpr int kKV = (D / 64) * kBox128;          // K or V: 128 keys x D
-  static constexpr int kQS = (D / 64) * kBox64;           // one Q or dO stage: 64 queries x D
+  static constexpr int kQS = (D / 64) * kBoxQ;            // one Q or dO stage: kQT queries x D
   static constexpr int kK = 0;
   static constexpr int kV = kKV;
   static constexpr int kQ = 2 * kKV;
   static constexpr int kDO = kQ + kStages * kQS;
-  static constexpr int kDS = kDO + kStages * kQS;         // dS^T: 128 keys x 64 queries = one 128-row box
-  static constexpr int kVec = kDS + kBox128;              // stages x (LSE2[64], D[64]) fp32
-  static constexpr int kBar = kVec + kStages * 512;
+  static constexpr int kDS = kDO + kStages * kQS;         // dS^T: 128 keys x kQT queries in one 128-row box
+  static constexpr int kVec = kDS + kBox128;              // stages x (LSE2[kQT], D[kQT]) fp32
+  static constexpr int kVecStage = 2 * kQT * 4;
+  static constexpr int kBar = kVec + kStages * kVecStage;
   // barriers: kv, full[S], empty[S], s, dp, p, ds, ds_free, dkdv, drain
   static constexpr int kNumBars = 1 + 2 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
@@ -128,6 +135,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
   using L = KvSmem<D>;
   constexpr int S = L::kStages;
   constexpr int NC = L::kCols;
+  constexpr int QT = L::kQT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (!smem_layout_fits(smem_raw, smem, L::kMisc + 16, p.err)) return;
@@ -160,9 +168,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const SeqUnit su = resolve_unit(p.seq, unit);
   if (kj * 128 >= su.nk) return;
   const int Npad = (p.seq.Nq + 127) / 128 * 128;  // padded rows per unit in LSE2 / D
-  const int n_qt = (su.nq + 63) / 64;            // 64-query tiles
+  const int n_qt = (su.nq + QT - 1) / QT;        // QT-query tiles
   const int delta = su.nk - su.nq;
-  const int q_first = CAUSAL ? max(0, floor_div(kj * 128 - delta, 64)) : 0;
+  const int q_first = CAUSAL ? max(0, floor_div(kj * 128 - delta, QT)) : 0;
   const int nq = n_qt - q_first;
   const bool key_valid = kj * 128 + static_cast<int>(threadIdx.x & 127) < su.nk;
   if (nq <= 0) {
@@ -203,7 +211,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM: S^T [0, 64) (P^T over [0, 32)), dP^T [64, 128), dK [128, 128 + NC), dV after it
+  // TMEM: S^T [0, QT) (P^T over [0, QT / 2)), dP^T [64, 64 + QT), dK [128, 128 + NC), dV after it
   constexpr uint32_t kColS = 0, kColDP = 64, kColDK = 128, kColDV = 128 + NC;
   const uint32_t sm_k = smem_u32(smem + L::kK), sm_v = smem_u32(smem + L::kV);
   const uint32_t sm_q = smem_u32(smem + L::kQ), sm_do = smem_u32(smem + L::kDO);
@@ -223,15 +231,15 @@ __global__ void __launch_bounds__(kWThreads, 1)
       int issued = 0;
       for (int it = 0; it < nq; ++it) {
         const int s = it % S;
-        const int qrow = (q_first + it) * 64;
+        const int qrow = (q_first + it) * QT;
         if (it >= S && !mbar_wait(&b_empty[s], ((it / S) - 1) & 1, abort_flag, p.err)) break;
-        mbar_expect_tx(&b_full[s], 2 * L::kQS + 512);
+        mbar_expect_tx(&b_full[s], 2 * L::kQS + L::kVecStage);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem + L::kQ + s * L::kQS + c * kBox64, &tmQ, c * 64, su.q0 + qrow, su.g, &b_full[s]);
-          tma_load_3d(smem + L::kDO + s * L::kQS + c * kBox64, &tmDO, c * 64, su.q0 + qrow, su.g, &b_full[s]);
+          tma_load_3d(smem + L::kQ + s * L::kQS + c * L::kBoxQ, &tmQ, c * 64, su.q0 + qrow, su.g, &b_full[s]);
+          tma_load_3d(smem + L::kDO + s * L::kQS + c * L::kBoxQ, &tmDO, c * 64, su.q0 + qrow, su.g, &b_full[s]);
         }
-        bulk_load_1d(smem + L::kVec + s * 512, p.lse2 + vrow0 + qrow, 256, &b_full[s]);
-        bulk_load_1d(smem + L::kVec + s * 512 + 256, p.Dvec + vrow0 + qrow, 256, &b_full[s]);
+        bulk_load_1d(smem + L::kVec + s * L::kVecStage, p.lse2 + vrow0 + qrow, QT * 4, &b_full[s]);
+        bulk_load_1d(smem + L::kVec + s * L::kVecStage + QT * 4, p.Dvec + vrow0 + qrow, QT * 4, &b_full[s]);
         issued = it + 1;
       }
       if (*abort_flag) {
@@ -249,16 +257,16 @@ __global__ void __launch_bounds__(kWThreads, 1)
       const uint64_t dk_k = sdesc_sw128(sm_k, 16, 1024), dk_v = sdesc_sw128(sm_v, 16, 1024);
       const uint64_t dk_q = sdesc_sw128(sm_q, 16, 1024), dk_do = sdesc_sw128(sm_do, 16, 1024);
       const uint64_t dk_ds = sdesc_sw128(sm_ds, 16, 1024);
-      const uint64_t dmn_q = sdesc_sw128(sm_q, kBox64, 1024), dmn_do = sdesc_sw128(sm_do, kBox64, 1024);
-      const uint32_t col_off = hc * (NC / 64) * kBox64;  // this CTA's output columns
+      const uint64_t dmn_q = sdesc_sw128(sm_q, L::kBoxQ, 1024), dmn_do = sdesc_sw128(sm_do, L::kBoxQ, 1024);
+      const uint32_t col_off = hc * (NC / 64) * L::kBoxQ;  // this CTA's output columns
       // every lane waits; the vote keeps the warp's decision uniform
 #define FA_WAIT(b, parity) __all_sync(0xffffffffu, mbar_wait((b), (parity), abort_flag, p.err))
       bool ok = FA_WAIT(b_kv, 0) && FA_WAIT(&b_full[0], 0);
       if (ok) {
         tc_fence_after();
-        mma_rows128_x_rows64<D, F16>(leader, tmem + kColS, dk_k, dk_q);
+        mma_rows128_x_rows64<D, F16, QT>(leader, tmem + kColS, dk_k, dk_q);
         if (leader) mma_commit(b_s);
-        mma_rows128_x_rows64<D, F16>(leader, tmem + kColDP, dk_v, dk_do);
+        mma_rows128_x_rows64<D, F16, QT>(leader, tmem + kColDP, dk_v, dk_do);
         if (leader) mma_commit(b_dp);
       }
       for (int it = 0; ok && it < nq; ++it) {
@@ -266,8 +274,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
         if (!FA_WAIT(b_p, it & 1)) { ok = false; break; }
         tc_fence_after();
         // dV += P^T dO (this CTA's columns)
-        mma_tmemA_x_rows64<NC, F16>(leader, tmem + kColDV, tmem + kColS, desc_off(dmn_do, s * L::kQS + col_off),
-                                    it > 0);
+        mma_tmemA_x_rows64<NC, F16, QT>(leader, tmem + kColDV, tmem + kColS,
+                                        desc_off(dmn_do, s * L::kQS + col_off), it > 0);
         if (!FA_WAIT(b_ds, it & 1)) { ok = false; break; }
         tc_fence_after();
         // dK += dS^T Q : A = dS^T (128 keys x 64 queries, K-major), B = Q columns (MN-major)
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
           constexpr uint32_t idesc = idesc_f32acc(128, NC, false, true, F16);
           if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+            for (int kk = 0; kk < QT / 16; ++kk)
               mma_ss(tmem + kColDK, desc_off(dk_ds, kk * 32), desc_off(dmn_q, s * L::kQS + col_off + kk * 2048),
                      idesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
@@ -288,9 +296,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
           const int s1 = (it + 1) % S;
           if (!FA_WAIT(&b_full[s1], ((it + 1) / S) & 1)) { ok = false; break; }
           tc_fence_after();
-          mma_rows128_x_rows64<D, F16>(leader, tmem + kColS, dk_k, desc_off(dk_q, s1 * L::kQS));
+          mma_rows128_x_rows64<D, F16, QT>(leader, tmem + kColS, dk_k, desc_off(dk_q, s1 * L::kQS));
           if (leader) mma_commit(b_s);
-          mma_rows128_x_rows64<D, F16>(leader, tmem + kColDP, dk_v, desc_off(dk_do, s1 * L::kQS));
+          mma_rows128_x_rows64<D, F16, QT>(leader, tmem + kColDP, dk_v, desc_off(dk_do, s1 * L::kQS));
           if (leader) mma_commit(b_dp);
         }
       }
@@ -316,37 +324,39 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const PhiloxFixed023 phx = philox_fix023(static_cast<uint32_t>((kj * 128 + r) >> 3), static_cast<uint32_t>(su.h),
                                            static_cast<uint32_t>(su.b), p.philox_rk);
   const uint32_t ds_row = sm_ds + r * 128;
-  // query i = qt * 64 + c sees key j = kj * 128 + r iff i + delta >= j
+  // query i = qt * QT + c sees key j = kj * 128 + r iff i + delta >= j
   const int lo0 = CAUSAL ? kj * 128 + r - delta : -(1 << 30);
   const bool tile_past_keys = kj * 128 + 128 > su.nk;
   bool ok = true;
   for (int it = 0; it < nq; ++it) {
     const int s = it % S;
     const int qt = q_first + it;
-    uint32_t zb[2] = {0u, 0u};
+    uint32_t zb[QT / 32];
+#pragma unroll
+    for (int w = 0; w < QT / 32; ++w) zb[w] = 0u;
     if (DROPOUT) {
-      const uint32_t q0 = static_cast<uint32_t>(qt * 64);
+      const uint32_t q0 = static_cast<uint32_t>(qt * QT);
       if (hi_t)
-        keep_bits<true, 2>(phx, q0, p.philox_rk, dk.c2, lane, zb);
+        keep_bits<true, QT / 32>(phx, q0, p.philox_rk, dk.c2, lane, zb);
       else
-        keep_bits<false, 2>(phx, q0, p.philox_rk, dk.c2, lane, zb);
+        keep_bits<false, QT / 32>(phx, q0, p.philox_rk, dk.c2, lane, zb);
     }
     if (!mbar_wait(&b_full[s], (it / S) & 1, abort_flag, p.err) || !mbar_wait(b_s, it & 1, abort_flag, p.err)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    uint32_t sr[64];
-    tmem_ld32(t_row + kColS, sr);
-    tmem_ld32(t_row + kColS + 32, sr + 32);
-    tmem_ld_wait();
-    reg_fence32(sr);
-    reg_fence32(sr + 32);
-    const float* lse2 = reinterpret_cast<const float*>(smem + L::kVec + s * 512);
-    const float* dvec = lse2 + 64;
-    float P[64];
+    uint32_t sr[QT];
 #pragma unroll
-    for (int c4 = 0; c4 < 16; ++c4) {
+    for (int c = 0; c < QT / 32; ++c) tmem_ld32(t_row + kColS + 32 * c, sr + 32 * c);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < QT / 32; ++c) reg_fence32(sr + 32 * c);
+    const float* lse2 = reinterpret_cast<const float*>(smem + L::kVec + s * L::kVecStage);
+    const float* dvec = lse2 + QT;
+    float P[QT];
+#pragma unroll
+    for (int c4 = 0; c4 < QT / 4; ++c4) {
       const float4 l4 = *reinterpret_cast<const float4*>(lse2 + 4 * c4);
       P[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 0]), sl2, -l4.x));
       P[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(sr[4 * c4 + 1]), sl2, -l4.y));
@@ -356,39 +366,42 @@ __global__ void __launch_bounds__(kWThreads, 1)
     {
       // masked: query columns before this key's position (causal), every column
       // for a key past the unit's keys; queries past the unit have LSE2 = +inf
-      const int lo = key_valid ? lo0 - qt * 64 : 64;
+      const int lo = key_valid ? lo0 - qt * QT : QT;
       if ((CAUSAL && lo > 0) || tile_past_keys) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
+        for (int c = 0; c < QT; ++c)
           if (c < lo) P[c] = 0.f;
       }
     }
     if (DROPOUT) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half)
+      for (int half = 0; half < QT / 32; ++half)
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) mark_dropped4(P + 32 * half + 4 * k4, zb[half] >> (4 * k4));
     }
-    uint32_t pk[32];
+    uint32_t pk[QT / 2];
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
+    for (int c = 0; c < QT / 2; ++c)
       pk[c] = DROPOUT ? pack2_relu<F16>(P[2 * c], P[2 * c + 1]) : pack2<F16>(P[2 * c], P[2 * c + 1]);
-    tmem_st32(t_row + kColS, pk);
+    if constexpr (QT == 64)
+      tmem_st32(t_row + kColS, pk);
+    else
+      tmem_st16(t_row + kColS, pk);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(b_p);
     if (!mbar_wait(b_dp, it & 1, abort_flag, p.err)) { ok = false; break; }
     tc_fence_after();
-    uint32_t dr[64];
-    tmem_ld32(t_row + kColDP, dr);
-    tmem_ld32(t_row + kColDP + 32, dr + 32);
-    tmem_ld_wait();
-    reg_fence32(dr);
-    reg_fence32(dr + 32);
-    uint32_t dsk[32];
+    uint32_t dr[QT];
 #pragma unroll
-    for (int c4 = 0; c4 < 16; ++c4) {
+    for (int c = 0; c < QT / 32; ++c) tmem_ld32(t_row + kColDP + 32 * c, dr + 32 * c);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < QT / 32; ++c) reg_fence32(dr + 32 * c);
+    uint32_t dsk[QT / 2];
+#pragma unroll
+    for (int c4 = 0; c4 < QT / 4; ++c4) {
       const float4 d4 = *reinterpret_cast<const float4*>(dvec + 4 * c4);
       const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
       float v[4];
@@ -402,8 +415,9 @@ __global__ void __launch_bounds__(kWThreads, 1)
       dsk[2 * c4 + 1] = pack2<F16>(v[2], v[3]);
     }
     if (it > 0 && !mbar_wait(b_dsfree, (it - 1) & 1, abort_flag, p.err)) { ok = false; break; }
+    // dS^T rows of QT queries (QT * 2 bytes of each 128-byte swizzled row)
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
+    for (int ch = 0; ch < QT / 8; ++ch)
       st_shared_v4(ds_row + ((ch ^ (r & 7)) << 4), dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
     fence_proxy_async_smem();
     tc_fence_before();
@@ -756,6 +770,8 @@ cudaError_t launch_wide_bwd_d(const BwdArgs& a, const CUtensorMap* mkv, const CU
 
 // maps_kv: Q, K, V, dO with 64-, 128-, 128-, 64-row boxes (kernel 1);
 // maps_q: Q, K, V, dO with 128-, 64-, 64-, 128-row boxes (kernel 2).
+int wide_kv_query_rows(int d) { return d > 192 ? KvSmem<256>::kQT : KvSmem<192>::kQT; }
+
 cudaError_t launch_bwd_wide(const BwdArgs& a, const CUtensorMap* maps_kv, const CUtensorMap* maps_q,
                             cudaStream_t stream) {
   if (a.d == 192)

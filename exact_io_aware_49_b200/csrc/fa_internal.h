@@ -156,9 +156,10 @@ cudaError_t launch_bwd_prepare(const BwdArgs& a, cudaStream_t stream);  // O, dO
 cudaError_t launch_bwd_tiles(const BwdArgs& a, cudaStream_t stream);    // maps, lse2, Dvec -> dK, dV, dQacc
 cudaError_t launch_bwd_finish(const BwdArgs& a, cudaStream_t stream);   // dQacc -> dQ
 // Head dimensions 192 and 256 (fa_bwd_wide.cu): maps_kv = Q, K, V, dO tensor
-// maps with 64-, 128-, 128-, 64-row boxes; maps_q = the same with 128-, 64-,
-// 64-, 128-row boxes.  Reads Dvec and lse2 (launch_bwd_prepare), writes dQ,
-// dK, dV.
+// maps with wide_kv_query_rows(d)-, 128-, 128-, wide_kv_query_rows(d)-row
+// boxes; maps_q = the same with 128-, 64-, 64-, 128-row boxes.  Reads Dvec and
+// lse2 (launch_bwd_prepare), writes dQ, dK, dV.
+int wide_kv_query_rows(int d);
 cudaError_t launch_bwd_wide(const BwdArgs& a, const CUtensorMap* maps_kv, const CUtensorMap* maps_q,
                             cudaStream_t stream);
 cudaError_t launch_wait_timeout_probe(unsigned* err, unsigned long long limit_ns, cudaStream_t stream);
