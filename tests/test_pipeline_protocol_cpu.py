@@ -7,7 +7,8 @@ kernel (fa_bwd.cu: K/V once, Q and dO rings of two stages, the dQ drain
 staged through the tile's dO buffer) and the paged decode kernel
 (fa_decode.cu: S^T double buffer issued a tile ahead, P and its products
 doubled by tile parity, stages refilled after their P V product, the tail
-tile's V rows zeroed by the softmax warps) are restated as roles that step
+tile's V rows zeroed by the softmax warps) and the wide forward's keep-word
+ring (fa_fwd_wide.cu with dropout) are restated as roles that step
 through their waits, arrivals and tensor-core operations: a TMA producer
 whose copies complete in any order, an MMA issuer whose operations and
 commits complete asynchronously but in issue order, and the softmax /
@@ -560,6 +561,63 @@ def test_decode_protocol():
             for _ in range(40):
                 errors = Decode(rng, n, S, rng.random() < 0.5, rng.choice([0.0, 0.5, 1.0])).check()
                 assert not errors, (S, n, errors[:2])
+
+
+class KeepRing(Protocol):
+    """The keep-word ring of fa_fwd_wide.cu (dropout): four keep-word warps
+    each write their 32 rows' words of tile t into buffer t & 1 once the four
+    softmax warps have released the buffer's tile t - 2 (keep_empty, four
+    arrivals), then arrive on keep_full (four arrivals); softmax warp c waits
+    for keep_full of tile t, reads its rows (written by keep-word warp c) and
+    arrives on keep_empty."""
+
+    def __init__(self, rng, nt, slip=None):
+        super().__init__(rng)
+        self.nt, self.slip = nt, slip
+        self.full = [Bar(f"keep_full{b}", 4) for b in range(2)]
+        self.empty = [Bar(f"keep_empty{b}", 4) for b in range(2)]
+        self.rows = [[None] * 4 for _ in range(2)]      # tile held by each warp's rows of a buffer
+        self.unread = [set(), set()]                     # softmax warps that have not read the buffer's tile
+
+    def producer(self, w):
+        for t in range(self.nt):
+            b = t & 1
+            if t >= 2 and self.slip != "no_empty_wait":
+                yield ("wait", self.empty[b], (t - 2) >> 1)
+            yield None  # the Philox draw
+            if self.rows[b][w] is not None and self.unread[b]:
+                self.errors.append(f"keep warp {w} wrote tile {t} over tile {self.rows[b][w]} "
+                                   f"not yet read by {sorted(self.unread[b])}")
+            self.rows[b][w] = t
+            if all(x == t for x in self.rows[b]):
+                self.unread[b] = {0, 1, 2, 3}
+            self.full[b].arrive()
+
+    def softmax(self, c):
+        for t in range(self.nt):
+            b = t & 1
+            yield ("wait", self.full[b], t >> 1)
+            if self.rows[b][c] != t:
+                self.errors.append(f"softmax warp {c} read tile {self.rows[b][c]} for tile {t}")
+            self.unread[b].discard(c)
+            yield None
+            self.empty[b].arrive()
+
+    def check(self):
+        self.run([self.producer(w) for w in range(4)] + [self.softmax(c) for c in range(4)])
+        return self.errors
+
+
+@pytest.mark.parametrize("nt", [1, 2, 3, 9])
+def test_wide_forward_keep_ring(nt):
+    rng = random.Random(nt)
+    for _ in range(200):
+        assert KeepRing(rng, nt).check() == []
+
+
+def test_wide_forward_keep_ring_slip_is_caught():
+    rng = random.Random(7)
+    assert any(KeepRing(rng, 6, slip="no_empty_wait").check() for _ in range(100))
 
 
 @pytest.mark.parametrize("slip", ["no_refill_wait", "single_p_ready"])
