@@ -460,7 +460,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         const uint64_t negm2 = f2_pack(-m_use, -m_use);
         uint32_t pk[64];
+        // the exponent arguments, row sums and keep products in packed f32x2
+        // operations, or (d = 128 with dropout) as pairs of scalar ones: the
+        // same per-lane arithmetic, fewer registers next to the keep words
+        constexpr bool kScalarFp = (D == 128) && DROPOUT;
         uint64_t rs0 = 0ull, rs1 = 0ull;
+        float r0a = 0.f, r0b = 0.f, r1a = 0.f, r1b = 0.f;
         // the other calls inside the exponential loop, 4 at a time, 32 keys
         // ahead of the pairs that use them (chunk k = pairs 16k .. 16k + 15)
         uint32_t wn[4][4], wc[4][4];
@@ -482,14 +487,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           const float sv0 = s[2 * c], sv1 = s[2 * c + 1];
           float x0, x1;
-          f2_unpack(fma_f2(f2_pack(sv0, sv1), sl2x2, negm2), x0, x1);
+          if constexpr (kScalarFp) {
+            x0 = fmaf(sv0, sl2, -m_use);
+            x1 = fmaf(sv1, sl2, -m_use);
+          } else {
+            f2_unpack(fma_f2(f2_pack(sv0, sv1), sl2x2, negm2), x0, x1);
+          }
           const float p0 = ex2_approx(x0);
           const float p1 = ex2_approx(x1);
           const uint64_t pp = f2_pack(p0, p1);
-          if (c & 1)
+          if constexpr (kScalarFp) {
+            if (c & 1) {
+              r1a += p0;
+              r1b += p1;
+            } else {
+              r0a += p0;
+              r0b += p1;
+            }
+          } else if (c & 1) {
             rs1 = add_f2(rs1, pp);
-          else
+          } else {
             rs0 = add_f2(rs0, pp);
+          }
           if (DROPOUT && c < 4 * kPre) {
             // keys of the calls drawn before S: the byte signs of kz spread
             // over 16-bit lanes (PRMT sign mode) zero the dropped P
@@ -505,7 +524,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             asm("add.rn.sat.f32 %0, %1, %2;" : "=f"(k1) : "f"(__uint_as_float(prmt(wv, 0x4B000000u, 0x7632u))),
                 "f"(drop_bias));
             float q0, q1;
-            f2_unpack(mul_f2(pp, f2_pack(k0, k1)), q0, q1);
+            if constexpr (kScalarFp) {
+              q0 = p0 * k0;
+              q1 = p1 * k1;
+            } else {
+              f2_unpack(mul_f2(pp, f2_pack(k0, k1)), q0, q1);
+            }
             pk[c] = pack2<F16>(q0, q1);
           } else {
             pk[c] = pack2<F16>(p0, p1);
@@ -514,7 +538,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         {
           float a0, a1;
-          f2_unpack(add_f2(rs0, rs1), a0, a1);
+          if constexpr (kScalarFp) {
+            a0 = r0a + r1a;
+            a1 = r0b + r1b;
+          } else {
+            f2_unpack(add_f2(rs0, rs1), a0, a1);
+          }
           l += a0 + a1;
         }
 
