@@ -52,7 +52,7 @@ extern "C" fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V,
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
   if (!isfinite(scale) || !(scale > 0.0f)) return FA_ERR_INVALID_ARG;
-  if (d != 32 && d != 64 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 32 && d != 64 && d != 96 && d != 128 && d != 192 && d != 256) return FA_ERR_UNSUPPORTED;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (need == 0) return FA_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(FA_NOALLOC_SCRATCH_BYTES)) return FA_ERR_UNSUPPORTED;
@@ -60,7 +60,8 @@ extern "C" fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V,
   void* scratch = scratch_address();
   if (!scratch) return FA_ERR_CUDA;
   // The prepare stage rewrites every scratch word this call reads (it zeroes the
-  // dQ accumulator and writes D and LSE2 for all B*H*N rows), so whatever an
-  // earlier call left in the array does not matter.
+  // dQ accumulator and writes D and LSE2 for all B*H*N rows; the d = 192 / 256
+  // kernels read only D and LSE2), so whatever an earlier call left in the
+  // array does not matter.
   return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, p_drop, seed, scratch, need, stream);
 }

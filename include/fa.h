@@ -323,8 +323,8 @@ fa_status fa_fwd_bwd_host(const void* Q, const void* K, const void* V, const voi
  *   - Limit: fa_bwd_workspace_size(B, H, N, d) must not exceed
  *     FA_NOALLOC_SCRATCH_BYTES; larger problems return FA_ERR_UNSUPPORTED
  *     (use fa_bwd with a caller-provided workspace); for N a multiple of
- *     128 that allows B*H*N <= 64512 rows at d = 128 and <= 126976 at
- *     d = 64.
+ *     128 that allows B*H*N <= 64512 rows at d = 128, <= 126976 at d = 64,
+ *     <= 43136 at d = 192 and <= 32512 at d = 256.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.  It calls no allocating routine.

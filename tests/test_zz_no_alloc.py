@@ -3,10 +3,10 @@
 Those callers (a plugin whose host framework owns every device allocation, a
 latency-critical loop, a fixed memory budget) get the backward's scratch from
 a fixed array in the library's static device memory instead of a workspace
-argument.  This test calls the entry point through the C ABI twice in a row on
-two problems of different size and head dimension -- the second call finds
-the first call's data, laid out for another shape, still in the shared array
--- and checks both results:
+argument.  This test calls the entry point through the C ABI three times in a
+row on problems of different size and head dimension (d = 128, 64, and 192 on
+the wide-head kernels) -- each call finds the previous call's data, laid out
+for another shape, still in the shared array -- and checks every result:
 
 * against fa_bwd with a caller-provided workspace: dK and dV bit for bit (the
   same kernels accumulate them in a fixed order), dQ within one bf16 rounding
@@ -59,11 +59,12 @@ def _one_rounding_step(got, want):
     return bool(((g - w).abs() <= step + 2.0 ** -20 * w.abs().max()).all())
 
 
-def test_noalloc_two_calls_in_a_row_match_fa_bwd_and_the_oracle():
+def test_noalloc_calls_in_a_row_match_fa_bwd_and_the_oracle():
     from exact_io_aware_49_b200 import fa_bwd, fa_fwd, fa_last_device_error
     lib = _lib()
     problems = [wl.Workload("noalloc_a", 1, 4, 1024, 128, True, 0.1, 11),
-                wl.Workload("noalloc_b", 2, 3, 768, 64, False, 0.0, 12)]
+                wl.Workload("noalloc_b", 2, 3, 768, 64, False, 0.0, 12),
+                wl.Workload("noalloc_c", 1, 2, 640, 192, True, 0.1, 13)]
     cases = []
     for w in problems:
         host = wl.draw_inputs(w)
