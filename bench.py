@@ -19,13 +19,17 @@ FLOPs per step: forward 4*B*H*N^2*d/2 (causal), backward 2.5x the forward.
   roofline  the kernel with the largest share of the step, achieved TFLOP/s
             from its own CUDA events against the measured bf16 burst peak
   other_workloads  fa_fwd and the backward on B=4 H=16 N=4096 d=128 causal
-            p=0.1 (the other dropout workload), each call timed with CUDA
-            events (median), TFLOP/s and % of the burst peak
+            p=0.1 (the other dropout workload) and on the wide head dims
+            (B=2 H=16 N=8192 d=192 and d=256, causal, p=0.1), each call timed
+            with CUDA events (median), TFLOP/s and % of the burst peak
   cpu_baseline  the fp64 oracle on this host's cores on a bounded sample
             (a causal prefix of one head, which is itself a complete causal
             attention problem)
 
 ``--impl reference`` times that oracle instead (rank 0 only).
+
+``--other-workloads-only`` prints just those per-call timings (a short run,
+also the command the wide kernels' ncu capture profiles).
 
 ``--decode`` prints a different line instead: the paged-cache decode kernel
 (fa_decode_paged) on 16 sequences x 32768 cached positions, 32 query / 8
@@ -350,10 +354,26 @@ def run_ours(args, w, world, device):
         "clocks": clocks,
     }
     if w.name == WORKLOAD and not args.no_other_workloads:
-        # the other d = 128 causal dropout workload the throughput target names
-        other = wl.BY_NAME["causal_dropout_N4096_d128"]
-        out["other_workloads"] = {other.name: time_other_workload(other, device, peaks)}
+        out["other_workloads"] = time_other_workloads(device, peaks)
     return out, (qh, kh, vh, doh)
+
+
+# the other d = 128 causal dropout workload the throughput target names, then
+# the head dims the d <= 128 kernels cannot hold (their own kernels, seeded as
+# the recipe of exact_io_aware_49_b200.workloads draws every input)
+OTHER_WORKLOADS = [
+    "causal_dropout_N4096_d128",
+    wl.Workload("causal_dropout_N8192_d192", 2, 16, 8192, 192, True, 0.1, 21),
+    wl.Workload("causal_dropout_N8192_d256", 2, 16, 8192, 256, True, 0.1, 22),
+]
+
+
+def time_other_workloads(device, peaks):
+    out = {}
+    for o in OTHER_WORKLOADS:
+        w = wl.BY_NAME[o] if isinstance(o, str) else o
+        out[w.name] = time_other_workload(w, device, peaks)
+    return out
 
 
 def time_other_workload(w, device, peaks, reps=20, warmup=3):
@@ -367,14 +387,16 @@ def time_other_workload(w, device, peaks, reps=20, warmup=3):
     lse = torch.empty((w.B, w.H, w.N), device=device, dtype=torch.float32)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     ws = torch.empty(binding.fa_bwd_workspace_size(w.B, w.H, w.N, w.d), device=device, dtype=torch.uint8)
+    # d <= 128: the three stages (prepare, tiles, finish); wider heads: fa_bwd,
+    # whose dK / dV and dQ kernels write the gradients directly
+    stages = binding.fa_bwd_stages if w.d <= 128 else binding.fa_bwd
     tf, tb = [], []
     for it in range(warmup + reps):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record(stream)
         binding.fa_fwd(q, k, v, w.causal, w.scale, w.p_drop, w.seed, out=o, lse=lse)
         e[1].record(stream)
-        binding.fa_bwd_stages(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, workspace=ws, dq=dq,
-                              dk=dk, dv=dv)
+        stages(q, k, v, o, do, lse, w.causal, w.scale, w.p_drop, w.seed, workspace=ws, dq=dq, dk=dk, dv=dv)
         e[2].record(stream)
         torch.cuda.synchronize(device)
         if it >= warmup:
@@ -388,7 +410,7 @@ def time_other_workload(w, device, peaks, reps=20, warmup=3):
             "fwd_pct_of_burst": 100 * fwd_tf / peaks["bf16_tflops"],
             "bwd_pct_of_burst": 100 * bwd_tf / peaks["bf16_tflops"],
             "timing": f"CUDA events per call, median of {reps} after {warmup} warm-up calls; "
-                      "inputs (Q, K, V, dO 67 MB each) are resident, no L2 flush"}
+                      f"inputs (Q, K, V, dO {q.numel() * 2 / 1e6:.0f} MB each) are resident, no L2 flush"}
 
 
 # --------------------------------------------------------------------- decode line
@@ -527,13 +549,20 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(wl.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-workloads", action="store_true",
-                    help="skip the per-call timing of the N=4096 dropout workload beside the main line")
+                    help="skip the per-call timings of the other workloads beside the main line")
     ap.add_argument("--decode", action="store_true", help="the paged-cache decode line instead (one GPU)")
+    ap.add_argument("--other-workloads-only", action="store_true",
+                    help="only the per-call timings of the other workloads (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.decode:
         print(json.dumps(run_decode(args, torch.device("cuda", 0))), flush=True)
+        return
+    if args.other_workloads_only:
+        peaks, peak_src = _peaks()
+        res = {"other_workloads": time_other_workloads(torch.device("cuda", 0), peaks), "peak_source": peak_src}
+        print(json.dumps(res), flush=True)
         return
     w = wl.BY_NAME[args.workload]
     world = _world()

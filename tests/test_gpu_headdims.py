@@ -178,6 +178,7 @@ def test_wide_forward_mask_and_guard_bands(d):
     (1, 1, 333, 333, True, 0.7, False, torch.float16),     # threshold above 0x8000
     (1, 2, 200, 700, True, 0.1, True, torch.bfloat16),     # Nq < Nk (deterministic is the only dQ order here)
     (1, 1, 700, 200, True, 0.0, False, torch.bfloat16),    # Nq > Nk: leading rows see no key
+    (1, 2, 384, 384, False, 0.1, False, torch.bfloat16),   # non-causal with dropout
 ])
 def test_wide_backward(d, B, H, Nq, Nk, causal, p, det, dtype):
     """The wide-head backward (a dK / dV kernel over 64-query tiles and a dQ
