@@ -1,6 +1,7 @@
 """Host-side checks of bench.py's bookkeeping (no GPU): recorded DRAM traffic is
-matched to kernel code, not to comments, and every record in the committed
-profile file is found for the current sources."""
+matched to kernel code, not to comments, every record in the committed
+profile file is found for the current sources, and the side workloads timed
+beside the main line are the ones their names say."""
 
 import os
 import sys
@@ -42,3 +43,15 @@ def test_peaks_come_from_the_measured_file_when_present():
     if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
         assert src == "measured"
     assert peaks["hbm_gbs"] > 1000 and peaks["bf16_tflops"] > 500
+
+
+def test_side_workloads_are_named_by_their_shapes():
+    """The per-call timings beside the main line cover the other d = 128
+    dropout workload and both wide head dims, each named by its shape."""
+    from exact_io_aware_49_b200 import workloads as wl
+    ws = [wl.BY_NAME[o] if isinstance(o, str) else o for o in bench.OTHER_WORKLOADS]
+    for w in ws:
+        assert w.name == f"causal_dropout_N{w.N}_d{w.d}", w.name
+        assert w.causal and w.p_drop == 0.1 and w.backward
+    assert sorted(w.d for w in ws) == [128, 192, 256]
+    assert len({w.seed for w in ws}) == len(ws)
