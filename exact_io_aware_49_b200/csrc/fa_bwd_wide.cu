@@ -126,6 +126,8 @@ struct KvSmem {
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;
 };
+static_assert(KvSmem<192>::kBytes <= kMaxSmemPerCta && KvSmem<256>::kBytes <= kMaxSmemPerCta,
+              "dK / dV kernel shared memory");
 
 template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kWThreads, 1)
@@ -471,6 +473,8 @@ struct QSmem {
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;
 };
+static_assert(QSmem<192>::kBytes <= kMaxSmemPerCta && QSmem<256>::kBytes <= kMaxSmemPerCta,
+              "dQ kernel shared memory");
 
 template <int D, bool CAUSAL, bool DROPOUT, bool F16>
 __global__ void __launch_bounds__(kWThreads, 1)

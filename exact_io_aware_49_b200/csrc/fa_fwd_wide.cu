@@ -66,6 +66,8 @@ struct WideSmem {
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;  // + slack for 1024-byte alignment
 };
+static_assert(WideSmem<192>::kBytes <= kMaxSmemPerCta && WideSmem<256>::kBytes <= kMaxSmemPerCta,
+              "wide forward shared memory");
 
 struct WideBars {
   uint64_t *q, *kfull, *kempty, *vfull, *vempty, *s_full, *p_ready, *pv_done, *o_ready, *drain, *keep_full,

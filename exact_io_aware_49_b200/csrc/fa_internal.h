@@ -8,6 +8,12 @@
 
 namespace fa {
 
+// Largest dynamic shared memory one CTA can opt into on sm_100 (227 KB); the
+// wide-head kernels' layouts are checked against it at compile time (for the
+// d <= 128 kernels, setting a size above the device's opt-in limit makes the
+// launch return an error).
+constexpr int kMaxSmemPerCta = 227 * 1024;
+
 // Where the rows of one (sequence, head) unit live.  Units are numbered
 // b * H + h; a launch processes ``units`` of them starting at ``unit0`` (a
 // fixed-length problem split into groups of heads: the tensors then hold only
