@@ -234,3 +234,18 @@ def test_decode_split_choice_and_workspace(lib):
         per = (tiles + s - 1) // s
         assert (tiles + per - 1) // per == s, (B, H_kv, H, Nq, L, s)
     assert lib.fa_decode_workspace_size(2, 8, 1, 128, 4) == 2 * 8 * 4 * 128 * 4 + 256
+
+
+@pytest.mark.parametrize("d", [32, 80, 128, 192, 256, 320])
+def test_noalloc_takes_the_head_dims_fa_bwd_takes(lib, d):
+    """With null pointers both backward entry points return the same status
+    for every head dim: FA_ERR_INVALID_ARG where d is supported (the wide
+    heads included), FA_ERR_UNSUPPORTED where it is not; both before any
+    CUDA call."""
+    vp, i, fl, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_uint64
+    f = lib.fa_bwd_noalloc
+    f.argtypes = [vp] * 9 + [i, i, i, i, i, fl, fl, u64, vp]
+    f.restype = i
+    got = f(*([None] * 9), 1, 1, 256, d, 1, 0.1, 0.0, 0, None)
+    want = lib.fa_bwd(*([None] * 9), 1, 1, 256, d, 1, 0.1, 0.0, 0, None, 0, None)
+    assert got == want == (1 if d in (32, 128, 192, 256) else 2)
