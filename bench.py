@@ -353,7 +353,8 @@ def run_ours(args, w, world, device):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
-    if w.name == WORKLOAD and not args.no_other_workloads:
+    if w.name == WORKLOAD and not args.no_other_workloads and world["rank"] == 0:
+        # after the last collective; only rank 0's line carries them
         out["other_workloads"] = time_other_workloads(device, peaks)
     return out, (qh, kh, vh, doh)
 
